@@ -1,0 +1,401 @@
+"""Benchmark of the capacity-limited, pooled-wave MoE block on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload train|full|mid|skewed]
+                    [--impl ours|reference]
+
+A step is one pass of the whole hot path on one batch: forward (latent down-projection,
+router, top-k, slot assignment, pack, unpack, grouped SwiGLU experts, combine, shared
+experts, up-projection), backward (every dgrad and wgrad, combine backward,
+un-dispatch, router backward) and the bias step.  The default workload is the
+full-width training layer (T=16384, d_model 6144, latent 3072, 384 experts, top-8,
+64 destinations x 3 waves, 2 shared experts of 3072).
+
+Prints one JSON line on rank 0.  For N > 1 (torchrun) every rank runs its own
+source of T tokens (data-parallel replicas, weak scaling); the only exchange is the
+all-reduce of the load histogram before the bias step, which keeps the bias the
+same on every replica.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-block tokens/s fwd & fwd+bwd on 1 B200; GEMM % BF16 peak; dispatch % HBM BW"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "_source": "fallback"}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["_source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+def workload_shape(name):
+    from capacity_limited_routed_b200 import synth
+    return {"train": synth.TRAIN, "full": synth.FULL, "mid": synth.MID, "skewed": synth.SKEWED,
+            "tiny": synth.TINY.with_(backward=True)}[name]
+
+
+def describe(s):
+    return (f"{s.name}: MoE block {'fwd+bwd+bias step' if s.backward else 'forward'}, T={s.T}, "
+            f"d_model {s.d_model}, latent {s.d_latent}, E={s.n_experts} top-{s.top_k}, "
+            f"D={s.n_dest} x {s.n_waves} waves, caps {s.cap_send[0]/s.cap_send[1]:.2f}/"
+            f"{s.cap_recv[0]/s.cap_recv[1]:.2f}, {s.n_shared} shared x {s.hidden_shared}"
+            + (f", Zipf({s.zipf_s}) logit skew, rho={s.rho} windows of {s.window}" if s.zipf_s else ""))
+
+
+# ------------------------------------------------------------------ algorithmic work per step
+
+
+def step_work(s, kept):
+    """Algorithmic FLOPs (2 per multiply-add) and HBM bytes of each named step.
+
+    Routed GEMMs count kept rows only."""
+    T, dm, dl, E, k, h, SH = s.T, s.d_model, s.d_latent, s.n_experts, s.top_k, s.hidden_routed, s.n_shared * s.hidden_shared
+    f = {
+        "fwd.lat_down": 2 * T * dm * dl,
+        "fwd.router": 2 * T * dl * E,
+        "experts.gate_up": 2 * kept * dl * 2 * h,
+        "experts.down": 2 * kept * h * dl,
+        "fwd.shared_gate_up": 2 * T * dm * 2 * SH,
+        "fwd.lat_up_shared_down": 2 * T * dm * (dl + SH),
+        "bwd.dr": 2 * T * dm * dl,
+        "bwd.shared_dgrad_swiglu": 2 * T * dm * SH,
+        "bwd.wgrad_lat_up_shared_down": 2 * T * dm * (dl + SH),
+        "bwd.experts_dgrad_down": 2 * kept * dl * h,
+        "bwd.experts_wgrad_down": 2 * kept * dl * h,
+        "bwd.experts_dgrad_gate_up": 2 * kept * 2 * h * dl,
+        "bwd.experts_wgrad_gate_up": 2 * kept * 2 * h * dl,
+        "bwd.router_dgrad": 2 * T * E * dl,
+        "bwd.router_wgrad": 2 * T * E * dl,
+        "bwd.dx": 2 * T * dm * (dl + 2 * SH),
+        "bwd.wgrad_lat_down_shared": 2 * T * dm * (dl + 2 * SH),
+    }
+    A = T * k
+    b = {
+        # logits read, idx + gate written
+        "fwd.route_topk": T * E * 4 + A * 8 + E * 4,
+        # z read once, every sender-kept row written with its 16-byte header
+        "fwd.dispatch_pack": T * dl * 2 + kept * (dl * 2 + 16),
+        # pools read (kept rows + headers), expert rows written
+        "experts.unpack": kept * (dl * 2 + 16) + kept * dl * 2,
+        # expert rows read, gate + slot read, r written
+        "fwd.combine": kept * dl * 2 + A * 12 + T * dl * 2,
+        # dr read, Y read, dY written, gate/slot read
+        "bwd.combine": T * dl * 2 + 2 * kept * dl * 2 + A * 16,
+        # dX read, dz (fp32) and dlogits written
+        "bwd.undispatch": kept * dl * 2 + T * dl * 4 + T * E * 2 + A * 16,
+        "fwd.slot_scan": A * 4 * 3 + A * 8,
+    }
+    return f, b
+
+
+# ------------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    def __init__(self, gpu_index, path):
+        self.path = path
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(path, "w")
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+
+
+def oracle_sample_shape(s):
+    """A bounded sample of the workload for the CPU oracle: 256 tokens at the full widths
+    (every token still runs top-k full-width experts, the shared experts and both latent
+    projections), with 24 routed experts (4 destinations x 6) instead of 384 so the
+    weights fit the host; per-token work is the same."""
+    return s.with_(T=256, n_experts=24, n_dest=4)
+
+
+def run_oracle_sample(s, reps=1):
+    import numpy as np
+    from capacity_limited_routed_b200 import synth
+    from oracle import moe_oracle as O
+    ss = oracle_sample_shape(s).with_(backward=True)
+    inp = synth.make_inputs(ss, seed=123)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        y, ctx = O.forward(inp["x"], inp["weights"], inp["bias"], ss, logit_offset=inp["logit_offset"])
+        if s.backward:
+            O.backward(inp["dy"], inp["weights"], ctx)
+            O.bias_update(ctx["hist"], inp["bias"], 1e-3, ss.T, ss.top_k)
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    return ss.T * reps / dt, cores, ss
+
+
+def reference_arm(args, s):
+    """The oracle as it stands, timed on the host cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    steps, warm = max(1, min(args.steps, 3)), max(0, min(args.warmup, 1))
+    for _ in range(warm):
+        run_oracle_sample(s)
+    rates = []
+    for _ in range(steps):
+        r, cores, ss = run_oracle_sample(s)
+        rates.append(r)
+    v = statistics.median(rates)
+    sample = (f"per step {ss.T} tokens at full widths ({ss.d_model}/{ss.d_latent}/{ss.hidden_routed}, "
+              f"top-{ss.top_k}, {ss.n_shared} shared), {ss.n_experts} routed experts instead of "
+              f"{s.n_experts}; forward{' + backward + bias step' if s.backward else ''}")
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": steps, "warmup": warm, "ms_per_step": 1000.0 * ss.T / v, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": describe(s)},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="train")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-only", action="store_true", help="a few steps, no baseline, no e2e (for ncu)")
+    args = ap.parse_args()
+    s = workload_shape(args.workload)
+    if args.impl == "reference":
+        reference_arm(args, s)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    from capacity_limited_routed_b200 import moe as M
+    from capacity_limited_routed_b200 import synth
+    from capacity_limited_routed_b200.block import MoEBlock
+
+    peaks = load_peaks()
+    inp = synth.make_inputs_device(s, device=dev, seed=s.seed + 7919 * rank)
+    blk = MoEBlock(s, device=dev, training=s.backward)
+    blk.load(inp)
+    x, dy = inp["x"], inp.get("dy")
+    hist_plan = M.Plan.from_shape(s.with_(T=s.T * world)) if world > 1 else blk.plan
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        blk.forward(x)
+        if s.backward:
+            blk.backward(x, dy)
+            if world > 1:
+                dist.all_reduce(blk.hist())
+            M.moe_bias_update(hist_plan, blk.hist(), blk.bias, 1e-3)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    st0 = blk.stats_dict()
+    if st0["status"] != 0:
+        raise RuntimeError(f"kernel status {st0['status']} after warm-up")
+
+    # ---------------- timed region: K steps, device-resident inputs
+    clocks = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
+                          if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/clocks_rank{rank}.csv")
+    launches0 = M.moe_kernel_launches()
+    M.moe_profile_start()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    prof = M.moe_profile_stop()
+    launches = M.moe_kernel_launches() - launches0
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    st = blk.stats_dict()
+    if st["status"] != 0:
+        raise RuntimeError(f"kernel status {st['status']} in the timed region")
+
+    # per-step timing from the library's events (same stream, same timed region)
+    per = {}
+    for name, t, n in prof:
+        d = per.setdefault(name, [0.0, 0, 0])
+        d[0] += t
+        d[1] += 1
+        d[2] += n
+    kept = st["kept"]
+    flops, bytes_ = step_work(s, kept)
+    tc_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    kernels = {}
+    for name, (tot, cnt, nl) in per.items():
+        avg = tot / cnt
+        e = {"ms": round(avg, 4), "share": round(tot / sum(v[0] for v in per.values()), 4)}
+        if name in flops:
+            e["tflops"] = round(flops[name] / (avg * 1e-3) / 1e12, 1)
+            e["frac"] = round(e["tflops"] / tc_peak, 3)
+        elif name in bytes_:
+            e["gbs"] = round(bytes_[name] / (avg * 1e-3) / 1e9, 1)
+            e["frac"] = round(e["gbs"] / peaks["hbm_gbs"], 3)
+        kernels[name] = e
+    top = max(per.items(), key=lambda kv: kv[1][0])[0]
+    avg_top = per[top][0] / per[top][1]
+    if top in flops:
+        achieved = flops[top] / (avg_top * 1e-3) / 1e12
+        roof = {"kernel": top, "bound": "tensor", "achieved": round(achieved, 1), "peak": tc_peak,
+                "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 3), "traffic": None,
+                "peak_kind": f"bf16_tflops_sustained ({peaks['_source']}): kernel timed inside a long step",
+                "flops_per_launch": flops[top]}
+    else:
+        achieved = bytes_.get(top, 0) / (avg_top * 1e-3) / 1e9
+        roof = {"kernel": top, "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 3), "traffic": None}
+    fwd_ms = sum(v[0] for k_, v in per.items() if k_.startswith("fwd.") or k_.startswith("experts.")) / args.steps
+    step_ms = ms_max / args.steps
+    value = world * s.T / (step_ms * 1e-3)
+
+    # ---------------- end to end through the public API, host buffers
+    e2e = None
+    if not args.profile_only:
+        x_h = x.cpu().pin_memory()
+        dy_h = dy.cpu().pin_memory() if dy is not None else None
+        out_h = torch.empty(8, dtype=torch.int32).pin_memory()
+        xs = torch.empty_like(x)
+        dys = torch.empty_like(dy) if dy is not None else None
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            xs.copy_(x_h, non_blocking=True)
+            if s.backward:
+                dys.copy_(dy_h, non_blocking=True)
+            blk.forward(xs)
+            if s.backward:
+                blk.backward(xs, dys)
+                if world > 1:
+                    dist.all_reduce(blk.hist())
+                M.moe_bias_update(hist_plan, blk.hist(), blk.bias, 1e-3)
+            out_h.copy_(blk.stats[:8], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        e_step = float(e_ms.item()) / args.steps
+        e2e = {"value": world * s.T / (e_step * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": x.numel() * 2 + (dy.numel() * 2 if dy is not None else 0),
+               "d2h_bytes_per_step": 32, "read_back": "stats head (kept / dropped counters)"}
+
+    # ---------------- CPU oracle baseline (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile_only:
+        r, cores, ss = run_oracle_sample(s)
+        cpu = {"value": r, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{ss.T} tokens of this workload at full widths with {ss.n_experts} routed experts "
+                         f"instead of {s.n_experts} (same per-token work), one pass, float64 numpy"}
+
+    if rank == 0:
+        A = s.T * s.top_k
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": describe(s), "parallelism": f"replicas x{world} (one source per GPU)",
+                       "l2": "inputs larger than L2 (22 GB of expert weights streamed every step)"},
+            "fwd_tokens_per_s": world * s.T / (fwd_ms * 1e-3) if fwd_ms > 0 else None,
+            "drop_fraction": {"sender": st["dropped_sender"] / A, "receiver": st["dropped_receiver"] / A},
+            "roofline": roof,
+            "dispatch_hbm_frac": kernels.get("fwd.dispatch_pack", {}).get("frac"),
+            "kernels": kernels,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,660 @@
+// gemm_sm100.cu -- persistent tcgen05 GEMM for sm_100a: TMA -> shared memory -> tcgen05.mma ->
+// TMEM accumulators -> fused epilogues.
+//
+// These are the dense contractions of the MoE block: the latent down- and
+// up-projections, the router, the grouped SwiGLU experts and the shared experts,
+// with their transposed forms for the backward pass ("Marin начинает открытое
+// обучение MoE-модели с 535 млрд параметров", §2; "Marin 535B-A23B：一场完全公开的前沿
+// MoE 训练直播", §2.2).
+//
+// Structure (one CTA per SM, 192 threads):
+//   warp 0      TMA producer: A tile 128 x 64 and B tile BN x 64 per stage, 128-byte
+//               swizzle, K-major or MN-major boxes, no multicast.
+//   warp 1      allocates 2*BN TMEM columns; lane 0 issues tcgen05.mma (M=128, N=BN,
+//               K=16) and commits stage releases and accumulator hand-offs.
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (lane quarter = warp % 4),
+//               fused element-wise work, stores to global memory.
+// Two accumulators in TMEM let the epilogue of one tile overlap the main loop of
+// the next.  Tiles of all groups (experts) form one list that CTAs stride over;
+// ragged groups take their row (or K) counts from device memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace moe {
+
+struct TmaMaps {
+  CUtensorMap a[3];
+  CUtensorMap b[3];
+  CUtensorMap bv;
+};
+
+struct KParams {
+  int M, N, groups, ragged;
+  const int32_t* group_rows;
+  int nseg;
+  int seg_kb[3];
+  int m_fastest;
+  void* out;
+  long long ldo, out_gs;
+  void* out2;
+  void* save_a;
+  void* save_b;
+  const void* aux_a;
+  const void* aux_b;
+  long long aux_ld, aux_gs;
+  const float* col_add;
+  const float* addend;
+  long long add_ld;
+  int32_t* status;
+};
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kThreads = 192;
+constexpr int kMaxGroups = 1024;
+
+template <int BN>
+struct Cfg {
+  static constexpr int kABytes = kBM * kBK * 2;  // 16 KB
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStage = kABytes + kBBytes;
+  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kBarBytes = 8 * (2 * kStages + 5) + 16;
+  static constexpr int kSmem = 1024 + kStages * kStage + kBarBytes + 4 * (kMaxGroups + 1);
+};
+
+__device__ __forceinline__ void record_status(int32_t* status, int code) {
+  if (status != nullptr) atomicCAS(status, 0, code);
+}
+
+// Tile bookkeeping shared by the three roles; all of them walk the same list.
+template <int BN, int EPI>
+struct Sched {
+  const KParams& p;
+  const int* prefix;  // ragged == 1: tiles before group g (shared memory)
+  int nt, mt_fixed, tiles_per_group, total;
+
+  __device__ Sched(const KParams& pp, const int* pre) : p(pp), prefix(pre) {
+    const int out_cols = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
+    nt = (p.N + out_cols - 1) / out_cols;
+    mt_fixed = (p.M + kBM - 1) / kBM;
+    tiles_per_group = mt_fixed * nt;
+    total = (p.ragged == 1) ? prefix[p.groups] : p.groups * tiles_per_group;
+  }
+
+  __device__ void decode(int t, int& g, int& m_tile, int& n_tile) const {
+    int base, mt;
+    if (p.ragged == 1) {
+      int lo = 0, hi = p.groups;  // largest g with prefix[g] <= t
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (prefix[mid] <= t) lo = mid; else hi = mid;
+      }
+      g = lo;
+      base = prefix[g];
+      mt = (prefix[g + 1] - prefix[g]) / nt;
+    } else {
+      g = t / tiles_per_group;
+      base = g * tiles_per_group;
+      mt = mt_fixed;
+    }
+    const int local = t - base;
+    if (p.m_fastest) {
+      m_tile = local % mt;
+      n_tile = local / mt;
+    } else {
+      n_tile = local % nt;
+      m_tile = local / nt;
+    }
+  }
+
+  __device__ int k_blocks(int g) const {
+    if (p.ragged == 2) {
+      int r = p.group_rows[g];
+      r = r < 0 ? 0 : r;
+      return (r + kBK - 1) / kBK;
+    }
+    return p.seg_kb[0] + p.seg_kb[1] + p.seg_kb[2];
+  }
+};
+
+template <int BN, bool A_MN, bool B_MN, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ TmaMaps maps, const KParams p) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStage);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int* prefix = reinterpret_cast<int*>(smem + C::kStages * C::kStage + C::kBarBytes);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < p.nseg; ++s) {
+      tma_prefetch_desc(&maps.a[s]);
+      tma_prefetch_desc(&maps.b[s]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  // tiles per group and their prefix (ragged rows only)
+  if (p.ragged == 1) {
+    const int out_cols = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
+    const int nt = (p.N + out_cols - 1) / out_cols;
+    const int per = (p.groups + kThreads - 1) / kThreads;
+    const int g0 = threadIdx.x * per;
+    int local = 0;
+    for (int i = 0; i < per; ++i) {
+      const int g = g0 + i;
+      if (g < p.groups) {
+        int r = p.group_rows[g];
+        r = r < 0 ? 0 : (r > p.M ? p.M : r);
+        local += ((r + kBM - 1) / kBM) * nt;
+      }
+    }
+    // block exclusive scan of `local` over 192 threads
+    __shared__ int warp_sums[kThreads / 32];
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += warp_sums[w];
+    int run = before + incl - local;
+    for (int i = 0; i < per; ++i) {
+      const int g = g0 + i;
+      if (g < p.groups) {
+        prefix[g] = run;
+        int r = p.group_rows[g];
+        r = r < 0 ? 0 : (r > p.M ? p.M : r);
+        run += ((r + kBM - 1) / kBM) * nt;
+      }
+    }
+    if (threadIdx.x == kThreads - 1) prefix[p.groups] = before + incl;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const volatile int* abort_v = abort_flag;
+
+  Sched<BN, EPI> sc(p, prefix);
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int armed_phase[C::kStages];
+      for (int s = 0; s < C::kStages; ++s) armed_phase[s] = -1;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < sc.total; t += gridDim.x) {
+        int g, mt, ntile;
+        sc.decode(t, g, mt, ntile);
+        const int kb_total = sc.k_blocks(g);
+        for (int kb = 0; kb < kb_total; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_v)) {
+            ok = false;
+            break;
+          }
+          int s = 0, kl = kb;
+          if (p.ragged != 2) {
+            while (s < p.nseg - 1 && kl >= p.seg_kb[s]) {
+              kl -= p.seg_kb[s];
+              ++s;
+            }
+          }
+          const int k0 = kl * kBK;
+          uint8_t* sa = smem + stage * C::kStage;
+          uint8_t* sb = sa + C::kABytes;
+          mbar_arrive_expect_tx(&full[stage], C::kStage);
+          armed_phase[stage] = static_cast<int>(phase);
+          const int m0 = mt * kBM;
+          if (!A_MN) {
+            tma_load_3d(&maps.a[s], sa, &full[stage], k0, m0, g);
+          } else {
+            tma_load_3d(&maps.a[s], sa, &full[stage], m0, k0, g);
+            tma_load_3d(&maps.a[s], sa + 8192, &full[stage], m0 + 64, k0, g);
+          }
+          if (EPI == EPI_SWIGLU) {
+            const int n0 = ntile * (BN / 2);
+            tma_load_3d(&maps.b[0], sb, &full[stage], k0, n0, g);
+            tma_load_3d(&maps.bv, sb + (BN / 2) * 128, &full[stage], k0, n0, g);
+          } else if (!B_MN) {
+            tma_load_3d(&maps.b[s], sb, &full[stage], k0, ntile * BN, g);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_3d(&maps.b[s], sb + j * 8192, &full[stage], ntile * BN + 64 * j, k0, g);
+          }
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_status(p.status, MOE_ERR_TIMEOUT);
+        // let every load already issued land before the CTA goes away
+        for (int s = 0; s < C::kStages; ++s)
+          if (armed_phase[s] >= 0) mbar_wait(&full[s], static_cast<uint32_t>(armed_phase[s]), nullptr, 50000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, A_MN, B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      bool issued = false;
+      for (int t = blockIdx.x; ok && t < sc.total; t += gridDim.x) {
+        int g, mt, ntile;
+        sc.decode(t, g, mt, ntile);
+        const int kb_total = sc.k_blocks(g);
+        if (kb_total == 0) continue;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_v)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < kb_total; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_v)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * C::kStage);
+          const uint32_t b_addr = a_addr + C::kABytes;
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t ad = A_MN ? smem_desc_sw128(a_addr + k * 2048, 8192, 1024)
+                                     : smem_desc_sw128(a_addr + k * 32, 16, 1024);
+            const uint64_t bd = B_MN ? smem_desc_sw128(b_addr + k * 2048, 8192, 1024)
+                                     : smem_desc_sw128(b_addr + k * 32, 16, 1024);
+            mma_bf16_ss(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          issued = true;
+          mma_commit(&empty[stage]);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_status(p.status, MOE_ERR_TIMEOUT);
+        if (issued) {
+          mma_commit(drain);
+          mbar_wait(drain, 0, nullptr, 50000000ull);
+        }
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row_in_tile = q * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < sc.total; t += gridDim.x) {
+      int g, mt, ntile;
+      sc.decode(t, g, mt, ntile);
+      const int kb_total = sc.k_blocks(g);
+      const int row = mt * kBM + row_in_tile;
+      const bool row_ok = row < p.M;
+      if (kb_total == 0) {
+        // an empty contraction (group with no rows): the product is zero
+        if (row_ok && (EPI == EPI_BF16 || EPI == EPI_F32)) {
+          for (int c = 0; c < BN; c += 8) {
+            const int col = ntile * BN + c;
+            if (col >= p.N) break;
+            if (EPI == EPI_BF16) {
+              uint16_t* o = static_cast<uint16_t*>(p.out) + g * p.out_gs + (long long)row * p.ldo + col;
+              *reinterpret_cast<uint4*>(o) = make_uint4(0, 0, 0, 0);
+            } else {
+              float* o = static_cast<float*>(p.out) + g * p.out_gs + (long long)row * p.ldo + col;
+              reinterpret_cast<uint4*>(o)[0] = make_uint4(0, 0, 0, 0);
+              reinterpret_cast<uint4*>(o)[1] = make_uint4(0, 0, 0, 0);
+            }
+          }
+        }
+        continue;
+      }
+      const bool got = mbar_wait(&tfull[acc], acc_phase, abort_v);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, got)) {
+        *abort_flag = 1;
+        record_status(p.status, MOE_ERR_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + lane_off + static_cast<uint32_t>(acc * BN);
+
+      if constexpr (EPI == EPI_SWIGLU) {
+        const int n_out0 = ntile * (BN / 2);
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          float gv[32], uv[32];
+          __syncwarp();
+          tmem_ld_32cols(tbase + c, gv);
+          tmem_ld_32cols(tbase + BN / 2 + c, uv);
+          const int col = n_out0 + c;
+          if (row_ok && col < p.N) {
+            const long long off = g * p.out_gs + (long long)row * p.ldo + col;
+            uint32_t h[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float a0 = gv[2 * i], a1 = gv[2 * i + 1];
+              const float s0 = a0 / (1.0f + expf(-a0)), s1 = a1 / (1.0f + expf(-a1));
+              h[i] = pack_bf16x2(s0 * uv[2 * i], s1 * uv[2 * i + 1]);
+            }
+            uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + off);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) o[v] = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+            if (p.save_a != nullptr) {
+              uint4* oa = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.save_a) + off);
+              uint4* ob = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.save_b) + off);
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                oa[v] = make_uint4(pack_bf16x2(gv[8 * v], gv[8 * v + 1]), pack_bf16x2(gv[8 * v + 2], gv[8 * v + 3]),
+                                   pack_bf16x2(gv[8 * v + 4], gv[8 * v + 5]), pack_bf16x2(gv[8 * v + 6], gv[8 * v + 7]));
+                ob[v] = make_uint4(pack_bf16x2(uv[8 * v], uv[8 * v + 1]), pack_bf16x2(uv[8 * v + 2], uv[8 * v + 3]),
+                                   pack_bf16x2(uv[8 * v + 4], uv[8 * v + 5]), pack_bf16x2(uv[8 * v + 6], uv[8 * v + 7]));
+              }
+            }
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          float v[32];
+          __syncwarp();
+          tmem_ld_32cols(tbase + c, v);
+          const int col0 = ntile * BN + c;
+          if (row_ok && col0 < p.N) {
+          const long long off = g * p.out_gs + (long long)row * p.ldo + col0;
+          const int nvalid = p.N - col0;  // multiple of 8
+          if constexpr (EPI == EPI_F32) {
+            float* o = static_cast<float*>(p.out) + off;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              if (i < nvalid) {
+                float4 f = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                if (p.col_add != nullptr) {
+                  f.x += p.col_add[col0 + i];
+                  f.y += p.col_add[col0 + i + 1];
+                  f.z += p.col_add[col0 + i + 2];
+                  f.w += p.col_add[col0 + i + 3];
+                }
+                *reinterpret_cast<float4*>(o + i) = f;
+              }
+            }
+          } else if constexpr (EPI == EPI_BF16 || EPI == EPI_BF16_ADD_F32) {
+            if constexpr (EPI == EPI_BF16_ADD_F32) {
+              const float* ad = p.addend + (long long)row * p.add_ld + col0;
+#pragma unroll
+              for (int i = 0; i < 32; i += 4) {
+                if (i < nvalid) {
+                  const float4 f = *reinterpret_cast<const float4*>(ad + i);
+                  v[i] += f.x;
+                  v[i + 1] += f.y;
+                  v[i + 2] += f.z;
+                  v[i + 3] += f.w;
+                }
+              }
+            }
+            uint16_t* o = static_cast<uint16_t*>(p.out) + off;
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              if (i < nvalid)
+                *reinterpret_cast<uint4*>(o + i) =
+                    make_uint4(pack_bf16x2(v[i], v[i + 1]), pack_bf16x2(v[i + 2], v[i + 3]),
+                               pack_bf16x2(v[i + 4], v[i + 5]), pack_bf16x2(v[i + 6], v[i + 7]));
+            }
+          } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+            const long long aoff = g * p.aux_gs + (long long)row * p.aux_ld + col0;
+            const uint16_t* pa = static_cast<const uint16_t*>(p.aux_a) + aoff;
+            const uint16_t* pb = static_cast<const uint16_t*>(p.aux_b) + aoff;
+            uint16_t* oa = static_cast<uint16_t*>(p.out) + off;
+            uint16_t* ob = static_cast<uint16_t*>(p.out2) + off;
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              if (i < nvalid) {
+                const uint4 av = *reinterpret_cast<const uint4*>(pa + i);
+                const uint4 bv = *reinterpret_cast<const uint4*>(pb + i);
+                const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+                const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+                uint32_t da[4], db[4];
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                  float rda[2], rdb[2];
+#pragma unroll
+                  for (int h = 0; h < 2; ++h) {
+                    const float a = h ? bf16_hi(aw[w]) : bf16_lo(aw[w]);
+                    const float b = h ? bf16_hi(bw[w]) : bf16_lo(bw[w]);
+                    const float dh = v[i + 2 * w + h];
+                    const float sg = 1.0f / (1.0f + expf(-a));
+                    const float si = a * sg;
+                    rda[h] = dh * b * (sg * (1.0f + a * (1.0f - sg)));
+                    rdb[h] = dh * si;
+                  }
+                  da[w] = pack_bf16x2(rda[0], rda[1]);
+                  db[w] = pack_bf16x2(rdb[0], rdb[1]);
+                }
+                *reinterpret_cast<uint4*>(oa + i) = make_uint4(da[0], da[1], da[2], da[3]);
+                *reinterpret_cast<uint4*>(ob + i) = make_uint4(db[0], db[1], db[2], db[3]);
+              }
+            }
+          }
+          }  // row_ok && col0 < N
+        }
+      }
+      __syncwarp();
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ====================================================================== host side
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+moe_status_t make_map(CUtensorMap* m, const Mat& t, uint32_t box_inner, uint32_t box_rows, const char* what) {
+  if (t.ptr == nullptr) return fail(MOE_ERR_INVALID_ARG, std::string("gemm operand is null: ") + what);
+  if ((reinterpret_cast<uintptr_t>(t.ptr) & 15) != 0)
+    return fail(MOE_ERR_INVALID_ARG, std::string("gemm operand not 16-byte aligned: ") + what);
+  if (t.inner <= 0 || t.rows <= 0 || t.groups <= 0 || t.ld < t.inner || (t.ld * 2) % 16 != 0 ||
+      (t.gs * 2) % 16 != 0)
+    return fail(MOE_ERR_INVALID_ARG, std::string("gemm operand has a bad shape or stride: ") + what);
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(t.inner), static_cast<cuuint64_t>(t.rows),
+                        static_cast<cuuint64_t>(t.groups)};
+  const int64_t gs = t.groups > 1 ? t.gs : t.ld * t.rows;
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(t.ld * 2), static_cast<cuuint64_t>(gs * 2)};
+  cuuint32_t box[3] = {box_inner, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(t.ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(MOE_ERR_CUDA, std::string("cuTensorMapEncodeTiled failed for ") + what + " (" +
+                                  std::to_string(static_cast<int>(r)) + ")");
+  return MOE_OK;
+}
+
+template <int BN, bool A_MN, bool B_MN, int EPI>
+moe_status_t launch_instance(const TmaMaps& maps, const KParams& kp, int grid, cudaStream_t st) {
+  auto kern = gemm_kernel<BN, A_MN, B_MN, EPI>;
+  const int smem = Cfg<BN>::kSmem;
+  static bool attr_set = false;  // per instantiation
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_check(e, "cudaFuncSetAttribute(gemm)");
+    attr_set = true;
+  }
+  kern<<<grid, kThreads, smem, st>>>(maps, kp);
+  count_launch();
+  return cuda_check(cudaGetLastError(), "gemm launch");
+}
+
+}  // namespace
+
+int device_sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
+  if (a.M <= 0 || a.N <= 0 || a.groups <= 0) return MOE_OK;
+  if (a.bn != 128 && a.bn != 256) return fail(MOE_ERR_UNSUPPORTED, "gemm tile width must be 128 or 256");
+  if (a.groups > kMaxGroups) return fail(MOE_ERR_UNSUPPORTED, "too many gemm groups");
+  if (a.nseg < 1 || a.nseg > 3) return fail(MOE_ERR_INVALID_ARG, "gemm needs 1..3 K segments");
+  if (a.ragged != 0 && a.group_rows == nullptr) return fail(MOE_ERR_INVALID_ARG, "ragged gemm needs group rows");
+  if (a.ragged == 2 && a.nseg != 1) return fail(MOE_ERR_INVALID_ARG, "ragged-K gemm takes one segment");
+  if (a.epi == EPI_SWIGLU && (a.nseg != 1 || a.b_mn || a.N % (a.bn / 2) != 0))
+    return fail(MOE_ERR_UNSUPPORTED, "SwiGLU gemm needs one K-major segment and N a multiple of BN/2");
+  if (a.N % 8 != 0) return fail(MOE_ERR_UNSUPPORTED, "gemm N must be a multiple of 8");
+  if (a.out == nullptr) return fail(MOE_ERR_INVALID_ARG, "gemm output is null");
+
+  TmaMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  KParams kp;
+  memset(&kp, 0, sizeof(kp));
+  kp.M = a.M;
+  kp.N = a.N;
+  kp.groups = a.groups;
+  kp.ragged = a.ragged;
+  kp.group_rows = a.group_rows;
+  kp.nseg = a.nseg;
+  for (int s = 0; s < a.nseg; ++s) {
+    moe_status_t r;
+    r = make_map(&maps.a[s], a.A[s], 64, a.a_mn ? 64 : 128, "A");
+    if (r != MOE_OK) return r;
+    const uint32_t b_rows = a.b_mn ? 64 : (a.epi == EPI_SWIGLU ? a.bn / 2 : a.bn);
+    r = make_map(&maps.b[s], a.B[s], 64, b_rows, "B");
+    if (r != MOE_OK) return r;
+    kp.seg_kb[s] = a.ragged == 2 ? 0 : static_cast<int>((a.K[s] + kBK - 1) / kBK);
+  }
+  if (a.epi == EPI_SWIGLU) {
+    moe_status_t r = make_map(&maps.bv, a.Bv, 64, a.bn / 2, "B value");
+    if (r != MOE_OK) return r;
+  }
+  kp.m_fastest = a.m_fastest ? 1 : 0;
+  kp.out = a.out;
+  kp.ldo = a.ldo;
+  kp.out_gs = a.out_gs;
+  kp.out2 = a.out2;
+  kp.save_a = a.save_a;
+  kp.save_b = a.save_b;
+  kp.aux_a = a.aux_a;
+  kp.aux_b = a.aux_b;
+  kp.aux_ld = a.aux_ld;
+  kp.aux_gs = a.aux_gs;
+  kp.col_add = a.col_add;
+  kp.addend = a.addend;
+  kp.add_ld = a.add_ld;
+  kp.status = a.status;
+
+  const int out_cols = a.epi == EPI_SWIGLU ? a.bn / 2 : a.bn;
+  const long long tiles = static_cast<long long>(a.groups) * ((a.M + kBM - 1) / kBM) * ((a.N + out_cols - 1) / out_cols);
+  const int grid = static_cast<int>(std::min<long long>(tiles, device_sm_count()));
+  if (grid <= 0) return MOE_OK;
+
+#define MOE_GEMM_CASE(BN_, AMN_, BMN_, EPI_)                                               \
+  if (a.bn == BN_ && a.a_mn == AMN_ && a.b_mn == BMN_ && a.epi == EPI_)                   \
+    return launch_instance<BN_, AMN_, BMN_, EPI_>(maps, kp, grid, st);
+  // forward
+  MOE_GEMM_CASE(256, false, false, EPI_BF16)
+  MOE_GEMM_CASE(256, false, false, EPI_SWIGLU)
+  MOE_GEMM_CASE(128, false, false, EPI_F32)
+  // backward: dgrad (B stored [K][N]) and wgrad (both stored [K][.])
+  MOE_GEMM_CASE(256, false, true, EPI_BF16)
+  MOE_GEMM_CASE(256, false, true, EPI_SWIGLU_BWD)
+  MOE_GEMM_CASE(256, false, true, EPI_BF16_ADD_F32)
+  MOE_GEMM_CASE(256, true, true, EPI_BF16)
+  // test entry point: every operand layout with a float32 result
+  MOE_GEMM_CASE(256, false, false, EPI_F32)
+  MOE_GEMM_CASE(256, false, true, EPI_F32)
+  MOE_GEMM_CASE(256, true, false, EPI_F32)
+  MOE_GEMM_CASE(256, true, true, EPI_F32)
+  MOE_GEMM_CASE(256, true, false, EPI_BF16)
+#undef MOE_GEMM_CASE
+  return fail(MOE_ERR_UNSUPPORTED, "no gemm instance for this layout / epilogue");
+}
+
+}  // namespace moe

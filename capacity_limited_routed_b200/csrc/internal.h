@@ -1,0 +1,133 @@
+// internal.h -- declarations shared by the translation units of libmoe (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// ------------------------------------------------------------------ errors
+
+void set_error(const std::string& msg);
+moe_status_t fail(moe_status_t code, const std::string& msg);
+moe_status_t cuda_check(cudaError_t e, const char* what);
+
+// ------------------------------------------------------------------ launch accounting
+
+void count_launch(int n = 1);
+int64_t launches_so_far();
+
+// Brackets one step of a call with CUDA events while profiling is on.
+class ProfScope {
+ public:
+  ProfScope(const char* name, cudaStream_t st);
+  ~ProfScope();
+  ProfScope(const ProfScope&) = delete;
+  ProfScope& operator=(const ProfScope&) = delete;
+
+ private:
+  int slot_ = -1;
+  cudaStream_t st_ = nullptr;
+  int64_t launches0_ = 0;
+};
+
+// ------------------------------------------------------------------ GEMM
+
+enum Epi : int {
+  EPI_BF16 = 0,          // out = bf16(acc)
+  EPI_F32 = 1,           // out = acc (+ col_add[col])
+  EPI_SWIGLU = 2,        // acc = [gate | value]; out = bf16(silu(gate) * value); save_a/b = bf16(gate/value)
+  EPI_SWIGLU_BWD = 3,    // acc = dH; out = dA = dH*b*silu'(a), out2 = dB = dH*silu(a)
+  EPI_BF16_ADD_F32 = 4,  // out = bf16(acc + addend[row][col])
+};
+
+// A bf16 tensor in global memory seen as [groups][rows][inner], inner contiguous.
+struct Mat {
+  const void* ptr = nullptr;
+  int64_t inner = 0, rows = 0, groups = 1;
+  int64_t ld = 0;   // elements between consecutive rows (>= inner)
+  int64_t gs = 0;   // elements between consecutive groups
+};
+
+// D[g][m][n] = sum over segments s, k of A_s(g, m, k) * B_s(g, n, k).
+//   A K-major: A_s stored [M][K] (Mat inner = K);  A MN-major: stored [K][M] (inner = M).
+//   B K-major: B_s stored [N][K];                  B MN-major: stored [K][N].
+// ragged == 0: dense (or fixed-size groups).  ragged == 1: group g has
+// group_rows[g] valid rows of M (tiles past them are skipped; rows up to M are
+// stored).  ragged == 2: group g has group_rows[g] valid K (one segment; the
+// operand's K extent zero-fills the rest).
+struct GemmArgs {
+  int bn = 256;
+  bool a_mn = false, b_mn = false;
+  int epi = EPI_BF16;
+  int M = 0, N = 0;  // per group; N counts output columns
+  int groups = 1;
+  int ragged = 0;
+  const int32_t* group_rows = nullptr;
+  int nseg = 1;
+  Mat A[3], B[3];
+  Mat Bv;            // value weights paired with B[0] for EPI_SWIGLU
+  int64_t K[3] = {0, 0, 0};
+  bool m_fastest = false;
+  void* out = nullptr;
+  int64_t ldo = 0, out_gs = 0;
+  void* out2 = nullptr;
+  void* save_a = nullptr;
+  void* save_b = nullptr;
+  const void* aux_a = nullptr;
+  const void* aux_b = nullptr;
+  int64_t aux_ld = 0, aux_gs = 0;
+  const float* col_add = nullptr;
+  const float* addend = nullptr;
+  int64_t add_ld = 0;
+  int32_t* status = nullptr;
+};
+
+moe_status_t gemm_run(const GemmArgs& a, cudaStream_t stream);
+int device_sm_count();
+
+// ------------------------------------------------------------------ routing / movement kernels
+
+struct Geo {
+  int T, E, k, D, W, L, P, NP, Cs, Cr, dl;
+  int n_chunks;      // token chunks of the slot scan
+};
+
+constexpr int kScanTokensPerChunk = 32;
+
+moe_status_t launch_route(const Geo& g, const float* logits, const float* bias, int32_t* idx, float* gate,
+                          int32_t* hist, int32_t* nan_count, cudaStream_t st);
+// scratch ints needed by the slot scan
+size_t scan_scratch_ints(const Geo& g);
+moe_status_t launch_slot_scan(const Geo& g, const int32_t* idx, int32_t* slot, int32_t* stats, int32_t* scratch,
+                              cudaStream_t st);
+moe_status_t launch_pack(const Geo& g, const uint16_t* z, const int32_t* idx, const int32_t* slot,
+                         const int32_t* stats, uint16_t* pools, cudaStream_t st);
+moe_status_t launch_unpack(const Geo& g, const uint16_t* pools, uint16_t* xe, int32_t* rows, int32_t* status,
+                           cudaStream_t st);
+moe_status_t launch_zero_tail_rows(const Geo& g, uint16_t* buf, int64_t width, const int32_t* rows,
+                                   cudaStream_t st);
+moe_status_t launch_combine(const Geo& g, const uint16_t* ye, const float* gate, const int32_t* idx,
+                            const int32_t* slot, uint16_t* r, cudaStream_t st);
+moe_status_t launch_combine_bwd(const Geo& g, const uint16_t* dr, const uint16_t* ye, const float* gate,
+                                const int32_t* idx, const int32_t* slot, uint16_t* dye, float* dg,
+                                cudaStream_t st);
+moe_status_t launch_undispatch(const Geo& g, const uint16_t* dxe, const float* gate, const float* dg,
+                               const int32_t* idx, const int32_t* slot, float* dz_routed, uint16_t* dlogits,
+                               cudaStream_t st);
+moe_status_t launch_bias_update(const Geo& g, const int32_t* hist, float* bias, float step, cudaStream_t st);
+
+// stats buffer layout (int32 words)
+constexpr int kStatsHead = 8;  // moe_stats_t
+inline int stats_hist(const Geo& g) { return kStatsHead; }
+inline int stats_kept_e(const Geo& g) { return kStatsHead + g.E; }
+inline int stats_ds_e(const Geo& g) { return kStatsHead + 2 * g.E; }
+inline int stats_dr_e(const Geo& g) { return kStatsHead + 3 * g.E; }
+inline int stats_pool_fill(const Geo& g) { return kStatsHead + 4 * g.E; }
+inline int stats_words(const Geo& g) { return kStatsHead + 4 * g.E + g.NP; }
+
+}  // namespace moe

@@ -1,0 +1,890 @@
+// moe_api.cu -- the C ABI of libmoe: plans, buffer layouts, argument checks and the order of
+// launches for the forward and backward pass of the capacity-limited, pooled-wave MoE block.
+//
+// Step order of the forward pass ("Marin начинает открытое обучение MoE-модели с 535 млрд
+// параметров", §2; "Marin 535B-A23B：一场完全公开的前沿 MoE 训练直播", §2.2, §3.2):
+// latent down-projection, router logits, top-k + gates + histogram, slot assignment,
+// pack into pools (sender), unpack by packed id (receiver), grouped SwiGLU experts,
+// combine, shared experts, up-projection fused with the shared down-projection.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "internal.h"
+
+struct moe_plan {
+  moe_config_t cfg;
+  moe::Geo g;
+  int dm, dl, E, k, h, S, hs;
+  // forward context layout (byte offsets); training adds the SwiGLU pre-activations
+  struct Ctx {
+    size_t z, logits, idx, gate, slot, rows, xe, ae, be, he, ye, r, as, bs, hsh, bytes;
+  } saved, infer;
+  // scratch layouts
+  size_t ws_scan, ws_pools, ws_ctx, ws_fwd_bytes;                        // forward
+  size_t ws_ffn_xe, ws_ffn_he, ws_ffn_rows, ws_ffn_bytes;                // moe_expert_ffn alone
+  size_t b_dr, b_das, b_dbs, b_dye, b_dg, b_dae, b_dbe, b_dxe, b_dlog, b_dzr, b_dz, ws_bwd_bytes;
+  size_t pools_bytes, expert_out_bytes, slot_bytes, stats_bytes, ws_bytes;
+};
+
+namespace moe {
+
+namespace {
+thread_local std::string g_last_error;
+}
+
+void set_error(const std::string& msg) { g_last_error = msg; }
+
+moe_status_t fail(moe_status_t code, const std::string& msg) {
+  g_last_error = msg;
+  return code;
+}
+
+moe_status_t cuda_check(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return MOE_OK;
+  return fail(MOE_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+// ---------------------------------------------------------------------- launch accounting
+
+namespace {
+std::atomic<int64_t> g_launches{0};
+
+struct ProfRecord {
+  char name[40];
+  cudaEvent_t start, stop;
+  int64_t launches;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRecord> g_prof;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+}  // namespace
+
+void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+int64_t launches_so_far() { return g_launches.load(std::memory_order_relaxed); }
+
+ProfScope::ProfScope(const char* name, cudaStream_t st) : st_(st) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (!g_prof_on) return;
+  ProfRecord r;
+  std::memset(&r, 0, sizeof(r));
+  std::strncpy(r.name, name, sizeof(r.name) - 1);
+  r.start = take_event();
+  r.stop = take_event();
+  if (r.start == nullptr || r.stop == nullptr) return;
+  cudaEventRecord(r.start, st);
+  launches0_ = launches_so_far();
+  slot_ = static_cast<int>(g_prof.size());
+  g_prof.push_back(r);
+}
+
+ProfScope::~ProfScope() {
+  if (slot_ < 0) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (slot_ >= static_cast<int>(g_prof.size())) return;
+  cudaEventRecord(g_prof[slot_].stop, st_);
+  g_prof[slot_].launches = launches_so_far() - launches0_;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t take(size_t& off, size_t bytes) {
+  off = (off + kAlign - 1) / kAlign * kAlign;
+  const size_t at = off;
+  off += bytes;
+  return at;
+}
+
+void layout_ctx(const moe_plan& p, bool training, moe_plan::Ctx& c) {
+  const size_t T = p.g.T, E = p.E, k = p.k, dl = p.dl, h = p.h, Cr = p.g.Cr, SH = size_t(p.S) * p.hs;
+  size_t off = 0;
+  c.z = take(off, T * dl * 2);
+  c.logits = take(off, T * E * 4);
+  c.idx = take(off, T * k * 4);
+  c.gate = take(off, T * k * 4);
+  c.slot = take(off, T * k * 8);
+  c.rows = take(off, E * 4);
+  c.xe = take(off, E * Cr * dl * 2);
+  c.ae = training ? take(off, E * Cr * h * 2) : 0;
+  c.be = training ? take(off, E * Cr * h * 2) : 0;
+  c.he = take(off, E * Cr * h * 2);
+  c.ye = take(off, E * Cr * dl * 2);
+  c.r = take(off, T * dl * 2);
+  c.as = training ? take(off, T * SH * 2) : 0;
+  c.bs = training ? take(off, T * SH * 2) : 0;
+  c.hsh = take(off, T * SH * 2);
+  c.bytes = (off + kAlign - 1) / kAlign * kAlign;
+}
+
+void layout(moe_plan& p) {
+  const size_t T = p.g.T, E = p.E, k = p.k, dl = p.dl, h = p.h, Cr = p.g.Cr, SH = size_t(p.S) * p.hs;
+  layout_ctx(p, true, p.saved);
+  layout_ctx(p, false, p.infer);
+  p.pools_bytes = size_t(p.g.NP) * p.g.Cs * (dl + 8) * 2;
+  p.expert_out_bytes = E * Cr * dl * 2;
+  p.slot_bytes = T * k * 8;
+  p.stats_bytes = size_t(stats_words(p.g)) * 4;
+  size_t off = 0;
+  p.ws_scan = take(off, scan_scratch_ints(p.g) * 4);
+  p.ws_pools = take(off, p.pools_bytes);
+  p.ws_ctx = take(off, p.infer.bytes);  // used only when the forward keeps no context
+  p.ws_fwd_bytes = off;
+  off = 0;
+  p.ws_ffn_xe = take(off, E * Cr * dl * 2);
+  p.ws_ffn_he = take(off, E * Cr * h * 2);
+  p.ws_ffn_rows = take(off, E * 4);
+  p.ws_ffn_bytes = off;
+  off = 0;
+  p.b_dr = take(off, T * dl * 2);
+  p.b_das = take(off, T * SH * 2);
+  p.b_dbs = take(off, T * SH * 2);
+  p.b_dye = take(off, E * Cr * dl * 2);
+  p.b_dg = take(off, T * k * 4);
+  p.b_dae = take(off, E * Cr * h * 2);
+  p.b_dbe = take(off, E * Cr * h * 2);
+  p.b_dxe = take(off, E * Cr * dl * 2);
+  p.b_dlog = take(off, T * E * 2);
+  p.b_dzr = take(off, T * dl * 4);
+  p.b_dz = take(off, T * dl * 2);
+  p.ws_bwd_bytes = off;
+  p.ws_bytes = std::max({p.ws_fwd_bytes, p.ws_ffn_bytes, p.ws_bwd_bytes, p.ws_scan + scan_scratch_ints(p.g) * 4});
+  p.ws_bytes = (p.ws_bytes + kAlign - 1) / kAlign * kAlign;
+}
+
+// Capacities: expected rows times num/den, rounded up exactly (64-bit integers).
+int32_t ceil_cap(int64_t rows_num, int64_t rows_den, int64_t num, int64_t den) {
+  const int64_t a = rows_num * num, b = rows_den * den;
+  return static_cast<int32_t>((a + b - 1) / b);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Once per device: is it an sm_100 part?
+moe_status_t device_ok() {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MOE_ERR_UNSUPPORTED, std::string("no CUDA device: ") + cudaGetErrorString(e));
+  }
+  static int checked[64] = {0};  // 0 unknown, 1 ok, 2 bad
+  if (dev >= 0 && dev < 64 && checked[dev] == 1) return MOE_OK;
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0) {
+    if (dev >= 0 && dev < 64) checked[dev] = 2;
+    return fail(MOE_ERR_UNSUPPORTED, "libmoe needs an sm_100 (B200) device, found sm_" + std::to_string(major) +
+                                         std::to_string(minor));
+  }
+  if (dev >= 0 && dev < 64) checked[dev] = 1;
+  return MOE_OK;
+}
+
+#define MOE_TRY(x)                       \
+  do {                                   \
+    moe_status_t _s = (x);               \
+    if (_s != MOE_OK) return _s;         \
+  } while (0)
+
+Mat mat(const void* ptr, int64_t inner, int64_t rows, int64_t groups = 1) {
+  Mat m;
+  m.ptr = ptr;
+  m.inner = inner;
+  m.rows = rows;
+  m.groups = groups;
+  m.ld = inner;
+  m.gs = inner * rows;
+  return m;
+}
+
+template <class T>
+T* at(void* base, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(base) + off);
+}
+template <class T>
+const T* at(const void* base, size_t off) {
+  return reinterpret_cast<const T*>(static_cast<const char*>(base) + off);
+}
+
+struct CtxPtrs {
+  uint16_t *z, *xe, *ae, *be, *he, *ye, *r, *as, *bs, *hsh;
+  float *logits, *gate;
+  int32_t *idx, *slot, *rows;
+};
+
+CtxPtrs ctx_ptrs(const moe_plan& p, void* base, bool training) {
+  const moe_plan::Ctx& c = training ? p.saved : p.infer;
+  CtxPtrs q;
+  q.z = at<uint16_t>(base, c.z);
+  q.logits = at<float>(base, c.logits);
+  q.idx = at<int32_t>(base, c.idx);
+  q.gate = at<float>(base, c.gate);
+  q.slot = at<int32_t>(base, c.slot);
+  q.rows = at<int32_t>(base, c.rows);
+  q.xe = at<uint16_t>(base, c.xe);
+  q.ae = training ? at<uint16_t>(base, c.ae) : nullptr;
+  q.be = training ? at<uint16_t>(base, c.be) : nullptr;
+  q.he = at<uint16_t>(base, c.he);
+  q.ye = at<uint16_t>(base, c.ye);
+  q.r = at<uint16_t>(base, c.r);
+  q.as = training ? at<uint16_t>(base, c.as) : nullptr;
+  q.bs = training ? at<uint16_t>(base, c.bs) : nullptr;
+  q.hsh = at<uint16_t>(base, c.hsh);
+  return q;
+}
+
+// receiver unpack + grouped SwiGLU experts (shared by moe_expert_ffn and moe_forward)
+moe_status_t run_experts(const moe_plan& p, const uint16_t* w1, const uint16_t* w3, const uint16_t* w2,
+                         const uint16_t* pools, uint16_t* xe, int32_t* rows, uint16_t* ae, uint16_t* be, uint16_t* he,
+                         uint16_t* ye, int32_t* status, cudaStream_t st) {
+  const Geo& g = p.g;
+  {
+    ProfScope ps("experts.unpack", st);
+    MOE_TRY(launch_unpack(g, pools, xe, rows, status, st));
+    MOE_TRY(launch_zero_tail_rows(g, xe, p.dl, rows, st));
+  }
+  GemmArgs a;
+  a.bn = 256;
+  a.epi = EPI_SWIGLU;
+  a.M = g.Cr;
+  a.N = p.h;
+  a.groups = p.E;
+  a.ragged = 1;
+  a.group_rows = rows;
+  a.A[0] = mat(xe, p.dl, g.Cr, p.E);
+  a.B[0] = mat(w1, p.dl, p.h, p.E);
+  a.Bv = mat(w3, p.dl, p.h, p.E);
+  a.K[0] = p.dl;
+  a.m_fastest = true;
+  a.out = he;
+  a.ldo = p.h;
+  a.out_gs = int64_t(g.Cr) * p.h;
+  a.save_a = ae;
+  a.save_b = be;
+  a.status = status;
+  {
+    ProfScope ps("experts.gate_up", st);
+    MOE_TRY(gemm_run(a, st));
+  }
+  GemmArgs d;
+  d.bn = 256;
+  d.epi = EPI_BF16;
+  d.M = g.Cr;
+  d.N = p.dl;
+  d.groups = p.E;
+  d.ragged = 1;
+  d.group_rows = rows;
+  d.A[0] = mat(he, p.h, g.Cr, p.E);
+  d.B[0] = mat(w2, p.h, p.dl, p.E);
+  d.K[0] = p.h;
+  d.m_fastest = true;
+  d.out = ye;
+  d.ldo = p.dl;
+  d.out_gs = int64_t(g.Cr) * p.dl;
+  d.status = status;
+  ProfScope ps("experts.down", st);
+  return gemm_run(d, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_last_error(void) { return g_last_error.c_str(); }
+
+moe_status_t moe_profile_start(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& r : g_prof) {
+    g_event_pool.push_back(r.start);
+    g_event_pool.push_back(r.stop);
+  }
+  g_prof.clear();
+  g_prof_on = true;
+  return MOE_OK;
+}
+
+moe_status_t moe_profile_stop(moe_profile_record_t* out, int32_t cap, int32_t* count) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = false;
+  int32_t n = 0;
+  for (auto& r : g_prof) {
+    if (cudaEventSynchronize(r.stop) != cudaSuccess) return cuda_check(cudaGetLastError(), "profile sync");
+    if (out != nullptr && n < cap) {
+      std::memcpy(out[n].name, r.name, sizeof(out[n].name));
+      float ms = 0.0f;
+      cudaEventElapsedTime(&ms, r.start, r.stop);
+      out[n].ms = ms;
+      out[n].launches = static_cast<int32_t>(r.launches);
+    }
+    ++n;
+  }
+  if (count != nullptr) *count = n;
+  return MOE_OK;
+}
+
+int64_t moe_kernel_launches(void) { return launches_so_far(); }
+
+moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out) {
+  if (cfg == nullptr || out == nullptr) return fail(MOE_ERR_INVALID_ARG, "null argument");
+  *out = nullptr;
+  const moe_config_t& c = *cfg;
+  if (c.T < 0 || c.d_model <= 0 || c.d_latent <= 0 || c.n_experts <= 0 || c.top_k <= 0 || c.n_dest <= 0 ||
+      c.n_waves <= 0 || c.hidden_routed <= 0 || c.n_shared <= 0 || c.hidden_shared <= 0)
+    return fail(MOE_ERR_INVALID_ARG, "sizes must be positive (T may be 0)");
+  if (c.cap_send_num <= 0 || c.cap_send_den <= 0 || c.cap_recv_num <= 0 || c.cap_recv_den <= 0)
+    return fail(MOE_ERR_INVALID_ARG, "capacity ratios must be positive");
+  if (c.n_experts % c.n_dest != 0) return fail(MOE_ERR_UNSUPPORTED, "E must be a multiple of D");
+  const int L = c.n_experts / c.n_dest;
+  if (L % c.n_waves != 0) return fail(MOE_ERR_UNSUPPORTED, "E/D must be a multiple of the wave count");
+  if (c.top_k > c.n_experts || c.top_k > 32) return fail(MOE_ERR_UNSUPPORTED, "top_k must be <= min(E, 32)");
+  if (c.n_experts > 1024 || c.n_experts % 8 != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "E must be a multiple of 8, at most 1024");
+  if (c.d_model % 64 || c.d_latent % 64) return fail(MOE_ERR_UNSUPPORTED, "d_model and d_latent must be multiples of 64");
+  if (c.hidden_routed % 128 || c.hidden_shared % 128)
+    return fail(MOE_ERR_UNSUPPORTED, "hidden widths must be multiples of 128");
+  if (L / c.n_waves > 32) return fail(MOE_ERR_UNSUPPORTED, "at most 32 experts per wave");
+  const int64_t A = int64_t(c.T) * c.top_k;
+  if (A > (int64_t(1) << 30)) return fail(MOE_ERR_UNSUPPORTED, "T * top_k too large");
+  moe_plan* p = new moe_plan();
+  std::memset(static_cast<void*>(p), 0, sizeof(*p));
+  p->cfg = c;
+  p->dm = c.d_model;
+  p->dl = c.d_latent;
+  p->E = c.n_experts;
+  p->k = c.top_k;
+  p->h = c.hidden_routed;
+  p->S = c.n_shared;
+  p->hs = c.hidden_shared;
+  Geo& g = p->g;
+  g.T = c.T;
+  g.E = c.n_experts;
+  g.k = c.top_k;
+  g.D = c.n_dest;
+  g.W = c.n_waves;
+  g.L = L;
+  g.P = L / c.n_waves;
+  g.NP = c.n_dest * c.n_waves;
+  g.Cs = ceil_cap(A, int64_t(c.n_dest) * c.n_waves, c.cap_send_num, c.cap_send_den);
+  g.Cr = ceil_cap(A, c.n_experts, c.cap_recv_num, c.cap_recv_den);
+  if (g.Cs < 1) g.Cs = 1;
+  if (g.Cr < 1) g.Cr = 1;
+  g.dl = c.d_latent;
+  g.n_chunks = (c.T + kScanTokensPerChunk - 1) / kScanTokensPerChunk;
+  if (g.n_chunks < 1) g.n_chunks = 1;
+  layout(*p);
+  *out = p;
+  return MOE_OK;
+}
+
+moe_status_t moe_plan_destroy(moe_plan_t plan) {
+  delete plan;
+  return MOE_OK;
+}
+
+moe_status_t moe_plan_info(moe_plan_t p, moe_plan_info_t* out) {
+  if (p == nullptr || out == nullptr) return fail(MOE_ERR_INVALID_ARG, "null argument");
+  out->local_experts = p->g.L;
+  out->experts_per_wave = p->g.P;
+  out->n_pools = p->g.NP;
+  out->cap_send = p->g.Cs;
+  out->cap_recv = p->g.Cr;
+  out->pool_row_elems = p->dl + 8;
+  out->pools_bytes = p->pools_bytes;
+  out->expert_out_bytes = p->expert_out_bytes;
+  out->slot_bytes = p->slot_bytes;
+  out->stats_bytes = p->stats_bytes;
+  out->saved_bytes = p->saved.bytes;
+  out->workspace_bytes = p->ws_bytes;
+  return MOE_OK;
+}
+
+moe_status_t moe_saved_view(moe_plan_t p, const void* saved, moe_saved_view_t* out) {
+  if (p == nullptr || saved == nullptr || out == nullptr) return fail(MOE_ERR_INVALID_ARG, "null argument");
+  CtxPtrs q = ctx_ptrs(*p, const_cast<void*>(saved), true);
+  out->z = q.z;
+  out->logits = q.logits;
+  out->topk_idx = q.idx;
+  out->topk_gate = q.gate;
+  out->slot = q.slot;
+  out->expert_rows = q.rows;
+  out->expert_in = q.xe;
+  out->expert_out = q.ye;
+  out->r = q.r;
+  return MOE_OK;
+}
+
+moe_status_t moe_route(moe_plan_t p, const float* logits, const float* bias, int32_t* topk_idx, float* topk_gate,
+                       int32_t* hist, void* stream) {
+  if (p == nullptr) return fail(MOE_ERR_INVALID_ARG, "null plan");
+  if (p->g.T > 0 && (!logits || !topk_idx || !topk_gate)) return fail(MOE_ERR_INVALID_ARG, "null buffer");
+  if (!bias || !hist) return fail(MOE_ERR_INVALID_ARG, "null buffer");
+  MOE_TRY(device_ok());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MOE_TRY(cuda_check(cudaMemsetAsync(hist, 0, sizeof(int32_t) * p->E, st), "hist memset"));
+  return launch_route(p->g, logits, bias, topk_idx, topk_gate, hist, nullptr, st);
+}
+
+moe_status_t moe_dispatch(moe_plan_t p, const uint16_t* z, const int32_t* topk_idx, uint16_t* pools, int32_t* slot,
+                          void* stats, void* ws, size_t ws_bytes, void* stream) {
+  if (p == nullptr) return fail(MOE_ERR_INVALID_ARG, "null plan");
+  if (!pools || !stats || !ws) return fail(MOE_ERR_INVALID_ARG, "null buffer");
+  if (p->g.T > 0 && (!z || !topk_idx || !slot)) return fail(MOE_ERR_INVALID_ARG, "null buffer");
+  if (!aligned16(z) || !aligned16(pools)) return fail(MOE_ERR_INVALID_ARG, "z and pools must be 16-byte aligned");
+  if (ws_bytes < p->ws_scan + scan_scratch_ints(p->g) * 4) return fail(MOE_ERR_WORKSPACE, "workspace too small");
+  MOE_TRY(device_ok());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* s = static_cast<int32_t*>(stats);
+  MOE_TRY(launch_slot_scan(p->g, topk_idx, slot, s, at<int32_t>(ws, p->ws_scan), st));
+  return launch_pack(p->g, z, topk_idx, slot, s, pools, st);
+}
+
+moe_status_t moe_expert_ffn(moe_plan_t p, const moe_expert_weights_t* w, const uint16_t* pools, uint16_t* expert_out,
+                            int32_t* expert_rows, void* ws, size_t ws_bytes, void* stream) {
+  if (p == nullptr || w == nullptr) return fail(MOE_ERR_INVALID_ARG, "null argument");
+  if (!w->w1 || !w->w3 || !w->w2 || !pools || !expert_out || !ws)
+    return fail(MOE_ERR_INVALID_ARG, "null buffer");
+  if (ws_bytes < p->ws_ffn_bytes) return fail(MOE_ERR_WORKSPACE, "workspace too small");
+  if (!aligned16(expert_out)) return fail(MOE_ERR_INVALID_ARG, "expert_out must be 16-byte aligned");
+  MOE_TRY(device_ok());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* rows = expert_rows ? expert_rows : at<int32_t>(ws, p->ws_ffn_rows);
+  return run_experts(*p, w->w1, w->w3, w->w2, pools, at<uint16_t>(ws, p->ws_ffn_xe), rows, nullptr, nullptr,
+                     at<uint16_t>(ws, p->ws_ffn_he), expert_out, nullptr, st);
+}
+
+moe_status_t moe_combine(moe_plan_t p, const uint16_t* expert_out, const float* topk_gate, const int32_t* topk_idx,
+                         const int32_t* slot, uint16_t* r, void* stream) {
+  if (p == nullptr) return fail(MOE_ERR_INVALID_ARG, "null plan");
+  if (p->g.T == 0) return MOE_OK;
+  if (!expert_out || !topk_gate || !topk_idx || !slot || !r) return fail(MOE_ERR_INVALID_ARG, "null buffer");
+  if (!aligned16(expert_out) || !aligned16(r)) return fail(MOE_ERR_INVALID_ARG, "buffers must be 16-byte aligned");
+  MOE_TRY(device_ok());
+  return launch_combine(p->g, expert_out, topk_gate, topk_idx, slot, r, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const uint16_t* x, const float* bias,
+                         const float* logit_offset, uint16_t* y, void* stats, void* saved, void* ws, size_t ws_bytes,
+                         void* stream) {
+  if (p == nullptr || w == nullptr) return fail(MOE_ERR_INVALID_ARG, "null argument");
+  if (!w->w_lat_down || !w->w_router || !w->w1 || !w->w3 || !w->w2 || !w->w_lat_up || !w->ws1 || !w->ws3 ||
+      !w->ws2)
+    return fail(MOE_ERR_INVALID_ARG, "null weight");
+  if (!bias || !stats || !ws) return fail(MOE_ERR_INVALID_ARG, "null buffer");
+  if (p->g.T > 0 && (!x || !y)) return fail(MOE_ERR_INVALID_ARG, "null buffer");
+  if (ws_bytes < p->ws_fwd_bytes) return fail(MOE_ERR_WORKSPACE, "workspace too small");
+  MOE_TRY(device_ok());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* s = static_cast<int32_t*>(stats);
+  const Geo& g = p->g;
+  MOE_TRY(cuda_check(cudaMemsetAsync(s, 0, p->stats_bytes, st), "stats memset"));
+  if (g.T == 0) return MOE_OK;
+  const bool training = saved != nullptr;
+  CtxPtrs c = ctx_ptrs(*p, training ? saved : at<void>(ws, p->ws_ctx), training);
+  int32_t* status = s + 3;
+  const int64_t SH = int64_t(p->S) * p->hs;
+
+  // latent down-projection: z = x W_lat_down^T
+  {
+    ProfScope ps("fwd.lat_down", st);
+    GemmArgs a;
+    a.M = g.T;
+    a.N = p->dl;
+    a.A[0] = mat(x, p->dm, g.T);
+    a.B[0] = mat(w->w_lat_down, p->dm, p->dl);
+    a.K[0] = p->dm;
+    a.out = c.z;
+    a.ldo = p->dl;
+    a.status = status;
+    MOE_TRY(gemm_run(a, st));
+  }
+  // router logits (float32, + per-expert offset)
+  {
+    ProfScope ps("fwd.router", st);
+    GemmArgs a;
+    a.bn = 128;
+    a.epi = EPI_F32;
+    a.M = g.T;
+    a.N = p->E;
+    a.A[0] = mat(c.z, p->dl, g.T);
+    a.B[0] = mat(w->w_router, p->dl, p->E);
+    a.K[0] = p->dl;
+    a.out = c.logits;
+    a.ldo = p->E;
+    a.col_add = logit_offset;
+    a.status = status;
+    MOE_TRY(gemm_run(a, st));
+  }
+  {
+    ProfScope ps("fwd.route_topk", st);
+    MOE_TRY(launch_route(g, c.logits, bias, c.idx, c.gate, s + stats_hist(g), s + 7, st));
+  }
+  {
+    ProfScope ps("fwd.slot_scan", st);
+    MOE_TRY(launch_slot_scan(g, c.idx, c.slot, s, at<int32_t>(ws, p->ws_scan), st));
+  }
+  uint16_t* pools = at<uint16_t>(ws, p->ws_pools);
+  {
+    ProfScope ps("fwd.dispatch_pack", st);
+    MOE_TRY(launch_pack(g, c.z, c.idx, c.slot, s, pools, st));
+  }
+  MOE_TRY(run_experts(*p, w->w1, w->w3, w->w2, pools, c.xe, c.rows, c.ae, c.be, c.he, c.ye, status, st));
+  {
+    ProfScope ps("fwd.combine", st);
+    MOE_TRY(launch_combine(g, c.ye, c.gate, c.idx, c.slot, c.r, st));
+  }
+  // shared experts: H_s = silu(x ws1^T) * (x ws3^T)
+  {
+    ProfScope ps("fwd.shared_gate_up", st);
+    GemmArgs a;
+    a.epi = EPI_SWIGLU;
+    a.M = g.T;
+    a.N = static_cast<int>(SH);
+    a.A[0] = mat(x, p->dm, g.T);
+    a.B[0] = mat(w->ws1, p->dm, SH);
+    a.Bv = mat(w->ws3, p->dm, SH);
+    a.K[0] = p->dm;
+    a.out = c.hsh;
+    a.ldo = SH;
+    a.save_a = c.as;
+    a.save_b = c.bs;
+    a.status = status;
+    MOE_TRY(gemm_run(a, st));
+  }
+  // y = r W_lat_up^T + H_s ws2^T (two K segments, one accumulator)
+  {
+    ProfScope ps("fwd.lat_up_shared_down", st);
+    GemmArgs a;
+    a.M = g.T;
+    a.N = p->dm;
+    a.nseg = 2;
+    a.A[0] = mat(c.r, p->dl, g.T);
+    a.B[0] = mat(w->w_lat_up, p->dl, p->dm);
+    a.K[0] = p->dl;
+    a.A[1] = mat(c.hsh, SH, g.T);
+    a.B[1] = mat(w->ws2, SH, p->dm);
+    a.K[1] = SH;
+    a.out = y;
+    a.ldo = p->dm;
+    a.status = status;
+    MOE_TRY(gemm_run(a, st));
+  }
+  return MOE_OK;
+}
+
+moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* saved, const uint16_t* x,
+                          const uint16_t* dy, uint16_t* dx, const moe_grads_t* gr, void* ws, size_t ws_bytes,
+                          void* stream) {
+  if (p == nullptr || w == nullptr || gr == nullptr) return fail(MOE_ERR_INVALID_ARG, "null argument");
+  if (!saved || !ws) return fail(MOE_ERR_INVALID_ARG, "null buffer");
+  if (!w->w_lat_down || !w->w_router || !w->w1 || !w->w3 || !w->w2 || !w->w_lat_up || !w->ws1 || !w->ws3 ||
+      !w->ws2)
+    return fail(MOE_ERR_INVALID_ARG, "null weight");
+  if (!gr->w_lat_down || !gr->w_router || !gr->w1 || !gr->w3 || !gr->w2 || !gr->w_lat_up || !gr->ws1 || !gr->ws3 ||
+      !gr->ws2)
+    return fail(MOE_ERR_INVALID_ARG, "null gradient");
+  if (p->g.T > 0 && (!x || !dy || !dx)) return fail(MOE_ERR_INVALID_ARG, "null buffer");
+  if (ws_bytes < p->ws_bwd_bytes) return fail(MOE_ERR_WORKSPACE, "workspace too small");
+  MOE_TRY(device_ok());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Geo& g = p->g;
+  const int64_t SH = int64_t(p->S) * p->hs;
+  const int64_t T = g.T, E = p->E, Cr = g.Cr, dl = p->dl, dm = p->dm, h = p->h;
+  if (g.T == 0) {
+    // no tokens: every gradient is zero
+    const size_t sizes[9] = {size_t(dl * dm), size_t(E * dl), size_t(E * h * dl), size_t(E * h * dl),
+                             size_t(E * dl * h), size_t(dm * dl), size_t(SH * dm), size_t(SH * dm), size_t(dm * SH)};
+    uint16_t* ptrs[9] = {gr->w_lat_down, gr->w_router, gr->w1, gr->w3, gr->w2, gr->w_lat_up, gr->ws1, gr->ws3, gr->ws2};
+    for (int i = 0; i < 9; ++i) MOE_TRY(cuda_check(cudaMemsetAsync(ptrs[i], 0, sizes[i] * 2, st), "grad memset"));
+    return MOE_OK;
+  }
+  CtxPtrs c = ctx_ptrs(*p, const_cast<void*>(saved), true);
+  uint16_t* dr = at<uint16_t>(ws, p->b_dr);
+  uint16_t* das = at<uint16_t>(ws, p->b_das);
+  uint16_t* dbs = at<uint16_t>(ws, p->b_dbs);
+  uint16_t* dye = at<uint16_t>(ws, p->b_dye);
+  float* dg = at<float>(ws, p->b_dg);
+  uint16_t* dae = at<uint16_t>(ws, p->b_dae);
+  uint16_t* dbe = at<uint16_t>(ws, p->b_dbe);
+  uint16_t* dxe = at<uint16_t>(ws, p->b_dxe);
+  uint16_t* dlog = at<uint16_t>(ws, p->b_dlog);
+  float* dzr = at<float>(ws, p->b_dzr);
+  uint16_t* dz = at<uint16_t>(ws, p->b_dz);
+  int32_t* status = nullptr;
+
+  // y = r W_up^T + H_s ws2^T:  dr = dy W_up,  dH_s = dy ws2 -> SwiGLU backward
+  {
+    ProfScope ps("bwd.dr", st);
+    GemmArgs a;
+    a.b_mn = true;
+    a.M = g.T;
+    a.N = p->dl;
+    a.A[0] = mat(dy, dm, T);
+    a.B[0] = mat(w->w_lat_up, dl, dm);
+    a.K[0] = dm;
+    a.out = dr;
+    a.ldo = dl;
+    MOE_TRY(gemm_run(a, st));
+  }
+  {
+    ProfScope ps("bwd.shared_dgrad_swiglu", st);
+    GemmArgs a;
+    a.b_mn = true;
+    a.epi = EPI_SWIGLU_BWD;
+    a.M = g.T;
+    a.N = static_cast<int>(SH);
+    a.A[0] = mat(dy, dm, T);
+    a.B[0] = mat(w->ws2, SH, dm);
+    a.K[0] = dm;
+    a.aux_a = c.as;
+    a.aux_b = c.bs;
+    a.aux_ld = SH;
+    a.out = das;
+    a.out2 = dbs;
+    a.ldo = SH;
+    MOE_TRY(gemm_run(a, st));
+  }
+  // dW_up = dy^T r,  dws2 = dy^T H_s
+  {
+    ProfScope ps("bwd.wgrad_lat_up_shared_down", st);
+    GemmArgs a;
+    a.a_mn = a.b_mn = true;
+    a.M = static_cast<int>(dm);
+    a.N = static_cast<int>(dl);
+    a.A[0] = mat(dy, dm, T);
+    a.B[0] = mat(c.r, dl, T);
+    a.K[0] = T;
+    a.out = gr->w_lat_up;
+    a.ldo = dl;
+    MOE_TRY(gemm_run(a, st));
+    a.N = static_cast<int>(SH);
+    a.B[0] = mat(c.hsh, SH, T);
+    a.out = gr->ws2;
+    a.ldo = SH;
+    MOE_TRY(gemm_run(a, st));
+  }
+  // combine backward: dY = g dr on kept rows, dg = <dr, Y>
+  {
+    ProfScope ps("bwd.combine", st);
+    MOE_TRY(launch_combine_bwd(g, dr, c.ye, c.gate, c.idx, c.slot, dye, dg, st));
+    MOE_TRY(launch_zero_tail_rows(g, dye, dl, c.rows, st));
+  }
+  // routed experts: dH = dY w2 -> (dA, dB);  dw2 = dY^T H;  dX = dA w1 + dB w3;  dw1 = dA^T X, dw3 = dB^T X
+  {
+    ProfScope ps("bwd.experts_dgrad_down", st);
+    GemmArgs a;
+    a.b_mn = true;
+    a.epi = EPI_SWIGLU_BWD;
+    a.M = g.Cr;
+    a.N = static_cast<int>(h);
+    a.groups = p->E;
+    a.ragged = 1;
+    a.group_rows = c.rows;
+    a.A[0] = mat(dye, dl, Cr, E);
+    a.B[0] = mat(w->w2, h, dl, E);
+    a.K[0] = dl;
+    a.m_fastest = true;
+    a.aux_a = c.ae;
+    a.aux_b = c.be;
+    a.aux_ld = h;
+    a.aux_gs = Cr * h;
+    a.out = dae;
+    a.out2 = dbe;
+    a.ldo = h;
+    a.out_gs = Cr * h;
+    MOE_TRY(gemm_run(a, st));
+  }
+  {
+    ProfScope ps("bwd.experts_wgrad_down", st);
+    GemmArgs a;
+    a.a_mn = a.b_mn = true;
+    a.M = static_cast<int>(dl);
+    a.N = static_cast<int>(h);
+    a.groups = p->E;
+    a.ragged = 2;
+    a.group_rows = c.rows;
+    a.A[0] = mat(dye, dl, Cr, E);
+    a.B[0] = mat(c.he, h, Cr, E);
+    a.m_fastest = true;
+    a.out = gr->w2;
+    a.ldo = h;
+    a.out_gs = dl * h;
+    MOE_TRY(gemm_run(a, st));
+  }
+  {
+    ProfScope ps("bwd.experts_dgrad_gate_up", st);
+    GemmArgs a;
+    a.b_mn = true;
+    a.M = g.Cr;
+    a.N = static_cast<int>(dl);
+    a.groups = p->E;
+    a.ragged = 1;
+    a.group_rows = c.rows;
+    a.nseg = 2;
+    a.A[0] = mat(dae, h, Cr, E);
+    a.B[0] = mat(w->w1, dl, h, E);
+    a.K[0] = h;
+    a.A[1] = mat(dbe, h, Cr, E);
+    a.B[1] = mat(w->w3, dl, h, E);
+    a.K[1] = h;
+    a.m_fastest = true;
+    a.out = dxe;
+    a.ldo = dl;
+    a.out_gs = Cr * dl;
+    MOE_TRY(gemm_run(a, st));
+  }
+  {
+    ProfScope ps("bwd.experts_wgrad_gate_up", st);
+    GemmArgs a;
+    a.a_mn = a.b_mn = true;
+    a.M = static_cast<int>(h);
+    a.N = static_cast<int>(dl);
+    a.groups = p->E;
+    a.ragged = 2;
+    a.group_rows = c.rows;
+    a.A[0] = mat(dae, h, Cr, E);
+    a.B[0] = mat(c.xe, dl, Cr, E);
+    a.m_fastest = true;
+    a.out = gr->w1;
+    a.ldo = dl;
+    a.out_gs = h * dl;
+    MOE_TRY(gemm_run(a, st));
+    a.A[0] = mat(dbe, h, Cr, E);
+    a.out = gr->w3;
+    MOE_TRY(gemm_run(a, st));
+  }
+  // un-dispatch and the softmax backward to the logits
+  {
+    ProfScope ps("bwd.undispatch", st);
+    MOE_TRY(launch_undispatch(g, dxe, c.gate, dg, c.idx, c.slot, dzr, dlog, st));
+  }
+  // dz = dlogits W_r + dz_routed;  dW_r = dlogits^T z
+  {
+    ProfScope ps("bwd.router_dgrad", st);
+    GemmArgs a;
+    a.b_mn = true;
+    a.epi = EPI_BF16_ADD_F32;
+    a.M = g.T;
+    a.N = static_cast<int>(dl);
+    a.A[0] = mat(dlog, E, T);
+    a.B[0] = mat(w->w_router, dl, E);
+    a.K[0] = E;
+    a.addend = dzr;
+    a.add_ld = dl;
+    a.out = dz;
+    a.ldo = dl;
+    MOE_TRY(gemm_run(a, st));
+  }
+  {
+    ProfScope ps("bwd.router_wgrad", st);
+    GemmArgs a;
+    a.a_mn = a.b_mn = true;
+    a.M = static_cast<int>(E);
+    a.N = static_cast<int>(dl);
+    a.A[0] = mat(dlog, E, T);
+    a.B[0] = mat(c.z, dl, T);
+    a.K[0] = T;
+    a.out = gr->w_router;
+    a.ldo = dl;
+    MOE_TRY(gemm_run(a, st));
+  }
+  // dx = dz W_down + dA_s ws1 + dB_s ws3 (three K segments)
+  {
+    ProfScope ps("bwd.dx", st);
+    GemmArgs a;
+    a.b_mn = true;
+    a.M = g.T;
+    a.N = static_cast<int>(dm);
+    a.nseg = 3;
+    a.A[0] = mat(dz, dl, T);
+    a.B[0] = mat(w->w_lat_down, dm, dl);
+    a.K[0] = dl;
+    a.A[1] = mat(das, SH, T);
+    a.B[1] = mat(w->ws1, dm, SH);
+    a.K[1] = SH;
+    a.A[2] = mat(dbs, SH, T);
+    a.B[2] = mat(w->ws3, dm, SH);
+    a.K[2] = SH;
+    a.out = dx;
+    a.ldo = dm;
+    MOE_TRY(gemm_run(a, st));
+  }
+  // dW_down = dz^T x,  dws1 = dA_s^T x,  dws3 = dB_s^T x
+  {
+    ProfScope ps("bwd.wgrad_lat_down_shared", st);
+    GemmArgs a;
+    a.a_mn = a.b_mn = true;
+    a.M = static_cast<int>(dl);
+    a.N = static_cast<int>(dm);
+    a.A[0] = mat(dz, dl, T);
+    a.B[0] = mat(x, dm, T);
+    a.K[0] = T;
+    a.out = gr->w_lat_down;
+    a.ldo = dm;
+    MOE_TRY(gemm_run(a, st));
+    a.M = static_cast<int>(SH);
+    a.A[0] = mat(das, SH, T);
+    a.out = gr->ws1;
+    MOE_TRY(gemm_run(a, st));
+    a.A[0] = mat(dbs, SH, T);
+    a.out = gr->ws3;
+    MOE_TRY(gemm_run(a, st));
+  }
+  (void)status;
+  return MOE_OK;
+}
+
+moe_status_t moe_bias_update(moe_plan_t p, const int32_t* hist, float* bias, float step, void* stream) {
+  if (p == nullptr || !hist || !bias) return fail(MOE_ERR_INVALID_ARG, "null argument");
+  MOE_TRY(device_ok());
+  ProfScope ps("bias_update", static_cast<cudaStream_t>(stream));
+  return launch_bias_update(p->g, hist, bias, step, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_gemm_bf16(int32_t M, int32_t N, int32_t K, const uint16_t* A, int32_t a_mn_major, const uint16_t* B,
+                           int32_t b_mn_major, void* D, int32_t d_f32, int32_t* status, void* stream) {
+  if (M <= 0 || N <= 0 || K <= 0) return fail(MOE_ERR_INVALID_ARG, "sizes must be positive");
+  if (!A || !B || !D) return fail(MOE_ERR_INVALID_ARG, "null buffer");
+  const int64_t a_inner = a_mn_major ? M : K, b_inner = b_mn_major ? N : K;
+  if (a_inner % 8 || b_inner % 8 || N % 8)
+    return fail(MOE_ERR_UNSUPPORTED, "contiguous dimensions and N must be multiples of 8");
+  MOE_TRY(device_ok());
+  GemmArgs a;
+  a.a_mn = a_mn_major != 0;
+  a.b_mn = b_mn_major != 0;
+  a.epi = d_f32 ? EPI_F32 : EPI_BF16;
+  a.M = M;
+  a.N = N;
+  a.A[0] = a.a_mn ? mat(A, M, K) : mat(A, K, M);
+  a.B[0] = a.b_mn ? mat(B, N, K) : mat(B, K, N);
+  a.K[0] = K;
+  a.out = D;
+  a.ldo = N;
+  a.status = status;
+  return gemm_run(a, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,750 @@
+// moe_kernels.cu -- routing, capacity-limited slot assignment and the HBM-bound data movement
+// of the MoE block (sm_100a).
+//
+//   route_topk      one warp per token: top-k of float32 logits + bias (ties to the lower
+//                   expert index), softmax gates of the chosen unbiased logits, load histogram
+//                   ("Marin 535B-A23B：一场完全公开的前沿 MoE 训练直播", §2.2)
+//   slot scan       deterministic two-level prefix scan in (token, rank) order: sender slot
+//                   per (destination, wave) pool capped at C_s, receiver slot per expert among
+//                   sender-kept rows capped at C_r ("Marin начинает открытое обучение
+//                   MoE-модели с 535 млрд параметров", §2: caps 1.10 / 1.15, drops counted
+//                   separately)
+//   pack            sender: z rows into the fixed pools with the expert id in a 16-byte row
+//                   header (same page, §2: one pool per receiving GPU, ids in the payload)
+//   unpack          receiver: reads only the pools; ranks rows of each local expert by the
+//                   packed id, keeps the first C_r, gathers them per expert
+//   combine         r_t = sum_j kept g_tj Y[e_tj][rslot_tj], fixed j order, fp32 accumulation
+//   combine_bwd     dY = g dr on kept rows, dg = <dr, Y>
+//   undispatch      dz_routed = sum_j kept dX, and the softmax backward to the logits
+//   bias_update     zero-mean sign step from the histogram
+// All data movement uses 16-byte vector loads and stores on row-contiguous data.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kMaxE = 1024;
+constexpr int kVals = kMaxE / 32;  // logits held per lane
+
+__device__ __forceinline__ bool better(float v, int e, float bv, int be) {
+  return v > bv || (v == bv && e < be);
+}
+
+// ---------------------------------------------------------------------- routing
+
+template <int VPL>
+__global__ void route_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E,
+                                  int k, int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
+                                  int32_t* __restrict__ hist, int32_t* __restrict__ nan_count) {
+  __shared__ int sh_hist[kMaxE];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) sh_hist[e] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  const int gw = blockIdx.x * warps + (threadIdx.x >> 5);
+  const int nw = gridDim.x * warps;
+  float bsv[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int e = i * 32 + lane;
+    bsv[i] = e < E ? bias[e] : 0.0f;
+  }
+  int nan_local = 0;
+  for (int t = gw; t < T; t += nw) {
+    const float* row = logits + static_cast<long long>(t) * E;
+    float raw[VPL], sc[VPL];
+    unsigned chosen = 0;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = i * 32 + lane;
+      raw[i] = e < E ? row[e] : 0.0f;
+      sc[i] = __fadd_rn(raw[i], bsv[i]);
+      if (e < E && isnan(sc[i])) {
+        ++nan_local;          // input error, counted; the expert ranks last
+        sc[i] = -INFINITY;
+      }
+    }
+    float my_raw = 0.0f;  // lane j < k keeps the raw logit of its rank-j choice
+    int my_e = 0;
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int e = i * 32 + lane;
+        if (e < E && !((chosen >> i) & 1u) && better(sc[i], e, bv, be)) {
+          bv = sc[i];
+          be = e;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+        if (better(ov, oe, bv, be)) {
+          bv = ov;
+          be = oe;
+        }
+      }
+      // be is now the same on every lane; its owner marks it and shares the raw logit
+      const int owner = be & 31;
+      const int slot = be >> 5;
+      float r = 0.0f;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        if (i == slot && lane == owner) {
+          chosen |= 1u << i;
+          r = raw[i];
+        }
+      r = __shfl_sync(0xffffffffu, r, owner);
+      if (lane == j) {
+        my_raw = r;
+        my_e = be;
+      }
+    }
+    // softmax over the k chosen raw logits (lanes 0..k-1)
+    float m = lane < k ? my_raw : -INFINITY;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    const float ex = lane < k ? expf(my_raw - m) : 0.0f;
+    float sum = ex;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane < k) {
+      idx_out[static_cast<long long>(t) * k + lane] = my_e;
+      gate_out[static_cast<long long>(t) * k + lane] = ex / sum;
+      if (my_e >= 0 && my_e < E) atomicAdd(&sh_hist[my_e], 1);
+    }
+  }
+  if (nan_local && nan_count != nullptr) atomicAdd(nan_count, nan_local);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    if (sh_hist[e]) atomicAdd(&hist[e], sh_hist[e]);
+}
+
+// ---------------------------------------------------------------------- slot scan
+//
+// Chunks of kScanTokensPerChunk tokens (their k assignments, in (t, j) order).
+//   A  count per chunk and pool                      cnt_pool[p][c]
+//   B  exclusive scan over chunks per pool            base_pool[p][c]
+//   C  sender slot = base + rank in chunk (warp-ordered); count sender-kept per expert
+//   D  exclusive scan over chunks per expert          base_exp[e][c]
+//   E  receiver slot = base + rank among kept in chunk; counters
+// Each per-chunk pass is one warp walking its chunk 32 assignments at a time, so the
+// ranks follow the visiting order exactly.
+
+__device__ __forceinline__ int pool_of(int e, int L, int P, int W) { return (e / L) * W + (e % L) / P; }
+
+__global__ void scan_count_pools(const int32_t* __restrict__ idx, int A_total, int chunk_assign, int n_chunks,
+                                 int L, int P, int W, int NP, int E, int32_t* __restrict__ cnt_pool) {
+  extern __shared__ int sh[];
+  const int c = blockIdx.x;
+  for (int p = threadIdx.x; p < NP; p += blockDim.x) sh[p] = 0;
+  __syncthreads();
+  const int a0 = c * chunk_assign;
+  const int a1 = min(A_total, a0 + chunk_assign);
+  for (int a = a0 + threadIdx.x; a < a1; a += blockDim.x) {
+    const int e = idx[a];
+    if (e >= 0 && e < E) atomicAdd(&sh[pool_of(e, L, P, W)], 1);
+  }
+  __syncthreads();
+  for (int p = threadIdx.x; p < NP; p += blockDim.x) cnt_pool[static_cast<long long>(p) * n_chunks + c] = sh[p];
+}
+
+// exclusive scan of each row of a [rows][n] int array, one block per row; writes the
+// row total to totals[row] (optional), clamped at cap into clamp_out[row] (optional)
+__global__ void scan_rows(int32_t* __restrict__ data, int n, int32_t* __restrict__ totals, int cap,
+                          int32_t* __restrict__ clamp_out) {
+  __shared__ int warp_tot[32];
+  __shared__ int carry;
+  int32_t* row = data + static_cast<long long>(blockIdx.x) * n;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < n; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    const int v = i < n ? row[i] : 0;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int before = carry;
+    for (int w = 0; w < warp; ++w) before += warp_tot[w];
+    if (i < n) row[i] = before + incl - v;
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) carry = before + incl;
+    __syncthreads();
+    (void)nwarp;
+  }
+  if (threadIdx.x == 0) {
+    if (totals) totals[blockIdx.x] = carry;
+    if (clamp_out) clamp_out[blockIdx.x] = carry < cap ? carry : cap;
+  }
+}
+
+// pass C: one warp per chunk
+__global__ void scan_sender_slots(const int32_t* __restrict__ idx, int A_total, int chunk_assign, int n_chunks,
+                                  int L, int P, int W, int NP, int E, int Cs,
+                                  const int32_t* __restrict__ base_pool, int32_t* __restrict__ slot,
+                                  int32_t* __restrict__ cnt_exp, int32_t* __restrict__ status) {
+  extern __shared__ int sh[];  // per warp: NP running counters + E kept counters
+  const int lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
+  const int c = blockIdx.x * (blockDim.x >> 5) + wib;
+  int* run = sh + wib * (NP + E);
+  int* kept = run + NP;
+  for (int i = lane; i < NP + E; i += 32) run[i] = 0;
+  __syncwarp();
+  if (c >= n_chunks) return;
+  const int a0 = c * chunk_assign;
+  const int a1 = min(A_total, a0 + chunk_assign);
+  for (int it = a0; it < a1; it += 32) {
+    const int a = it + lane;
+    const int e_raw = a < a1 ? idx[a] : 0;
+    const bool bad = a < a1 && (e_raw < 0 || e_raw >= E);
+    if (bad) {
+      atomicCAS(status, 0, MOE_ERR_INVALID_ARG);
+      slot[2LL * a] = -1;
+    }
+    const bool valid = a < a1 && !bad;
+    const int e = valid ? e_raw : 0;
+    const int p = valid ? pool_of(e, L, P, W) : -1 - lane;
+    const unsigned act = __ballot_sync(0xffffffffu, valid);
+    const unsigned peers = __match_any_sync(0xffffffffu, p) & act;
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    int s = -1;
+    if (valid) {
+      s = base_pool[static_cast<long long>(p) * n_chunks + c] + run[p] + rank;
+    }
+    __syncwarp();
+    if (valid && rank == __popc(peers) - 1) run[p] += __popc(peers);  // last of its group
+    if (valid) {
+      const bool sk = s < Cs;
+      slot[2LL * a] = sk ? s : -1;
+      if (sk) atomicAdd(&kept[e], 1);
+    }
+    __syncwarp();
+  }
+  __syncwarp();
+  for (int e = lane; e < E; e += 32) cnt_exp[static_cast<long long>(e) * n_chunks + c] = kept[e];
+}
+
+// pass E: one warp per chunk
+__global__ void scan_receiver_slots(const int32_t* __restrict__ idx, int A_total, int chunk_assign, int n_chunks,
+                                    int E, int Cr, const int32_t* __restrict__ base_exp,
+                                    int32_t* __restrict__ slot, int32_t* __restrict__ stats_kept_e,
+                                    int32_t* __restrict__ stats_ds_e, int32_t* __restrict__ stats_dr_e) {
+  extern __shared__ int sh[];  // per warp: E running counters
+  const int lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
+  const int c = blockIdx.x * (blockDim.x >> 5) + wib;
+  int* run = sh + wib * E;
+  for (int i = lane; i < E; i += 32) run[i] = 0;
+  __syncwarp();
+  if (c >= n_chunks) return;
+  const int a0 = c * chunk_assign;
+  const int a1 = min(A_total, a0 + chunk_assign);
+  for (int it = a0; it < a1; it += 32) {
+    const int a = it + lane;
+    const int e_raw = a < a1 ? idx[a] : 0;
+    const bool valid = a < a1 && e_raw >= 0 && e_raw < E;
+    const int e = valid ? e_raw : 0;
+    const bool sk = valid && slot[2LL * a] >= 0;
+    const int key = sk ? e : -1 - lane;
+    const unsigned act = __ballot_sync(0xffffffffu, sk);
+    const unsigned peers = __match_any_sync(0xffffffffu, key) & act;
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    int r = -1;
+    if (sk) r = base_exp[static_cast<long long>(e) * n_chunks + c] + run[e] + rank;
+    __syncwarp();
+    if (sk && rank == __popc(peers) - 1) run[e] += __popc(peers);
+    if (a < a1 && !valid) slot[2LL * a + 1] = -1;
+    if (valid) {
+      const bool rk = sk && r < Cr;
+      slot[2LL * a + 1] = rk ? r : -1;
+      if (rk) atomicAdd(&stats_kept_e[e], 1);
+      else if (sk) atomicAdd(&stats_dr_e[e], 1);
+      else atomicAdd(&stats_ds_e[e], 1);
+    }
+    __syncwarp();
+  }
+}
+
+// totals and maxima from the per-expert / per-pool counters (one block)
+__global__ void scan_totals(int32_t* __restrict__ stats, int E, int NP, int A_total, int off_kept, int off_ds,
+                            int off_dr, int off_fill) {
+  __shared__ int s_kept, s_ds, s_dr, s_mp, s_me;
+  if (threadIdx.x == 0) s_kept = s_ds = s_dr = s_mp = s_me = 0;
+  __syncthreads();
+  int k = 0, ds = 0, dr = 0, me = 0, mp = 0;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    k += stats[off_kept + e];
+    ds += stats[off_ds + e];
+    dr += stats[off_dr + e];
+    me = max(me, stats[off_kept + e]);
+  }
+  for (int p = threadIdx.x; p < NP; p += blockDim.x) mp = max(mp, stats[off_fill + p]);
+  atomicAdd(&s_kept, k);
+  atomicAdd(&s_ds, ds);
+  atomicAdd(&s_dr, dr);
+  atomicMax(&s_me, me);
+  atomicMax(&s_mp, mp);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    stats[0] = s_kept;
+    stats[1] = s_ds;
+    stats[2] = s_dr;
+    stats[4] = s_mp;
+    stats[5] = s_me;
+    stats[6] = A_total;
+  }
+}
+
+// ---------------------------------------------------------------------- pack / unpack
+
+// one warp per token: read z_t once, write it into every pool row it was given
+__global__ void pack_kernel(const uint16_t* __restrict__ z, const int32_t* __restrict__ idx,
+                            const int32_t* __restrict__ slot, int T, int k, int dl, int L, int P, int W, int Cs,
+                            int E, uint16_t* __restrict__ pools) {
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  const long long row_elems = dl + 8;
+  const int nvec = dl / 8;
+  for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += gridDim.x * warps) {
+    int e_j = -1, s_j = -1;
+    if (lane < k) {
+      e_j = idx[static_cast<long long>(t) * k + lane];
+      s_j = slot[2LL * (static_cast<long long>(t) * k + lane)];
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(z + static_cast<long long>(t) * dl);
+    for (int v = lane; v < nvec; v += 32) {
+      const uint4 val = src[v];
+      for (int j = 0; j < k; ++j) {
+        const int e = __shfl_sync(0xffffffffu, e_j, j);
+        const int s = __shfl_sync(0xffffffffu, s_j, j);
+        if (s >= 0 && s < Cs && e >= 0 && e < E) {
+          uint16_t* dst = pools + (static_cast<long long>(pool_of(e, L, P, W)) * Cs + s) * row_elems;
+          reinterpret_cast<uint4*>(dst)[v] = val;
+        }
+      }
+    }
+    if (lane < k && s_j >= 0 && s_j < Cs && e_j >= 0 && e_j < E) {
+      uint16_t* dst = pools + (static_cast<long long>(pool_of(e_j, L, P, W)) * Cs + s_j) * row_elems + dl;
+      *reinterpret_cast<int4*>(dst) = make_int4(e_j, 0, 0, 0);
+    }
+  }
+}
+
+// header -1 for the rows of each pool past its fill
+__global__ void pack_empty_headers(const int32_t* __restrict__ pool_fill, int NP, int Cs, int dl,
+                                   uint16_t* __restrict__ pools) {
+  const long long row_elems = dl + 8;
+  const long long total = static_cast<long long>(NP) * Cs;
+  for (long long r = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; r < total;
+       r += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int p = static_cast<int>(r / Cs);
+    const int s = static_cast<int>(r % Cs);
+    if (s >= pool_fill[p]) *reinterpret_cast<int4*>(pools + r * row_elems + dl) = make_int4(-1, 0, 0, 0);
+  }
+}
+
+// receiver: one block per pool.  Rows are visited in pool order in tiles of the block
+// size; a row whose packed id names local expert q of this pool gets the next slot of
+// q; the first C_r rows of each expert are gathered into xe[e][slot].
+__global__ void unpack_kernel(const uint16_t* __restrict__ pools, int Cs, int Cr, int dl, int L, int P, int W,
+                              uint16_t* __restrict__ xe, int32_t* __restrict__ rows_out,
+                              int32_t* __restrict__ status) {
+  constexpr int kTile = 256;
+  __shared__ int s_slot[kTile];
+  __shared__ int s_exp[kTile];
+  __shared__ int s_warp_cnt[kTile / 32][32];
+  __shared__ int s_run[32];
+  const int pool = blockIdx.x;
+  const int dest = pool / W, wave = pool % W;
+  const int e_first = dest * L + wave * P;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long long row_elems = dl + 8;
+  if (threadIdx.x < 32) s_run[threadIdx.x] = 0;
+  __syncthreads();
+  const uint16_t* pbase = pools + static_cast<long long>(pool) * Cs * row_elems;
+  for (int r0 = 0; r0 < Cs; r0 += kTile) {
+    const int r = r0 + threadIdx.x;
+    int q = -1;
+    if (r < Cs) {
+      const int e = *reinterpret_cast<const int*>(pbase + r * row_elems + dl);
+      if (e >= 0) {
+        if (e >= e_first && e < e_first + P) q = e - e_first;
+        else atomicCAS(status, 0, MOE_ERR_INVALID_ARG);  // an id this pool cannot hold
+      }
+    }
+    // rank of this row among the tile's rows of the same local expert, in row order
+    int rank = 0;
+    for (int qq = 0; qq < P; ++qq) {
+      const unsigned m = __ballot_sync(0xffffffffu, q == qq);
+      if (q == qq) rank = __popc(m & ((1u << lane) - 1u));
+      if (lane == 0) s_warp_cnt[warp][qq] = __popc(m);
+    }
+    __syncthreads();
+    int slot = -1;
+    if (q >= 0) {
+      int before = s_run[q];
+      for (int w = 0; w < warp; ++w) before += s_warp_cnt[w][q];
+      slot = before + rank;
+    }
+    s_slot[threadIdx.x] = (slot >= 0 && slot < Cr) ? slot : -1;
+    s_exp[threadIdx.x] = q >= 0 ? e_first + q : -1;
+    __syncthreads();
+    if (threadIdx.x < P) {
+      int tot = 0;
+      for (int w = 0; w < kTile / 32; ++w) tot += s_warp_cnt[w][threadIdx.x];
+      s_run[threadIdx.x] += tot;
+    }
+    // gather the kept rows of this tile: one warp per row
+    const int nvec = dl / 8;
+    for (int i = warp; i < kTile && r0 + i < Cs; i += kTile / 32) {
+      const int sl = s_slot[i];
+      if (sl < 0) continue;
+      const uint4* src = reinterpret_cast<const uint4*>(pbase + (r0 + i) * row_elems);
+      uint4* dst = reinterpret_cast<uint4*>(xe + (static_cast<long long>(s_exp[i]) * Cr + sl) * dl);
+      for (int v = lane; v < nvec; v += 32) dst[v] = src[v];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x < P) rows_out[e_first + threadIdx.x] = min(s_run[threadIdx.x], Cr);
+}
+
+// rows [n_e, min(round_up(n_e, 128), C_r)) of each expert's buffer become zero, so that
+// the GEMM tiles that cover them read zeros
+__global__ void zero_tail_rows_kernel(uint16_t* __restrict__ buf, long long width, int Cr,
+                                      const int32_t* __restrict__ rows) {
+  const int e = blockIdx.y;
+  const int n = rows[e];
+  const int end = min(((n + 127) / 128) * 128, Cr);
+  const long long nvec = width / 8;
+  const long long total = static_cast<long long>(end - n) * nvec;
+  uint4* base = reinterpret_cast<uint4*>(buf + (static_cast<long long>(e) * Cr + n) * width);
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    base[i] = make_uint4(0, 0, 0, 0);
+}
+
+// ---------------------------------------------------------------------- combine and its backward
+
+__device__ __forceinline__ void acc8(float (&acc)[8], const uint4& v, float g) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc[2 * i] = fmaf(g, __uint_as_float(w[i] << 16), acc[2 * i]);
+    acc[2 * i + 1] = fmaf(g, __uint_as_float(w[i] & 0xFFFF0000u), acc[2 * i + 1]);
+  }
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&a)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(a[2 * i], a[2 * i + 1]);
+    w[i] = *reinterpret_cast<uint32_t*>(&v);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__global__ void combine_kernel(const uint16_t* __restrict__ ye, const float* __restrict__ gate,
+                               const int32_t* __restrict__ idx, const int32_t* __restrict__ slot, int T, int k,
+                               int dl, int Cr, int E, uint16_t* __restrict__ r) {
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  const int nvec = dl / 8;
+  for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += gridDim.x * warps) {
+    float g_j = 0.0f;
+    long long row_j = -1;
+    if (lane < k) {
+      const long long a = static_cast<long long>(t) * k + lane;
+      const int rs = slot[2 * a + 1];
+      const int e = idx[a];
+      if (rs >= 0 && rs < Cr && e >= 0 && e < E) {
+        g_j = gate[a];
+        row_j = static_cast<long long>(e) * Cr + rs;
+      }
+    }
+    for (int v = lane; v < nvec; v += 32) {
+      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      for (int j = 0; j < k; ++j) {
+        const long long rj = __shfl_sync(0xffffffffu, row_j, j);
+        const float gj = __shfl_sync(0xffffffffu, g_j, j);
+        if (rj >= 0) acc8(acc, reinterpret_cast<const uint4*>(ye + rj * dl)[v], gj);
+      }
+      reinterpret_cast<uint4*>(r + static_cast<long long>(t) * dl)[v] = pack8(acc);
+    }
+  }
+}
+
+__global__ void combine_bwd_kernel(const uint16_t* __restrict__ dr, const uint16_t* __restrict__ ye,
+                                   const float* __restrict__ gate, const int32_t* __restrict__ idx,
+                                   const int32_t* __restrict__ slot, int T, int k, int dl, int Cr, int E,
+                                   uint16_t* __restrict__ dye, float* __restrict__ dg) {
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  const int nvec = dl / 8;
+  for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += gridDim.x * warps) {
+    const uint4* drow = reinterpret_cast<const uint4*>(dr + static_cast<long long>(t) * dl);
+    for (int j = 0; j < k; ++j) {
+      const long long a = static_cast<long long>(t) * k + j;
+      const int rs_raw = slot[2 * a + 1];
+      const int e = idx[a];
+      const int rs = (rs_raw < Cr && e >= 0 && e < E) ? rs_raw : -1;
+      float dot = 0.0f;
+      if (rs >= 0) {
+        const float g = gate[a];
+        const long long rowo = (static_cast<long long>(e) * Cr + rs) * dl;
+        const uint4* yrow = reinterpret_cast<const uint4*>(ye + rowo);
+        uint4* out = reinterpret_cast<uint4*>(dye + rowo);
+        for (int v = lane; v < nvec; v += 32) {
+          const uint4 d = drow[v];
+          const uint4 y = yrow[v];
+          const uint32_t dw[4] = {d.x, d.y, d.z, d.w};
+          const uint32_t yw[4] = {y.x, y.y, y.z, y.w};
+          float o[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float d0 = __uint_as_float(dw[i] << 16), d1 = __uint_as_float(dw[i] & 0xFFFF0000u);
+            const float y0 = __uint_as_float(yw[i] << 16), y1 = __uint_as_float(yw[i] & 0xFFFF0000u);
+            dot = fmaf(d0, y0, dot);
+            dot = fmaf(d1, y1, dot);
+            o[2 * i] = g * d0;
+            o[2 * i + 1] = g * d1;
+          }
+          out[v] = pack8(o);
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+      if (lane == 0) dg[a] = rs >= 0 ? dot : 0.0f;
+    }
+  }
+}
+
+// dz_routed_t = sum_j kept dX[e_tj][rslot_tj]; dlogits_t = softmax backward over the
+// chosen experts, zero elsewhere
+__global__ void undispatch_kernel(const uint16_t* __restrict__ dxe, const float* __restrict__ gate,
+                                  const float* __restrict__ dg, const int32_t* __restrict__ idx,
+                                  const int32_t* __restrict__ slot, int T, int k, int dl, int Cr, int E,
+                                  float* __restrict__ dz, uint16_t* __restrict__ dlogits) {
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  const int nvec = dl / 8;
+  for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += gridDim.x * warps) {
+    long long row_j = -1;
+    float g_j = 0.0f, dg_j = 0.0f;
+    int e_j = -1;
+    if (lane < k) {
+      const long long a = static_cast<long long>(t) * k + lane;
+      const int rs = slot[2 * a + 1];
+      e_j = idx[a];
+      g_j = gate[a];
+      dg_j = dg[a];
+      if (e_j < 0 || e_j >= E) e_j = -1;
+      if (rs >= 0 && rs < Cr && e_j >= 0) row_j = static_cast<long long>(e_j) * Cr + rs;
+    }
+    for (int v = lane; v < nvec; v += 32) {
+      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      for (int j = 0; j < k; ++j) {
+        const long long rj = __shfl_sync(0xffffffffu, row_j, j);
+        if (rj >= 0) acc8(acc, reinterpret_cast<const uint4*>(dxe + rj * dl)[v], 1.0f);
+      }
+      float4* o = reinterpret_cast<float4*>(dz + static_cast<long long>(t) * dl + 8 * v);
+      o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
+    // softmax backward: dl_j = g_j (dg_j - sum_i g_i dg_i)
+    float s = lane < k ? g_j * dg_j : 0.0f;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    uint16_t* drow = dlogits + static_cast<long long>(t) * E;
+    for (int e = lane; e < E; e += 32) drow[e] = 0;
+    __syncwarp();
+    if (lane < k && e_j >= 0) {
+      const float d = g_j * (dg_j - s);
+      __nv_bfloat16 b = __float2bfloat16_rn(d);
+      drow[e_j] = *reinterpret_cast<uint16_t*>(&b);
+    }
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------------- bias step
+
+__global__ void bias_update_kernel(const int32_t* __restrict__ hist, float* __restrict__ bias, int E, long long Tk,
+                                   float step) {
+  __shared__ int warp_sum[32];
+  const int e = threadIdx.x;
+  int sgn = 0;
+  if (e < E) {
+    const long long load = static_cast<long long>(E) * hist[e];
+    sgn = (Tk > load) - (Tk < load);
+  }
+  int s = sgn;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if ((threadIdx.x & 31) == 0) warp_sum[threadIdx.x >> 5] = s;
+  __syncthreads();
+  int total = 0;
+  for (int w = 0; w < (blockDim.x + 31) / 32; ++w) total += warp_sum[w];
+  if (e < E) {
+    const float mean = __fdiv_rn(static_cast<float>(total), static_cast<float>(E));
+    const float delta = __fsub_rn(static_cast<float>(sgn), mean);
+    bias[e] = __fadd_rn(bias[e], __fmul_rn(step, delta));
+  }
+}
+
+int blocks_for(long long work, int per_block) {
+  long long b = (work + per_block - 1) / per_block;
+  const long long cap = 8LL * device_sm_count();
+  if (b > cap) b = cap;
+  return static_cast<int>(b < 1 ? 1 : b);
+}
+
+}  // namespace
+
+// ====================================================================== launchers
+
+moe_status_t launch_route(const Geo& g, const float* logits, const float* bias, int32_t* idx, float* gate,
+                          int32_t* hist, int32_t* nan_count, cudaStream_t st) {
+  if (g.T == 0) return MOE_OK;
+  const int warps = 8;
+  const int grid = blocks_for(g.T, warps);
+  const int vpl = (g.E + 31) / 32;
+#define MOE_ROUTE(V)                                                                                       \
+  if (vpl <= V) {                                                                                          \
+    route_topk_kernel<V><<<grid, 32 * warps, 0, st>>>(logits, bias, g.T, g.E, g.k, idx, gate, hist, nan_count); \
+    count_launch();                                                                                          \
+    return cuda_check(cudaGetLastError(), "route_topk");                                                    \
+  }
+  MOE_ROUTE(1)
+  MOE_ROUTE(2)
+  MOE_ROUTE(4)
+  MOE_ROUTE(8)
+  MOE_ROUTE(12)
+  MOE_ROUTE(16)
+  MOE_ROUTE(32)
+#undef MOE_ROUTE
+  return fail(MOE_ERR_UNSUPPORTED, "too many experts for the router kernel");
+}
+
+size_t scan_scratch_ints(const Geo& g) {
+  return static_cast<size_t>(g.n_chunks) * (g.NP + g.E) + g.NP;
+}
+
+moe_status_t launch_slot_scan(const Geo& g, const int32_t* idx, int32_t* slot, int32_t* stats, int32_t* scratch,
+                              cudaStream_t st) {
+  const int A = g.T * g.k;
+  const int chunk_assign = kScanTokensPerChunk * g.k;
+  int32_t* cnt_pool = scratch;                                        // [NP][n_chunks]
+  int32_t* cnt_exp = scratch + static_cast<size_t>(g.n_chunks) * g.NP;  // [E][n_chunks]
+  int32_t* pool_tot = cnt_exp + static_cast<size_t>(g.n_chunks) * g.E;  // [NP]
+  // counters of this call start at zero (hist is left to the router)
+  cudaError_t e = cudaMemsetAsync(stats + stats_kept_e(g), 0, sizeof(int32_t) * 3 * g.E, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(stats, 0, sizeof(int32_t) * 3, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(stats + 4, 0, sizeof(int32_t) * 3, st);
+  if (e != cudaSuccess) return cuda_check(e, "slot scan memset");
+  if (A == 0) {
+    e = cudaMemsetAsync(stats + stats_pool_fill(g), 0, sizeof(int32_t) * g.NP, st);
+    return cuda_check(e, "slot scan memset");
+  }
+  scan_count_pools<<<g.n_chunks, 256, g.NP * sizeof(int), st>>>(idx, A, chunk_assign, g.n_chunks, g.L, g.P, g.W,
+                                                                 g.NP, g.E, cnt_pool);
+  scan_rows<<<g.NP, 256, 0, st>>>(cnt_pool, g.n_chunks, pool_tot, g.Cs, stats + stats_pool_fill(g));
+  const int wpb = 4;
+  const int grid = (g.n_chunks + wpb - 1) / wpb;
+  scan_sender_slots<<<grid, 32 * wpb, wpb * (g.NP + g.E) * sizeof(int), st>>>(
+      idx, A, chunk_assign, g.n_chunks, g.L, g.P, g.W, g.NP, g.E, g.Cs, cnt_pool, slot, cnt_exp, stats + 3);
+  scan_rows<<<g.E, 256, 0, st>>>(cnt_exp, g.n_chunks, nullptr, 0, nullptr);
+  scan_receiver_slots<<<grid, 32 * wpb, wpb * g.E * sizeof(int), st>>>(
+      idx, A, chunk_assign, g.n_chunks, g.E, g.Cr, cnt_exp, slot, stats + stats_kept_e(g), stats + stats_ds_e(g),
+      stats + stats_dr_e(g));
+  scan_totals<<<1, 256, 0, st>>>(stats, g.E, g.NP, A, stats_kept_e(g), stats_ds_e(g), stats_dr_e(g),
+                                 stats_pool_fill(g));
+  count_launch(6);
+  return cuda_check(cudaGetLastError(), "slot scan");
+}
+
+moe_status_t launch_pack(const Geo& g, const uint16_t* z, const int32_t* idx, const int32_t* slot,
+                         const int32_t* stats, uint16_t* pools, cudaStream_t st) {
+  if (g.T > 0) {
+    const int warps = 8;
+    pack_kernel<<<blocks_for(g.T, warps), 32 * warps, 0, st>>>(z, idx, slot, g.T, g.k, g.dl, g.L, g.P, g.W, g.Cs,
+                                                               g.E, pools);
+    count_launch();
+  }
+  const long long rows = static_cast<long long>(g.NP) * g.Cs;
+  if (rows > 0)
+  {
+    pack_empty_headers<<<blocks_for(rows, 256), 256, 0, st>>>(stats + stats_pool_fill(g), g.NP, g.Cs, g.dl, pools);
+    count_launch();
+  }
+  return cuda_check(cudaGetLastError(), "pack");
+}
+
+moe_status_t launch_unpack(const Geo& g, const uint16_t* pools, uint16_t* xe, int32_t* rows, int32_t* status,
+                           cudaStream_t st) {
+  if (g.P > 32) return fail(MOE_ERR_UNSUPPORTED, "more than 32 experts per wave");
+  unpack_kernel<<<g.NP, 256, 0, st>>>(pools, g.Cs, g.Cr, g.dl, g.L, g.P, g.W, xe, rows, status);
+  count_launch();
+  return cuda_check(cudaGetLastError(), "unpack");
+}
+
+moe_status_t launch_zero_tail_rows(const Geo& g, uint16_t* buf, int64_t width, const int32_t* rows,
+                                   cudaStream_t st) {
+  dim3 grid(4, g.E);
+  zero_tail_rows_kernel<<<grid, 256, 0, st>>>(buf, width, g.Cr, rows);
+  count_launch();
+  return cuda_check(cudaGetLastError(), "zero tail rows");
+}
+
+moe_status_t launch_combine(const Geo& g, const uint16_t* ye, const float* gate, const int32_t* idx,
+                            const int32_t* slot, uint16_t* r, cudaStream_t st) {
+  if (g.T == 0) return MOE_OK;
+  const int warps = 8;
+  combine_kernel<<<blocks_for(g.T, warps), 32 * warps, 0, st>>>(ye, gate, idx, slot, g.T, g.k, g.dl, g.Cr, g.E, r);
+  count_launch();
+  return cuda_check(cudaGetLastError(), "combine");
+}
+
+moe_status_t launch_combine_bwd(const Geo& g, const uint16_t* dr, const uint16_t* ye, const float* gate,
+                                const int32_t* idx, const int32_t* slot, uint16_t* dye, float* dg,
+                                cudaStream_t st) {
+  if (g.T == 0) return MOE_OK;
+  const int warps = 8;
+  combine_bwd_kernel<<<blocks_for(g.T, warps), 32 * warps, 0, st>>>(dr, ye, gate, idx, slot, g.T, g.k, g.dl,
+                                                                    g.Cr, g.E, dye, dg);
+  count_launch();
+  return cuda_check(cudaGetLastError(), "combine_bwd");
+}
+
+moe_status_t launch_undispatch(const Geo& g, const uint16_t* dxe, const float* gate, const float* dg,
+                               const int32_t* idx, const int32_t* slot, float* dz_routed, uint16_t* dlogits,
+                               cudaStream_t st) {
+  if (g.T == 0) return MOE_OK;
+  const int warps = 8;
+  undispatch_kernel<<<blocks_for(g.T, warps), 32 * warps, 0, st>>>(dxe, gate, dg, idx, slot, g.T, g.k, g.dl, g.Cr,
+                                                                   g.E, dz_routed, dlogits);
+  count_launch();
+  return cuda_check(cudaGetLastError(), "undispatch");
+}
+
+moe_status_t launch_bias_update(const Geo& g, const int32_t* hist, float* bias, float step, cudaStream_t st) {
+  const int threads = ((g.E + 31) / 32) * 32;
+  bias_update_kernel<<<1, threads, 0, st>>>(hist, bias, g.E, static_cast<long long>(g.T) * g.k, step);
+  count_launch();
+  return cuda_check(cudaGetLastError(), "bias_update");
+}
+
+}  // namespace moe

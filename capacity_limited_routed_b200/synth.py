@@ -194,3 +194,59 @@ def make_logits(T: int, E: int, seed: int, ties: bool = False) -> np.ndarray:
         v[neg_zero] = np.float32(-0.0)
         return v
     return rng.standard_normal(size=(T, E), dtype=np.float32)
+
+
+# ------------------------------------------------------------------ device-side generation
+#
+# Full-width workloads carry 22 GB of expert weights; drawing them with numpy on the
+# host takes minutes.  For those the same recipe (N(0, 1/fan_in) weights, N(0, 1)
+# tokens, windowed correlation, Zipf logit skew) is drawn with PyTorch's seeded CUDA
+# generator instead.  Tensor i of a workload uses seed (1000003 * seed + i), so any
+# one tensor can be regenerated on its own.
+
+
+def _dev_normal(shape, std, seed, device):
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    out = torch.empty(shape, dtype=torch.bfloat16, device=device)
+    # draw in slabs to bound the float32 temporary
+    flat = out.view(-1)
+    step = 1 << 28
+    for lo in range(0, flat.numel(), step):
+        hi = min(flat.numel(), lo + step)
+        flat[lo:hi] = (torch.randn(hi - lo, generator=g, device=device, dtype=torch.float32) * std).to(torch.bfloat16)
+    return out
+
+
+def make_inputs_device(shape: MoEShape, device="cuda", seed: int | None = None) -> dict:
+    """Same keys as ``make_inputs`` but bf16 / float32 tensors on ``device``."""
+    import torch
+    s = shape
+    base = (shape.seed if seed is None else seed) * 1000003
+    dm, dl, E, h, S, hs = s.d_model, s.d_latent, s.n_experts, s.hidden_routed, s.n_shared, s.hidden_shared
+    spec = [("w_lat_down", (dl, dm), dm), ("w_router", (E, dl), dl), ("w1", (E, h, dl), dl),
+            ("w3", (E, h, dl), dl), ("w2", (E, dl, h), h), ("w_lat_up", (dm, dl), dl),
+            ("ws1", (S * hs, dm), dm), ("ws3", (S * hs, dm), dm), ("ws2", (dm, S * hs), hs)]
+    weights = {n: _dev_normal(shp, 1.0 / math.sqrt(fan), base + i, device) for i, (n, shp, fan) in enumerate(spec)}
+    if s.window and s.rho > 0.0:
+        n_win = (s.T + s.window - 1) // s.window
+        gwin = _dev_normal((n_win, dm), 1.0, base + 20, device).float()
+        eps = _dev_normal((s.T, dm), 1.0, base + 21, device)
+        x = torch.empty((s.T, dm), dtype=torch.bfloat16, device=device)
+        a, b = math.sqrt(s.rho), math.sqrt(1.0 - s.rho)
+        for wi in range(n_win):
+            lo, hi = wi * s.window, min(s.T, (wi + 1) * s.window)
+            x[lo:hi] = (a * gwin[wi][None, :] + b * eps[lo:hi].float()).to(torch.bfloat16)
+    else:
+        x = _dev_normal((s.T, dm), 1.0, base + 21, device)
+    lo_ = make_logit_offset(s)
+    out = {
+        "x": x,
+        "weights": weights,
+        "bias": torch.zeros(E, dtype=torch.float32, device=device),
+        "logit_offset": None if lo_ is None else torch.from_numpy(lo_).to(device),
+    }
+    if s.backward:
+        out["dy"] = _dev_normal((s.T, dm), 1.0, base + 22, device)
+    return out

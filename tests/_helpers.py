@@ -1,0 +1,45 @@
+"""Shared helpers of the GPU tests: device upload, tolerances, bf16 bit handling."""
+import numpy as np
+import torch
+
+# Floating-point bar of the block: max |gpu - oracle| <= 2e-2 * RMS(oracle) per tensor
+# (bf16 storage, float32 accumulation).
+REL_TOL = 2e-2
+
+
+def dev():
+    return torch.device("cuda:0")
+
+
+def bf16_dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev()).to(torch.bfloat16)
+
+
+def f32_dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev())
+
+
+def i32_dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev())
+
+
+def host64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def rms(a):
+    a = np.asarray(a, dtype=np.float64)
+    return float(np.sqrt(np.mean(a * a))) if a.size else 0.0
+
+
+def assert_close_rms(got, want, tol=REL_TOL, what=""):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    assert got.shape == want.shape, (what, got.shape, want.shape)
+    if want.size == 0:
+        return 0.0
+    err = float(np.max(np.abs(got - want)))
+    scale = rms(want)
+    assert np.isfinite(got).all(), f"{what}: non-finite values"
+    assert err <= tol * scale + 1e-30, f"{what}: max|err| {err:.3e} > {tol} * rms {scale:.3e}"
+    return err / scale if scale else 0.0

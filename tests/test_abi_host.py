@@ -1,0 +1,103 @@
+"""Host-side checks of libmoe that need no GPU: the library loads, exports every symbol
+include/moe.h declares, computes the same capacities as the oracle, and rejects bad
+arguments with status codes (never by crashing)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from capacity_limited_routed_b200 import synth
+from oracle import moe_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def M():
+    from capacity_limited_routed_b200 import moe
+    return moe
+
+
+def test_header_and_binding_agree_on_exports(M):
+    with open(os.path.join(ROOT, "include", "moe.h"), encoding="utf-8") as f:
+        hdr = f.read()
+    declared = set(re.findall(r"^MOE_API\s+(?:moe_status_t|const char\*|int64_t)\s+(moe_\w+)\s*\(", hdr, re.M))
+    assert declared == set(M.EXPORTS)
+    lib = ctypes.CDLL(M.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+@pytest.mark.parametrize("wid", [1, 2, 3, 4, 5])
+def test_plan_capacities_match_oracle(M, wid):
+    s = synth.WORKLOADS[wid]
+    plan = M.Plan.from_shape(s)
+    g = O.geometry(s)
+    assert (plan.info.cap_send, plan.info.cap_recv) == (g.C_s, g.C_r)
+    assert plan.info.local_experts == g.L and plan.info.experts_per_wave == g.P
+    assert plan.info.n_pools == g.D * g.W
+    assert plan.info.pool_row_elems == s.d_latent + 8
+    assert plan.info.pools_bytes == g.D * g.W * g.C_s * (s.d_latent + 8) * 2
+    assert plan.info.expert_out_bytes == s.n_experts * g.C_r * s.d_latent * 2
+    assert plan.info.stats_bytes == 4 * (8 + 4 * s.n_experts + g.D * g.W)
+    assert plan.info.workspace_bytes % 256 == 0 and plan.info.saved_bytes % 256 == 0
+
+
+def test_plan_rejects_bad_shapes(M):
+    base = dict(T=64, d_model=128, d_latent=64, n_experts=24, top_k=2, n_dest=4, hidden_routed=128,
+                n_shared=1, hidden_shared=128)
+    M.Plan(**base)
+    bad = [
+        (dict(n_experts=25), M.STATUS[2]),            # E % D
+        (dict(n_dest=8), M.STATUS[2]),                # E/D = 3 = W but (E/D) % W ok? 24/8 = 3 -> P = 1: valid
+        (dict(d_model=100), M.STATUS[2]),
+        (dict(hidden_routed=64), M.STATUS[2]),
+        (dict(top_k=0), M.STATUS[1]),
+        (dict(top_k=33, n_experts=48, n_dest=4), M.STATUS[2]),
+        (dict(T=-1), M.STATUS[1]),
+    ]
+    for kw, _ in bad:
+        args = dict(base, **kw)
+        if kw == dict(n_dest=8):
+            M.Plan(**args)                            # 24 experts over 8 destinations of 3 waves is fine
+            continue
+        with pytest.raises(M.MoEError):
+            M.Plan(**args)
+    with pytest.raises(M.MoEError) as ei:
+        M.Plan(**dict(base, cap_send=(0, 100)))
+    assert ei.value.code == 1
+
+
+def test_empty_batch_plan(M):
+    p = M.Plan(T=0, d_model=128, d_latent=64, n_experts=24, top_k=2, n_dest=4, hidden_routed=128,
+               n_shared=1, hidden_shared=128)
+    assert p.info.cap_send >= 1 and p.info.cap_recv >= 1
+
+
+def test_compute_calls_fail_cleanly_without_a_device(M):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    p = M.Plan.from_shape(synth.TINY)
+    lib = M.lib()
+    fake = ctypes.c_void_p(0x1000)
+    code = lib.moe_route(p.handle, fake, fake, fake, fake, fake, None)
+    assert code == 2 and "device" in M.moe_last_error()
+    code = lib.moe_bias_update(p.handle, fake, fake, ctypes.c_float(1e-3), None)
+    assert code == 2
+    code = lib.moe_gemm_bf16(128, 128, 64, fake, 0, fake, 0, fake, 1, None, None)
+    assert code == 2
+
+
+def test_null_arguments_are_rejected(M):
+    p = M.Plan.from_shape(synth.TINY)
+    lib = M.lib()
+    assert lib.moe_route(p.handle, None, None, None, None, None, None) == 1
+    assert lib.moe_forward(p.handle, None, None, None, None, None, None, None, None, 0, None) == 1
+    w = M.moe_weights_t()
+    assert lib.moe_forward(p.handle, ctypes.byref(w), None, None, None, None, None, None, None, 0, None) == 1
+    assert lib.moe_gemm_bf16(0, 8, 8, None, 0, None, 0, None, 1, None, None) == 1
+    fake = ctypes.c_void_p(0x1000)
+    # too-small workspace is reported before anything runs
+    assert lib.moe_dispatch(p.handle, fake, fake, fake, fake, fake, fake, 16, None) == 3

@@ -1,0 +1,113 @@
+"""Whole forward and backward pass through moe_forward / moe_backward against the oracle.
+
+The GPU computes its own router logits, so a token whose float32 scores nearly tie
+can be routed differently from the oracle (float64 accumulation).  The rate of such
+routing mismatches is reported; outputs are compared on the tokens whose chosen
+experts and drop decisions agree, and weight gradients on the experts no mismatched
+token touches (all of them when nothing mismatches).
+"""
+import numpy as np
+import pytest
+import torch
+
+from _helpers import REL_TOL, assert_close_rms, bf16_dev, dev, host64
+from capacity_limited_routed_b200 import synth
+from oracle import moe_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+RAGGED = synth.MoEShape("ragged", T=333, d_model=192, d_latent=128, n_experts=48, top_k=3, n_dest=8,
+                        hidden_routed=256, n_shared=2, hidden_shared=128, seed=9)
+
+
+def _run(shape, backward):
+    from capacity_limited_routed_b200.block import MoEBlock
+    s = shape.with_(backward=backward)
+    inp = synth.make_inputs(s)
+    blk = MoEBlock(s, training=True)
+    blk.load(inp)
+    x = bf16_dev(inp["x"])
+    y = blk.forward(x)
+    out = {"s": s, "inp": inp, "blk": blk, "x": x, "y": y}
+    if backward:
+        out["dx"] = blk.backward(x, bf16_dev(inp["dy"]))
+    torch.cuda.synchronize()
+    return out
+
+
+def _routing_agreement(views, ctx):
+    idx_g = views["topk_idx"].cpu().numpy()
+    kept_g = views["slot"][..., 1].cpu().numpy() >= 0
+    match = (idx_g == ctx["idx"]).all(axis=1) & (kept_g == ctx["kept"]).all(axis=1)
+    affected = set(np.unique(idx_g[~match]).tolist()) | set(np.unique(ctx["idx"][~match]).tolist())
+    return match, affected
+
+
+@pytest.mark.parametrize("shape", [synth.TINY, RAGGED, synth.MID], ids=lambda s: s.name)
+def test_forward_matches_oracle(shape):
+    r = _run(shape, backward=False)
+    s, inp, blk = r["s"], r["inp"], r["blk"]
+    y_o, ctx = O.forward(inp["x"], inp["weights"], inp["bias"], s, logit_offset=inp["logit_offset"])
+    st = blk.stats_dict()
+    assert st["status"] == 0 and st["nan_logits"] == 0
+    v = blk.saved_views()
+    assert_close_rms(host64(v["z"]), ctx["z"], tol=1e-2, what="z")
+    assert_close_rms(host64(v["logits"]), ctx["logits"], tol=1e-2, what="logits")
+    match, _ = _routing_agreement(v, ctx)
+    rate = 1.0 - match.mean()
+    print(f"\n[{s.name}] routing mismatch rate {rate:.5f} ({(~match).sum()} of {s.T} tokens)")
+    assert rate <= 0.01
+    assert_close_rms(host64(r["y"])[match], y_o[match], what="y")
+    if match.all():
+        sl = ctx["slots"]
+        assert (st["kept"], st["dropped_sender"], st["dropped_receiver"]) == (
+            sl["kept"], sl["dropped_sender"], sl["dropped_receiver"])
+        assert np.array_equal(st["hist"], ctx["hist"])
+        assert np.array_equal(v["slot"][..., 0].cpu().numpy(), sl["sslot"])
+        assert np.array_equal(v["slot"][..., 1].cpu().numpy(), sl["rslot"])
+        assert np.array_equal(v["expert_rows"].cpu().numpy(), sl["expert_kept"])
+
+
+@pytest.mark.parametrize("shape", [synth.TINY, RAGGED, synth.MID], ids=lambda s: s.name)
+def test_backward_matches_oracle(shape):
+    r = _run(shape, backward=True)
+    s, inp, blk = r["s"], r["inp"], r["blk"]
+    y_o, ctx = O.forward(inp["x"], inp["weights"], inp["bias"], s, logit_offset=inp["logit_offset"])
+    dx_o, grads_o, _ = O.backward(inp["dy"], inp["weights"], ctx)
+    v = blk.saved_views()
+    match, affected = _routing_agreement(v, ctx)
+    print(f"\n[{s.name}] routing mismatch rate {1 - match.mean():.5f}")
+    assert_close_rms(host64(r["dx"])[match], dx_o[match], what="dx")
+    keep_e = np.array([e not in affected for e in range(s.n_experts)])
+    for name in ("w1", "w3", "w2"):
+        assert_close_rms(host64(blk.grads[name])[keep_e], grads_o[name][keep_e], what=f"d{name}")
+    assert_close_rms(host64(blk.grads["w_router"])[keep_e], grads_o["w_router"][keep_e], what="dw_router")
+    if match.all():
+        for name in ("w_lat_down", "w_lat_up", "ws1", "ws3", "ws2"):
+            assert_close_rms(host64(blk.grads[name]), grads_o[name], what=f"d{name}")
+    assert blk.stats_dict()["status"] == 0
+
+
+def test_bias_step_after_forward_matches_oracle():
+    r = _run(synth.TINY, backward=False)
+    s, inp, blk = r["s"], r["inp"], r["blk"]
+    hist = blk.stats_dict()["hist"]
+    want = O.bias_update(hist, inp["bias"], 1e-3, s.T, s.top_k)
+    blk.bias_update(1e-3)
+    got = blk.bias.cpu().numpy()
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    assert abs(float(got.astype(np.float64).sum())) < 1e-7
+
+
+def test_empty_batch_is_a_no_op():
+    from capacity_limited_routed_b200.block import MoEBlock
+    s = synth.TINY.with_(T=0)
+    blk = MoEBlock(s, training=True)
+    blk.load(synth.make_inputs(synth.TINY.with_(backward=True)))
+    x = torch.empty((0, s.d_model), dtype=torch.bfloat16, device=dev())
+    y = blk.forward(x)
+    dx = blk.backward(x, x)
+    torch.cuda.synchronize()
+    assert y.shape == (0, s.d_model) and dx.shape == (0, s.d_model)
+    assert all(int(g.abs().max().item()) == 0 for g in blk.grads.values())
+    assert blk.stats_dict()["kept"] == 0

@@ -1,0 +1,68 @@
+"""The tcgen05 GEMM core against a float64 matmul of the same bf16 operands, for every
+operand layout the block uses (K-major and MN-major A and B), on sizes that span
+several 128 x 256 x 64 tiles and leave ragged tails in M, N and K."""
+import numpy as np
+import pytest
+import torch
+
+from _helpers import dev, rms
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def M():
+    from capacity_limited_routed_b200 import moe
+    return moe
+
+
+def _operands(m, n, k, seed):
+    rng = np.random.default_rng(seed)
+    a = torch.from_numpy(rng.standard_normal((m, k), dtype=np.float32)).to(torch.bfloat16)
+    b = torch.from_numpy(rng.standard_normal((n, k), dtype=np.float32)).to(torch.bfloat16)
+    return a, b
+
+
+@pytest.mark.parametrize("a_mn", [0, 1])
+@pytest.mark.parametrize("b_mn", [0, 1])
+@pytest.mark.parametrize("mnk", [(128, 256, 64), (296, 264, 200), (1000, 776, 1048)])
+def test_gemm_layouts_f32(M, a_mn, b_mn, mnk):
+    m, n, k = mnk
+    a, b = _operands(m, n, k, seed=m + n + k + 2 * a_mn + b_mn)
+    ref = a.double() @ b.double().T
+    A = (a.T.contiguous() if a_mn else a).to(dev())
+    B = (b.T.contiguous() if b_mn else b).to(dev())
+    D = torch.full((m, n), float("nan"), dtype=torch.float32, device=dev())
+    status = torch.zeros(1, dtype=torch.int32, device=dev())
+    M.moe_gemm_bf16(m, n, k, A, a_mn, B, b_mn, D, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    got = D.double().cpu()
+    err = (got - ref).abs().max().item()
+    assert err <= 1e-4 * rms(ref.numpy()) * np.sqrt(k / 64), err
+
+
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 1), (1, 0)])
+def test_gemm_bf16_output(M, a_mn, b_mn):
+    m, n, k = 520, 392, 320
+    a, b = _operands(m, n, k, seed=5)
+    ref = (a.double() @ b.double().T)
+    A = (a.T.contiguous() if a_mn else a).to(dev())
+    B = (b.T.contiguous() if b_mn else b).to(dev())
+    D = torch.zeros((m, n), dtype=torch.bfloat16, device=dev())
+    M.moe_gemm_bf16(m, n, k, A, a_mn, B, b_mn, D)
+    got = D.double().cpu()
+    # one bf16 rounding of a float32 sum
+    assert ((got - ref).abs() <= 2.0 ** -8 * ref.abs() + 1e-3 * rms(ref.numpy())).all()
+
+
+def test_gemm_single_tile_exact_small_integers(M):
+    """Small integers multiply and add exactly in float32: the result must be exact."""
+    m, n, k = 128, 256, 192
+    rng = np.random.default_rng(1)
+    a = torch.from_numpy(rng.integers(-3, 4, size=(m, k)).astype(np.float32)).to(torch.bfloat16)
+    b = torch.from_numpy(rng.integers(-3, 4, size=(n, k)).astype(np.float32)).to(torch.bfloat16)
+    ref = a.double() @ b.double().T
+    D = torch.zeros((m, n), dtype=torch.float32, device=dev())
+    M.moe_gemm_bf16(m, n, k, a.to(dev()), 0, b.to(dev()), 0, D)
+    assert torch.equal(D.double().cpu(), ref)
