@@ -54,14 +54,15 @@ class MoEBlock:
         else:
             self.logit_offset = torch.from_numpy(np.asarray(lo, np.float32)).to(self.device)
         if self.training:
-            self.grads = {n: torch.empty_like(self.weights[n]) for n in WEIGHT_NAMES}
+            self.grads = {n: torch.empty(self.weights[n].shape, dtype=torch.float32, device=self.device)
+                          for n in WEIGHT_NAMES}
 
     # ------------------------------------------------------------------ steps
 
     def forward(self, x: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
         s = self.shape
         if y is None:
-            y = torch.empty((s.T, s.d_model), dtype=torch.bfloat16, device=self.device)
+            y = torch.empty((s.T, s.d_model), dtype=torch.float32, device=self.device)
         M.moe_forward(self.plan, self.weights, x, self.bias, self.logit_offset, y, self.stats, self.saved, self.ws,
                       stream)
         return y
@@ -71,7 +72,7 @@ class MoEBlock:
             raise RuntimeError("backward needs a block built with training=True")
         s = self.shape
         if dx is None:
-            dx = torch.empty((s.T, s.d_model), dtype=torch.bfloat16, device=self.device)
+            dx = torch.empty((s.T, s.d_model), dtype=torch.float32, device=self.device)
         M.moe_backward(self.plan, self.weights, self.saved, x, dy, dx, self.grads, self.ws, stream)
         return dx
 

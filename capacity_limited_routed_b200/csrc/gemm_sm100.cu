@@ -638,20 +638,20 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
 #define MOE_GEMM_CASE(BN_, AMN_, BMN_, EPI_)                                               \
   if (a.bn == BN_ && a.a_mn == AMN_ && a.b_mn == BMN_ && a.epi == EPI_)                   \
     return launch_instance<BN_, AMN_, BMN_, EPI_>(maps, kp, grid, st);
-  // forward
+  // forward: projections / experts (bf16 out), SwiGLU, router logits, block output (f32)
   MOE_GEMM_CASE(256, false, false, EPI_BF16)
   MOE_GEMM_CASE(256, false, false, EPI_SWIGLU)
   MOE_GEMM_CASE(128, false, false, EPI_F32)
-  // backward: dgrad (B stored [K][N]) and wgrad (both stored [K][.])
+  MOE_GEMM_CASE(256, false, false, EPI_F32)
+  // backward: dgrad (B stored [K][N]); dx in f32; wgrad (both stored [K][.]) in f32
   MOE_GEMM_CASE(256, false, true, EPI_BF16)
   MOE_GEMM_CASE(256, false, true, EPI_SWIGLU_BWD)
   MOE_GEMM_CASE(256, false, true, EPI_BF16_ADD_F32)
-  MOE_GEMM_CASE(256, true, true, EPI_BF16)
-  // test entry point: every operand layout with a float32 result
-  MOE_GEMM_CASE(256, false, false, EPI_F32)
   MOE_GEMM_CASE(256, false, true, EPI_F32)
-  MOE_GEMM_CASE(256, true, false, EPI_F32)
   MOE_GEMM_CASE(256, true, true, EPI_F32)
+  // the remaining layouts of the test entry point
+  MOE_GEMM_CASE(256, true, false, EPI_F32)
+  MOE_GEMM_CASE(256, true, true, EPI_BF16)
   MOE_GEMM_CASE(256, true, false, EPI_BF16)
 #undef MOE_GEMM_CASE
   return fail(MOE_ERR_UNSUPPORTED, "no gemm instance for this layout / epilogue");

@@ -36,6 +36,7 @@ namespace moe {
 
 namespace {
 thread_local std::string g_last_error;
+thread_local const char* g_step = "";
 }
 
 void set_error(const std::string& msg) { g_last_error = msg; }
@@ -47,7 +48,7 @@ moe_status_t fail(moe_status_t code, const std::string& msg) {
 
 moe_status_t cuda_check(cudaError_t e, const char* what) {
   if (e == cudaSuccess) return MOE_OK;
-  return fail(MOE_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+  return fail(MOE_ERR_CUDA, std::string("[") + g_step + "] " + what + ": " + cudaGetErrorString(e));
 }
 
 // ---------------------------------------------------------------------- launch accounting
@@ -81,6 +82,7 @@ void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 int64_t launches_so_far() { return g_launches.load(std::memory_order_relaxed); }
 
 ProfScope::ProfScope(const char* name, cudaStream_t st) : st_(st) {
+  g_step = name;
   std::lock_guard<std::mutex> lk(g_prof_mu);
   if (!g_prof_on) return;
   ProfRecord r;
@@ -487,7 +489,7 @@ moe_status_t moe_combine(moe_plan_t p, const uint16_t* expert_out, const float* 
 }
 
 moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const uint16_t* x, const float* bias,
-                         const float* logit_offset, uint16_t* y, void* stats, void* saved, void* ws, size_t ws_bytes,
+                         const float* logit_offset, float* y, void* stats, void* saved, void* ws, size_t ws_bytes,
                          void* stream) {
   if (p == nullptr || w == nullptr) return fail(MOE_ERR_INVALID_ARG, "null argument");
   if (!w->w_lat_down || !w->w_router || !w->w1 || !w->w3 || !w->w2 || !w->w_lat_up || !w->ws1 || !w->ws3 ||
@@ -574,10 +576,11 @@ moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const uint16_t* x
     a.status = status;
     MOE_TRY(gemm_run(a, st));
   }
-  // y = r W_lat_up^T + H_s ws2^T (two K segments, one accumulator)
+  // y = r W_lat_up^T + H_s ws2^T (two K segments, one accumulator), float32 out
   {
     ProfScope ps("fwd.lat_up_shared_down", st);
     GemmArgs a;
+    a.epi = EPI_F32;
     a.M = g.T;
     a.N = p->dm;
     a.nseg = 2;
@@ -596,7 +599,7 @@ moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const uint16_t* x
 }
 
 moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* saved, const uint16_t* x,
-                          const uint16_t* dy, uint16_t* dx, const moe_grads_t* gr, void* ws, size_t ws_bytes,
+                          const uint16_t* dy, float* dx, const moe_grads_t* gr, void* ws, size_t ws_bytes,
                           void* stream) {
   if (p == nullptr || w == nullptr || gr == nullptr) return fail(MOE_ERR_INVALID_ARG, "null argument");
   if (!saved || !ws) return fail(MOE_ERR_INVALID_ARG, "null buffer");
@@ -617,8 +620,8 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
     // no tokens: every gradient is zero
     const size_t sizes[9] = {size_t(dl * dm), size_t(E * dl), size_t(E * h * dl), size_t(E * h * dl),
                              size_t(E * dl * h), size_t(dm * dl), size_t(SH * dm), size_t(SH * dm), size_t(dm * SH)};
-    uint16_t* ptrs[9] = {gr->w_lat_down, gr->w_router, gr->w1, gr->w3, gr->w2, gr->w_lat_up, gr->ws1, gr->ws3, gr->ws2};
-    for (int i = 0; i < 9; ++i) MOE_TRY(cuda_check(cudaMemsetAsync(ptrs[i], 0, sizes[i] * 2, st), "grad memset"));
+    float* ptrs[9] = {gr->w_lat_down, gr->w_router, gr->w1, gr->w3, gr->w2, gr->w_lat_up, gr->ws1, gr->ws3, gr->ws2};
+    for (int i = 0; i < 9; ++i) MOE_TRY(cuda_check(cudaMemsetAsync(ptrs[i], 0, sizes[i] * 4, st), "grad memset"));
     return MOE_OK;
   }
   CtxPtrs c = ctx_ptrs(*p, const_cast<void*>(saved), true);
@@ -672,6 +675,7 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
     ProfScope ps("bwd.wgrad_lat_up_shared_down", st);
     GemmArgs a;
     a.a_mn = a.b_mn = true;
+    a.epi = EPI_F32;
     a.M = static_cast<int>(dm);
     a.N = static_cast<int>(dl);
     a.A[0] = mat(dy, dm, T);
@@ -721,6 +725,7 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
     ProfScope ps("bwd.experts_wgrad_down", st);
     GemmArgs a;
     a.a_mn = a.b_mn = true;
+    a.epi = EPI_F32;
     a.M = static_cast<int>(dl);
     a.N = static_cast<int>(h);
     a.groups = p->E;
@@ -760,6 +765,7 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
     ProfScope ps("bwd.experts_wgrad_gate_up", st);
     GemmArgs a;
     a.a_mn = a.b_mn = true;
+    a.epi = EPI_F32;
     a.M = static_cast<int>(h);
     a.N = static_cast<int>(dl);
     a.groups = p->E;
@@ -802,6 +808,7 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
     ProfScope ps("bwd.router_wgrad", st);
     GemmArgs a;
     a.a_mn = a.b_mn = true;
+    a.epi = EPI_F32;
     a.M = static_cast<int>(E);
     a.N = static_cast<int>(dl);
     a.A[0] = mat(dlog, E, T);
@@ -811,10 +818,11 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
     a.ldo = dl;
     MOE_TRY(gemm_run(a, st));
   }
-  // dx = dz W_down + dA_s ws1 + dB_s ws3 (three K segments)
+  // dx = dz W_down + dA_s ws1 + dB_s ws3 (three K segments), float32 out
   {
     ProfScope ps("bwd.dx", st);
     GemmArgs a;
+    a.epi = EPI_F32;
     a.b_mn = true;
     a.M = g.T;
     a.N = static_cast<int>(dm);
@@ -837,6 +845,7 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
     ProfScope ps("bwd.wgrad_lat_down_shared", st);
     GemmArgs a;
     a.a_mn = a.b_mn = true;
+    a.epi = EPI_F32;
     a.M = static_cast<int>(dl);
     a.N = static_cast<int>(dm);
     a.A[0] = mat(dz, dl, T);

@@ -314,32 +314,36 @@ __global__ void scan_totals(int32_t* __restrict__ stats, int E, int NP, int A_to
 __global__ void pack_kernel(const uint16_t* __restrict__ z, const int32_t* __restrict__ idx,
                             const int32_t* __restrict__ slot, int T, int k, int dl, int L, int P, int W, int Cs,
                             int E, uint16_t* __restrict__ pools) {
+  // destination row of each of the token's k assignments, staged per warp in shared
+  // memory (no warp shuffle inside the lane-divergent column loop)
+  __shared__ long long s_dst[8][32];
   const int lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
   const int warps = blockDim.x >> 5;
   const long long row_elems = dl + 8;
   const int nvec = dl / 8;
-  for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += gridDim.x * warps) {
+  for (int t = blockIdx.x * warps + wib; t < T; t += gridDim.x * warps) {
     int e_j = -1, s_j = -1;
     if (lane < k) {
       e_j = idx[static_cast<long long>(t) * k + lane];
       s_j = slot[2LL * (static_cast<long long>(t) * k + lane)];
+      const bool ok = s_j >= 0 && s_j < Cs && e_j >= 0 && e_j < E;
+      s_dst[wib][lane] = ok ? (static_cast<long long>(pool_of(e_j, L, P, W)) * Cs + s_j) * row_elems : -1;
     }
+    __syncwarp();
     const uint4* src = reinterpret_cast<const uint4*>(z + static_cast<long long>(t) * dl);
     for (int v = lane; v < nvec; v += 32) {
       const uint4 val = src[v];
       for (int j = 0; j < k; ++j) {
-        const int e = __shfl_sync(0xffffffffu, e_j, j);
-        const int s = __shfl_sync(0xffffffffu, s_j, j);
-        if (s >= 0 && s < Cs && e >= 0 && e < E) {
-          uint16_t* dst = pools + (static_cast<long long>(pool_of(e, L, P, W)) * Cs + s) * row_elems;
-          reinterpret_cast<uint4*>(dst)[v] = val;
-        }
+        const long long d = s_dst[wib][j];
+        if (d >= 0) reinterpret_cast<uint4*>(pools + d)[v] = val;
       }
     }
     if (lane < k && s_j >= 0 && s_j < Cs && e_j >= 0 && e_j < E) {
       uint16_t* dst = pools + (static_cast<long long>(pool_of(e_j, L, P, W)) * Cs + s_j) * row_elems + dl;
       *reinterpret_cast<int4*>(dst) = make_int4(e_j, 0, 0, 0);
     }
+    __syncwarp();
   }
 }
 
@@ -460,30 +464,31 @@ __device__ __forceinline__ uint4 pack8(const float (&a)[8]) {
 __global__ void combine_kernel(const uint16_t* __restrict__ ye, const float* __restrict__ gate,
                                const int32_t* __restrict__ idx, const int32_t* __restrict__ slot, int T, int k,
                                int dl, int Cr, int E, uint16_t* __restrict__ r) {
+  __shared__ long long s_row[8][32];
+  __shared__ float s_g[8][32];
   const int lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
   const int warps = blockDim.x >> 5;
   const int nvec = dl / 8;
-  for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += gridDim.x * warps) {
-    float g_j = 0.0f;
-    long long row_j = -1;
+  for (int t = blockIdx.x * warps + wib; t < T; t += gridDim.x * warps) {
     if (lane < k) {
       const long long a = static_cast<long long>(t) * k + lane;
       const int rs = slot[2 * a + 1];
       const int e = idx[a];
-      if (rs >= 0 && rs < Cr && e >= 0 && e < E) {
-        g_j = gate[a];
-        row_j = static_cast<long long>(e) * Cr + rs;
-      }
+      const bool ok = rs >= 0 && rs < Cr && e >= 0 && e < E;
+      s_row[wib][lane] = ok ? static_cast<long long>(e) * Cr + rs : -1;
+      s_g[wib][lane] = ok ? gate[a] : 0.0f;
     }
+    __syncwarp();
     for (int v = lane; v < nvec; v += 32) {
       float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
       for (int j = 0; j < k; ++j) {
-        const long long rj = __shfl_sync(0xffffffffu, row_j, j);
-        const float gj = __shfl_sync(0xffffffffu, g_j, j);
-        if (rj >= 0) acc8(acc, reinterpret_cast<const uint4*>(ye + rj * dl)[v], gj);
+        const long long rj = s_row[wib][j];
+        if (rj >= 0) acc8(acc, reinterpret_cast<const uint4*>(ye + rj * dl)[v], s_g[wib][j]);
       }
       reinterpret_cast<uint4*>(r + static_cast<long long>(t) * dl)[v] = pack8(acc);
     }
+    __syncwarp();
   }
 }
 
@@ -538,11 +543,12 @@ __global__ void undispatch_kernel(const uint16_t* __restrict__ dxe, const float*
                                   const float* __restrict__ dg, const int32_t* __restrict__ idx,
                                   const int32_t* __restrict__ slot, int T, int k, int dl, int Cr, int E,
                                   float* __restrict__ dz, uint16_t* __restrict__ dlogits) {
+  __shared__ long long s_row[8][32];
   const int lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
   const int warps = blockDim.x >> 5;
   const int nvec = dl / 8;
-  for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += gridDim.x * warps) {
-    long long row_j = -1;
+  for (int t = blockIdx.x * warps + wib; t < T; t += gridDim.x * warps) {
     float g_j = 0.0f, dg_j = 0.0f;
     int e_j = -1;
     if (lane < k) {
@@ -552,12 +558,13 @@ __global__ void undispatch_kernel(const uint16_t* __restrict__ dxe, const float*
       g_j = gate[a];
       dg_j = dg[a];
       if (e_j < 0 || e_j >= E) e_j = -1;
-      if (rs >= 0 && rs < Cr && e_j >= 0) row_j = static_cast<long long>(e_j) * Cr + rs;
+      s_row[wib][lane] = (rs >= 0 && rs < Cr && e_j >= 0) ? static_cast<long long>(e_j) * Cr + rs : -1;
     }
+    __syncwarp();
     for (int v = lane; v < nvec; v += 32) {
       float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
       for (int j = 0; j < k; ++j) {
-        const long long rj = __shfl_sync(0xffffffffu, row_j, j);
+        const long long rj = s_row[wib][j];
         if (rj >= 0) acc8(acc, reinterpret_cast<const uint4*>(dxe + rj * dl)[v], 1.0f);
       }
       float4* o = reinterpret_cast<float4*>(dz + static_cast<long long>(t) * dl + 8 * v);

@@ -26,6 +26,9 @@
  *   - Pointers named "device" are CUDA device pointers; others are host pointers.
  *     bf16 tensors are passed as uint16_t bit patterns.  All tensors are dense,
  *     row-major, with the shapes given; weights are [out][in].
+ *   - Precision: operands and every tensor passed between two steps are bf16, all
+ *     accumulation is float32; the block's outputs (y, dx, weight gradients) are
+ *     returned in float32, unrounded.
  *   - The caller owns every buffer.  The library never allocates device memory.
  *     Scratch ("ws") and the forward context kept for the backward ("saved") are
  *     caller-allocated with the sizes moe_plan_info reports, 256-byte aligned.
@@ -126,9 +129,11 @@ typedef struct {
   const uint16_t* ws2;         /* [d_model][S*hidden_shared]  shared down, expert s on columns s*h_s.. */
 } moe_weights_t;
 
-/* Weight gradients, bf16 device pointers, same shapes as moe_weights_t. */
+/* Weight gradients, float32 device pointers, same shapes as moe_weights_t.  They
+ * are the float32 accumulators of the wgrad GEMMs, not rounded to bf16 (the
+ * precision of fp32 main-gradient buffers in mixed-precision training). */
 typedef struct {
-  uint16_t *w_lat_down, *w_router, *w1, *w3, *w2, *w_lat_up, *ws1, *ws3, *ws2;
+  float *w_lat_down, *w_router, *w1, *w3, *w2, *w_lat_up, *ws1, *ws3, *ws2;
 } moe_grads_t;
 
 /* The routed experts alone (for moe_expert_ffn). */
@@ -198,19 +203,19 @@ MOE_API moe_status_t moe_combine(moe_plan_t plan, const uint16_t* expert_out, co
                          const int32_t* topk_idx, const int32_t* slot, uint16_t* r,
                          void* stream);
 
-/* Whole forward pass: y [T][d_model] bf16 device from x [T][d_model] bf16 device.
+/* Whole forward pass: y [T][d_model] float32 device from x [T][d_model] bf16 device.
  * bias [E] float32 device; logit_offset [E] float32 device or NULL.  stats: stats
  * buffer (device), fully overwritten.  saved: forward context for moe_backward
  * (saved_bytes) or NULL for inference. */
 MOE_API moe_status_t moe_forward(moe_plan_t plan, const moe_weights_t* w, const uint16_t* x,
-                         const float* bias, const float* logit_offset, uint16_t* y,
+                         const float* bias, const float* logit_offset, float* y,
                          void* stats, void* saved, void* ws, size_t ws_bytes, void* stream);
 
-/* Whole backward pass for the loss sum(y * dy): dx [T][d_model] bf16 device and
- * every weight gradient (overwritten, bf16).  Dropped assignments get no gradient;
+/* Whole backward pass for the loss sum(y * dy): dy [T][d_model] bf16 device, dx
+ * [T][d_model] float32 device and every weight gradient (overwritten, float32).  Dropped assignments get no gradient;
  * the bias gets none.  x must be the forward's input, saved its context. */
 MOE_API moe_status_t moe_backward(moe_plan_t plan, const moe_weights_t* w, const void* saved,
-                          const uint16_t* x, const uint16_t* dy, uint16_t* dx,
+                          const uint16_t* x, const uint16_t* dy, float* dx,
                           const moe_grads_t* grads, void* ws, size_t ws_bytes, void* stream);
 
 /* Bias step from a selection histogram: sgn_e = sign(T*k - E*hist_e) decided on

@@ -42,7 +42,9 @@ What the pages fix, and the readings taken where they are silent:
   * Precision: the block stores every tensor that passes between two of its steps
     in bfloat16 and accumulates in float32.  With ``storage="bf16"`` the oracle
     rounds at those same points (arithmetic stays float64); with
-    ``storage="f64"`` nothing is rounded.  The two places where floating point
+    ``storage="f64"`` nothing is rounded.  The block's own outputs (y, dx and the
+    weight gradients) are returned unrounded in both modes: they are the values
+    the device's results are measured against.  The two places where floating point
     decides an integer, the score ``logits + bias`` and its comparison, are taken
     in float32, the precision of the logits and of the bias.  The bias step is
     float32 arithmetic on the float32 bias.
@@ -289,10 +291,13 @@ def receive(payload: np.ndarray, header: np.ndarray, g: Geometry):
 
 
 def swiglu_hidden(X, w_gate, w_value, st):
-    """Pre-activations a = X w_gate^T, b = X w_value^T and hidden H = silu(a) * b."""
+    """Pre-activations a = X w_gate^T, b = X w_value^T and hidden H = silu(a) * b.
+
+    H is formed from the unrounded a and b; the a and b returned are the values kept
+    for the backward pass, which pass between steps and so are stored (rounded)."""
     a = X @ w_gate.T
     b = X @ w_value.T
-    return a, b, st(silu(a) * b)
+    return st(a), st(b), st(silu(a) * b)
 
 
 def forward(x, weights: dict, bias, shape, logit_offset=None, storage: str = "bf16",
@@ -346,7 +351,7 @@ def forward(x, weights: dict, bias, shape, logit_offset=None, storage: str = "bf
     r = st(r)
     # always-on shared experts on x, experts stacked on the hidden axis
     a_s, b_s, H_s = swiglu_hidden(x, W["ws1"], W["ws3"], st)
-    y = st(r @ W["w_lat_up"].T + H_s @ W["ws2"].T)
+    y = r @ W["w_lat_up"].T + H_s @ W["ws2"].T
     ctx = {
         "geometry": g, "storage": storage, "x": x, "z": z, "logits": logits,
         "idx": idx, "gate": gate, "hist": hist, "slots": slots, "kept": kept,
@@ -408,8 +413,7 @@ def backward(dy, weights: dict, ctx: dict):
     grads["w_lat_down"] = dz.T @ x
     grads["ws1"] = da_s.T @ x
     grads["ws3"] = db_s.T @ x
-    dx = st(dz @ W["w_lat_down"] + da_s @ W["ws1"] + db_s @ W["ws3"])
-    grads = {kk: st(v) for kk, v in grads.items()}
+    dx = dz @ W["w_lat_down"] + da_s @ W["ws1"] + db_s @ W["ws3"]
     inter = {"dr": dr, "dg": dg, "dlogits": dlogits, "dz": dz, "da_s": da_s, "db_s": db_s}
     return dx, grads, inter
 

@@ -43,3 +43,14 @@ def assert_close_rms(got, want, tol=REL_TOL, what=""):
     assert np.isfinite(got).all(), f"{what}: non-finite values"
     assert err <= tol * scale + 1e-30, f"{what}: max|err| {err:.3e} > {tol} * rms {scale:.3e}"
     return err / scale if scale else 0.0
+
+
+def assert_bf16_close(got, want, what=""):
+    """Both sides rounded the same float32/float64 value to bf16: allow one bf16 ulp
+    (2^-7 relative) where the two sums fall on different sides of a rounding point."""
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    # the absolute term covers float32-vs-float64 accumulation where a sum cancels
+    bound = 2.0 ** -7 * np.abs(want) + 1e-4 * rms(want)
+    bad = np.abs(got - want) > bound
+    assert not bad.any(), f"{what}: {int(bad.sum())} elements beyond one bf16 ulp, e.g. {got[bad][:4]} vs {want[bad][:4]}"
