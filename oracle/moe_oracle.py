@@ -57,7 +57,6 @@ from __future__ import annotations
 from dataclasses import dataclass
 
 import numpy as np
-import torch
 
 # --------------------------------------------------------------------------------------
 # precision helpers
@@ -65,17 +64,34 @@ import torch
 
 
 def round_bf16(a: np.ndarray) -> np.ndarray:
-    """Nearest bfloat16 value of each element (round to nearest even), as float64."""
-    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
-    return t.to(torch.bfloat16).to(torch.float64).numpy()
+    """Nearest bfloat16 value of each element, as float64.
+
+    The value is first taken to float32 (round to nearest), then to the 8-bit
+    significand of bfloat16 by round-to-nearest-even on the float32 bit pattern: add
+    0x7FFF plus the lowest kept bit, clear the 16 dropped bits.  NaN stays NaN."""
+    f = np.ascontiguousarray(a, dtype=np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000).astype(np.uint32)
+    out = r.view(np.float32).astype(np.float64)
+    nan = np.isnan(f)
+    if nan.any():
+        out[nan] = np.nan
+    return out
 
 
-def _storage(mode: str):
+def _storage(mode: str, dt=np.float64):
     if mode == "bf16":
-        return round_bf16
+        return lambda a: round_bf16(a).astype(dt)
     if mode == "f64":
-        return lambda a: np.asarray(a, dtype=np.float64)
+        return lambda a: np.asarray(a, dtype=dt)
     raise ValueError(f"unknown storage mode {mode!r}")
+
+
+def _acc_dtype(acc: str):
+    """Accumulation precision.  "f64" is the oracle.  "f32" runs the same steps with
+    float32 arithmetic; it exists only to measure how far two correct implementations
+    with bf16 storage drift apart when nothing but the accumulation precision differs."""
+    return {"f64": np.float64, "f32": np.float32}[acc]
 
 
 def silu(a: np.ndarray) -> np.ndarray:
@@ -301,24 +317,25 @@ def swiglu_hidden(X, w_gate, w_value, st):
 
 
 def forward(x, weights: dict, bias, shape, logit_offset=None, storage: str = "bf16",
-            logits_override=None):
+            logits_override=None, acc: str = "f64"):
     """One forward pass of the block.  Returns (y [T][d_model], ctx) where ctx holds
     every intermediate the backward pass and the tests need.
 
     ``logits_override`` replaces the computed router logits (float32 [T][E]); tests
     use it to study routing separately from the GEMMs.
     """
-    st = _storage(storage)
+    dt = _acc_dtype(acc)
+    st = _storage(storage, dt)
     g = geometry(shape)
-    W = {k: np.asarray(v, dtype=np.float64) for k, v in weights.items()}
-    x = np.asarray(x, dtype=np.float64)
+    W = {k: np.asarray(v, dtype=dt) for k, v in weights.items()}
+    x = np.asarray(x, dtype=dt)
     # latent down-projection
     z = st(x @ W["w_lat_down"].T)
     # router logits (float32, as the router hands them to top-k)
     if logits_override is None:
         lg = z @ W["w_router"].T
         if logit_offset is not None:
-            lg = lg + np.asarray(logit_offset, dtype=np.float64)[None, :]
+            lg = lg + np.asarray(logit_offset, dtype=dt)[None, :]
         logits = lg.astype(np.float32) if storage == "bf16" else lg
     else:
         logits = np.asarray(logits_override, dtype=np.float32)
@@ -333,11 +350,11 @@ def forward(x, weights: dict, bias, shape, logit_offset=None, storage: str = "bf
             if slots["rslot"][t, j] >= 0:
                 rows_of[idx[t, j]].append((t, j))
     expert = []
-    Yrow = np.zeros((T, k, d_l))
+    Yrow = np.zeros((T, k, d_l), dtype=dt)
     for e in range(g.E):
         tj = rows_of[e]
         ts = np.array([a for a, _ in tj], dtype=np.int64)
-        X = z[ts] if ts.size else np.zeros((0, d_l))
+        X = z[ts] if ts.size else np.zeros((0, d_l), dtype=dt)
         a, b, H = swiglu_hidden(X, W["w1"][e], W["w3"][e], st)
         Y = st(H @ W["w2"][e].T)
         expert.append({"tj": tj, "X": X, "a": a, "b": b, "H": H, "Y": Y})
@@ -345,7 +362,8 @@ def forward(x, weights: dict, bias, shape, logit_offset=None, storage: str = "bf
             Yrow[t, j] = Y[n]
     kept = slots["rslot"] >= 0
     # gate-weighted combine in latent space, in rank order
-    r = np.zeros((T, d_l))
+    r = np.zeros((T, d_l), dtype=dt)
+    gate = gate.astype(dt)
     for j in range(k):
         r += np.where(kept[:, j:j + 1], gate[:, j:j + 1] * Yrow[:, j, :], 0.0)
     r = st(r)
@@ -353,7 +371,7 @@ def forward(x, weights: dict, bias, shape, logit_offset=None, storage: str = "bf
     a_s, b_s, H_s = swiglu_hidden(x, W["ws1"], W["ws3"], st)
     y = r @ W["w_lat_up"].T + H_s @ W["ws2"].T
     ctx = {
-        "geometry": g, "storage": storage, "x": x, "z": z, "logits": logits,
+        "geometry": g, "storage": storage, "acc": acc, "x": x, "z": z, "logits": logits,
         "idx": idx, "gate": gate, "hist": hist, "slots": slots, "kept": kept,
         "expert": expert, "Yrow": Yrow, "r": r, "a_s": a_s, "b_s": b_s, "H_s": H_s,
     }
@@ -367,10 +385,11 @@ def forward(x, weights: dict, bias, shape, logit_offset=None, storage: str = "bf
 
 def backward(dy, weights: dict, ctx: dict):
     """Gradients of sum(y * dy) w.r.t. x and every weight.  Returns (dx, grads)."""
-    st = _storage(ctx["storage"])
+    dt = _acc_dtype(ctx.get("acc", "f64"))
+    st = _storage(ctx["storage"], dt)
     g: Geometry = ctx["geometry"]
-    W = {k: np.asarray(v, dtype=np.float64) for k, v in weights.items()}
-    dy = np.asarray(dy, dtype=np.float64)
+    W = {k: np.asarray(v, dtype=dt) for k, v in weights.items()}
+    dy = np.asarray(dy, dtype=dt)
     x, z, idx, gate, kept = ctx["x"], ctx["z"], ctx["idx"], ctx["gate"], ctx["kept"]
     T, k = idx.shape
     d_l = z.shape[1]
@@ -384,13 +403,12 @@ def backward(dy, weights: dict, ctx: dict):
     db_s = st(dH_s * silu(ctx["a_s"]))
     # r = sum_j kept g_j Y_j
     dg = np.where(kept, np.einsum("td,tjd->tj", dr, ctx["Yrow"]), 0.0)
-    dXrow = np.zeros((T, k, d_l))
+    dXrow = np.zeros((T, k, d_l), dtype=dt)
+    for n in ("w1", "w3", "w2"):
+        grads[n] = np.zeros_like(W[n])
     for e, ex in enumerate(ctx["expert"]):
         tj = ex["tj"]
         if not tj:
-            grads.setdefault("w1", np.zeros_like(W["w1"]))
-            grads.setdefault("w3", np.zeros_like(W["w3"]))
-            grads.setdefault("w2", np.zeros_like(W["w2"]))
             continue
         ts = np.array([a for a, _ in tj])
         js = np.array([b for _, b in tj])
@@ -399,13 +417,13 @@ def backward(dy, weights: dict, ctx: dict):
         dA = st(dH * ex["b"] * silu_grad(ex["a"]))
         dB = st(dH * silu(ex["a"]))
         dX = st(dA @ W["w1"][e] + dB @ W["w3"][e])
-        grads.setdefault("w1", np.zeros_like(W["w1"]))[e] = dA.T @ ex["X"]
-        grads.setdefault("w3", np.zeros_like(W["w3"]))[e] = dB.T @ ex["X"]
-        grads.setdefault("w2", np.zeros_like(W["w2"]))[e] = dY.T @ ex["H"]
+        grads["w1"][e] = dA.T @ ex["X"]
+        grads["w3"][e] = dB.T @ ex["X"]
+        grads["w2"][e] = dY.T @ ex["H"]
         dXrow[ts, js] = dX
     # softmax over the chosen logits: dl_j = g_j (dg_j - sum_i g_i dg_i)
     dl_chosen = gate * (dg - (gate * dg).sum(axis=1, keepdims=True))
-    dlogits = np.zeros((T, g.E))
+    dlogits = np.zeros((T, g.E), dtype=dt)
     np.put_along_axis(dlogits, idx.astype(np.int64), dl_chosen, axis=1)
     dlogits = st(dlogits)
     grads["w_router"] = dlogits.T @ z

@@ -5,6 +5,11 @@ import torch
 # Floating-point bar of the block: max |gpu - oracle| <= 2e-2 * RMS(oracle) per tensor
 # (bf16 storage, float32 accumulation).
 REL_TOL = 2e-2
+# Routed expert weight gradients: the float32-vs-float64 spread of bf16-stored
+# intermediates alone reaches ~4% of RMS there (tests/test_oracle_precision.py), so
+# they are held to max-abs <= 6e-2 * RMS and relative Frobenius error <= 1e-2.
+ROUTED_GRAD_TOL = 6e-2
+ROUTED_GRAD_FRO = 1e-2
 
 
 def dev():
@@ -54,3 +59,11 @@ def assert_bf16_close(got, want, what=""):
     bound = 2.0 ** -7 * np.abs(want) + 1e-4 * rms(want)
     bad = np.abs(got - want) > bound
     assert not bad.any(), f"{what}: {int(bad.sum())} elements beyond one bf16 ulp, e.g. {got[bad][:4]} vs {want[bad][:4]}"
+
+
+def assert_fro_close(got, want, tol, what=""):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    err = float(np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-300))
+    assert err <= tol, f"{what}: relative Frobenius error {err:.3e} > {tol}"
+    return err
