@@ -472,3 +472,121 @@ def forward_flops(shape, kept_rows: int | None = None) -> int:
     up = 2 * T * s.d_latent * s.d_model
     shared = T * 2 * (3 * s.d_model * s.hidden_shared) * s.n_shared
     return down + router + routed + up + shared
+
+
+# --------------------------------------------------------------------------------------
+# the same definition evaluated on a sample (for full-size workloads)
+# --------------------------------------------------------------------------------------
+#
+# At full width one forward is ~1e13 FLOPs: too much for float64 on the host.  The
+# functions below take the same steps as forward()/backward() above, but evaluate the
+# routed experts only for the sampled tokens (or experts).  Routing and drop
+# decisions are still computed over the whole batch, since every token's drops
+# depend on the tokens before it.  Routed weights are read one expert at a time
+# (``weights["w1"][e]``), so they may be a lazy view of device memory.
+
+
+def route_batch(x, weights, bias, shape, logit_offset=None, storage="bf16"):
+    """Latent projection, logits, top-k, gates and slots for every token."""
+    st = _storage(storage)
+    g = geometry(shape)
+    x = np.asarray(x, dtype=np.float64)
+    z = st(x @ np.asarray(weights["w_lat_down"], np.float64).T)
+    lg = z @ np.asarray(weights["w_router"], np.float64).T
+    if logit_offset is not None:
+        lg = lg + np.asarray(logit_offset, dtype=np.float64)[None, :]
+    logits = lg.astype(np.float32) if storage == "bf16" else lg
+    idx, gate, hist = route(logits, bias, g.k)
+    slots = assign_slots(idx, g)
+    return {"geometry": g, "storage": storage, "x": x, "z": z, "logits": logits, "idx": idx, "gate": gate,
+            "hist": hist, "slots": slots, "kept": slots["rslot"] >= 0}
+
+
+def _expert_rows(X, weights, e, st):
+    W1 = np.asarray(weights["w1"][e], np.float64)
+    W3 = np.asarray(weights["w3"][e], np.float64)
+    W2 = np.asarray(weights["w2"][e], np.float64)
+    a, b, H = swiglu_hidden(X, W1, W3, st)
+    return a, b, H, st(H @ W2.T), (W1, W3, W2)
+
+
+def forward_tokens(weights, rb: dict, tokens):
+    """y for the given tokens of a batch routed by ``route_batch``; also the per-token
+    pieces the sampled backward needs."""
+    st = _storage(rb["storage"])
+    idx, gate, kept, z, x = rb["idx"], rb["gate"], rb["kept"], rb["z"], rb["x"]
+    W_up = np.asarray(weights["w_lat_up"], np.float64)
+    ws1 = np.asarray(weights["ws1"], np.float64)
+    ws3 = np.asarray(weights["ws3"], np.float64)
+    ws2 = np.asarray(weights["ws2"], np.float64)
+    out, per = [], []
+    for t in tokens:
+        r = np.zeros(z.shape[1])
+        rows = []
+        for j in range(idx.shape[1]):
+            if kept[t, j]:
+                a, b, H, Y, Ws = _expert_rows(z[t:t + 1], weights, int(idx[t, j]), st)
+                r = r + gate[t, j] * Y[0]
+                rows.append((j, a[0], b[0], H[0], Y[0], Ws))
+        r = st(r)
+        a_s, b_s, H_s = swiglu_hidden(x[t:t + 1], ws1, ws3, st)
+        out.append(r @ W_up.T + H_s[0] @ ws2.T)
+        per.append({"r": r, "rows": rows, "a_s": a_s[0], "b_s": b_s[0]})
+    return np.array(out), per
+
+
+def backward_tokens(dy_rows, weights, rb: dict, tokens, per):
+    """dx for the given tokens (rows of dy given for those tokens, in order)."""
+    st = _storage(rb["storage"])
+    idx, gate = rb["idx"], rb["gate"]
+    W_up = np.asarray(weights["w_lat_up"], np.float64)
+    W_r = np.asarray(weights["w_router"], np.float64)
+    W_dn = np.asarray(weights["w_lat_down"], np.float64)
+    ws1 = np.asarray(weights["ws1"], np.float64)
+    ws3 = np.asarray(weights["ws3"], np.float64)
+    ws2 = np.asarray(weights["ws2"], np.float64)
+    E = W_r.shape[0]
+    out = []
+    for n, t in enumerate(tokens):
+        dy = np.asarray(dy_rows[n], np.float64)
+        p = per[n]
+        dr = st(dy @ W_up)
+        dH_s = dy @ ws2
+        da_s = st(dH_s * p["b_s"] * silu_grad(p["a_s"]))
+        db_s = st(dH_s * silu(p["a_s"]))
+        k = idx.shape[1]
+        dg = np.zeros(k)
+        dXsum = np.zeros(dr.shape[0])
+        for (j, a, b, H, Y, (W1, W3, W2)) in p["rows"]:
+            dg[j] = float(dr @ Y)
+            dY = st(gate[t, j] * dr)
+            dH = dY @ W2
+            dA = st(dH * b * silu_grad(a))
+            dB = st(dH * silu(a))
+            dXsum = dXsum + st(dA @ W1 + dB @ W3)
+        dl_chosen = gate[t] * (dg - (gate[t] * dg).sum())
+        dlog = np.zeros(E)
+        dlog[idx[t].astype(np.int64)] = dl_chosen
+        dlog = st(dlog)
+        dz = st(dlog @ W_r + dXsum)
+        out.append(dz @ W_dn + da_s @ ws1 + db_s @ ws3)
+    return np.array(out)
+
+
+def expert_weight_grads(dy, weights, rb: dict, e: int):
+    """Gradients of w1[e], w3[e], w2[e] over every row expert e kept."""
+    st = _storage(rb["storage"])
+    idx, gate, kept, z = rb["idx"], rb["gate"], rb["kept"], rb["z"]
+    W_up = np.asarray(weights["w_lat_up"], np.float64)
+    tj = [(t, j) for t, j in zip(*np.nonzero((idx == e) & kept))]
+    tj.sort(key=lambda p: rb["slots"]["rslot"][p])
+    ts = np.array([t for t, _ in tj], dtype=np.int64)
+    js = np.array([j for _, j in tj], dtype=np.int64)
+    X = z[ts]
+    a, b, H, Y, (W1, W3, W2) = _expert_rows(X, weights, e, st)
+    dr = st(np.asarray(dy, np.float64)[ts] @ W_up)
+    dY = st(gate[ts, js][:, None] * dr)
+    dH = dY @ W2
+    dA = st(dH * b * silu_grad(a))
+    dB = st(dH * silu(a))
+    return {"w1": dA.T @ X, "w3": dB.T @ X, "w2": dY.T @ H}

@@ -1,0 +1,159 @@
+"""Parity at full width, in the launch configuration the benchmark times.
+
+Inputs come from the benchmark's own seeded generator (drawn on the device by
+PyTorch's RNG).  Checks:
+  * routing and slot assignment bit-exact against the oracle on the same float32
+    logits, at T = 16,384 and 65,536 with 384 experts (plain and Zipf-skewed);
+  * properties that hold at any size on the whole block's own routing: counters add
+    up, no pool or expert exceeds its capacity, slots are dense and unique;
+  * y (and dx, and the gradients of two experts) on sampled tokens against the
+    oracle, whose routing and drops are computed over the whole batch; the routing
+    mismatch rate is reported.
+"""
+import numpy as np
+import pytest
+import torch
+
+from _helpers import (REL_TOL, ROUTED_GRAD_FRO, ROUTED_GRAD_TOL, assert_close_rms, assert_fro_close, dev,
+                      f32_dev, host64, i32_dev)
+from capacity_limited_routed_b200 import synth
+from oracle import moe_oracle as O
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+
+@pytest.fixture(scope="module")
+def M():
+    from capacity_limited_routed_b200 import moe
+    return moe
+
+
+# ------------------------------------------------------------------ routing and slots, bit-exact
+
+
+@pytest.mark.parametrize("shape", [synth.FULL, synth.SKEWED], ids=["full", "skewed"])
+def test_route_and_dispatch_bit_exact_full_size(M, shape):
+    s = shape
+    g = O.geometry(s)
+    plan = M.Plan.from_shape(s)
+    logits = synth.make_logits(s.T, s.n_experts, seed=s.seed + 100)
+    off = synth.make_logit_offset(s)
+    if off is not None:
+        logits = (logits + off[None, :]).astype(np.float32)
+    bias = (np.random.default_rng(5).standard_normal(s.n_experts) * 1e-2).astype(np.float32)
+    idx_o, gate_o, hist_o = O.route(logits, bias, s.top_k)
+    idx = torch.empty((s.T, s.top_k), dtype=torch.int32, device=dev())
+    gate = torch.empty((s.T, s.top_k), dtype=torch.float32, device=dev())
+    hist = torch.empty((s.n_experts,), dtype=torch.int32, device=dev())
+    M.moe_route(plan, f32_dev(logits), f32_dev(bias), idx, gate, hist)
+    assert np.array_equal(idx.cpu().numpy(), idx_o)
+    assert np.array_equal(hist.cpu().numpy(), hist_o)
+    np.testing.assert_allclose(gate.cpu().numpy(), gate_o, rtol=2e-6, atol=1e-7)
+    slots = O.assign_slots(idx_o, g)
+    info = plan.info
+    z = torch.zeros((s.T, s.d_latent), dtype=torch.bfloat16, device=dev())
+    pools = torch.empty(info.pools_bytes // 2, dtype=torch.int16, device=dev())
+    slot = torch.empty((s.T, s.top_k, 2), dtype=torch.int32, device=dev())
+    stats = torch.zeros(info.stats_bytes // 4, dtype=torch.int32, device=dev())
+    ws = torch.empty(info.workspace_bytes, dtype=torch.uint8, device=dev())
+    M.moe_dispatch(plan, z, i32_dev(idx_o), pools, slot, stats, ws)
+    sl = slot.cpu().numpy()
+    assert np.array_equal(sl[..., 0], slots["sslot"]) and np.array_equal(sl[..., 1], slots["rslot"])
+    st = stats.cpu().numpy()
+    assert (st[0], st[1], st[2], st[3]) == (slots["kept"], slots["dropped_sender"], slots["dropped_receiver"], 0)
+    E = s.n_experts
+    assert np.array_equal(st[8 + E:8 + 4 * E], np.concatenate(
+        [slots["expert_kept"], slots["expert_dropped_sender"], slots["expert_dropped_receiver"]]))
+    print(f"\n[{s.name}] drops: sender {slots['dropped_sender']}, receiver {slots['dropped_receiver']} "
+          f"of {s.T * s.top_k}")
+
+
+# ------------------------------------------------------------------ whole block on sampled tokens
+
+
+class _LazyExperts:
+    def __init__(self, t):
+        self.t = t
+
+    def __getitem__(self, e):
+        return self.t[e].float().cpu().numpy()
+
+
+def _host_weights(w):
+    out = {n: w[n].float().cpu().numpy() for n in ("w_lat_down", "w_router", "w_lat_up", "ws1", "ws3", "ws2")}
+    for n in ("w1", "w3", "w2"):
+        out[n] = _LazyExperts(w[n])
+    return out
+
+
+def _slot_properties(s, g, idx, slot, st):
+    """Whatever the routing, the slot map of the block must be a valid capacity-limited
+    assignment of it: dense unique slots, caps respected, counters adding up."""
+    E = s.n_experts
+    T, k = idx.shape
+    assert st["kept"] + st["dropped_sender"] + st["dropped_receiver"] == T * k
+    assert int(st["hist"].sum()) == T * k and st["status"] == 0
+    assert st["max_pool_fill"] <= g.C_s and st["max_expert_fill"] <= g.C_r
+    pool = O.placement(g)["pool"][idx]
+    ss, rs = slot[..., 0], slot[..., 1]
+    for p in range(g.n_pools):
+        v = np.sort(ss[(pool == p) & (ss >= 0)])
+        assert np.array_equal(v, np.arange(v.size))
+    for e in range(E):
+        v = np.sort(rs[(idx == e) & (rs >= 0)])
+        assert np.array_equal(v, np.arange(v.size))
+        assert v.size == st["expert_kept"][e]
+    assert not np.any((rs >= 0) & (ss < 0))
+
+
+@pytest.mark.parametrize("wid", [3, 4, 5], ids=["full", "skewed", "train"])
+def test_block_full_size_sampled(wid):
+    from capacity_limited_routed_b200.block import MoEBlock
+    s = synth.WORKLOADS[wid]
+    g = O.geometry(s)
+    inp = synth.make_inputs_device(s, device=dev())
+    blk = MoEBlock(s, device=dev(), training=True)
+    blk.load(inp)
+    y = blk.forward(inp["x"])
+    dx = blk.backward(inp["x"], inp["dy"]) if s.backward else None
+    torch.cuda.synchronize()
+    st = blk.stats_dict()
+    v = blk.saved_views()
+    idx_g = v["topk_idx"].cpu().numpy()
+    slot_g = v["slot"].cpu().numpy()
+    _slot_properties(s, g, idx_g, slot_g, st)
+    A = s.T * s.top_k
+    print(f"\n[{s.name}] drop fraction sender {st['dropped_sender'] / A:.4f} receiver "
+          f"{st['dropped_receiver'] / A:.4f}")
+
+    W = _host_weights(inp["weights"])
+    x_h = inp["x"].float().cpu().numpy()
+    off = None if inp["logit_offset"] is None else inp["logit_offset"].cpu().numpy()
+    rb = O.route_batch(x_h, W, inp["bias"].cpu().numpy(), s, logit_offset=off)
+    match = (idx_g == rb["idx"]).all(axis=1) & ((slot_g[..., 1] >= 0) == rb["kept"]).all(axis=1)
+    rate = 1.0 - match.mean()
+    print(f"[{s.name}] routing mismatch rate {rate:.5f} ({(~match).sum()} of {s.T})")
+    assert rate <= 0.01
+    sl = rb["slots"]
+    # drop counts of the two routings differ at most by what the mismatched tokens move
+    assert abs(st["dropped_sender"] + st["dropped_receiver"] - sl["dropped_sender"] - sl["dropped_receiver"]) \
+        <= s.top_k * (~match).sum() + 1
+    rng = np.random.default_rng(wid)
+    toks = rng.choice(np.nonzero(match)[0], size=48, replace=False)
+    ys, per = O.forward_tokens(W, rb, toks)
+    e_y = assert_close_rms(host64(y)[toks], ys, what="y (sampled)")
+    print(f"[{s.name}] y: max-abs / rms {e_y:.4f} on {toks.size} tokens")
+    if s.backward:
+        dy_h = inp["dy"].float().cpu().numpy()
+        dxs = O.backward_tokens(dy_h[toks], W, rb, toks, per)
+        e_dx = assert_close_rms(host64(dx)[toks], dxs, what="dx (sampled)")
+        print(f"[{s.name}] dx: max-abs / rms {e_dx:.4f}")
+        touched = set(np.unique(idx_g[~match]).tolist()) | set(np.unique(rb["idx"][~match]).tolist())
+        clean = [e for e in range(s.n_experts) if e not in touched]
+        for e in (clean[0], clean[len(clean) // 2]):
+            gw = O.expert_weight_grads(dy_h, W, rb, e)
+            for n in ("w1", "w3", "w2"):
+                got = host64(blk.grads[n][e])
+                er = assert_close_rms(got, gw[n], tol=ROUTED_GRAD_TOL, what=f"d{n}[{e}]")
+                fr = assert_fro_close(got, gw[n], ROUTED_GRAD_FRO, what=f"d{n}[{e}]")
+                print(f"[{s.name}] d{n}[{e}]: max-abs / rms {er:.4f}, frobenius {fr:.2e}")
