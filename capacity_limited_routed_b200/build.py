@@ -15,7 +15,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["moe_api.cu", "moe_kernels.cu", "gemm_sm100.cu"]
+SOURCES = ["moe_api.cu", "moe_kernels.cu", "gemm_sm100.cu", "moe_static_scratch.cu"]
 HEADERS = ["internal.h", "ptx.cuh", os.path.join("..", "..", "include", "moe.h")]
 LIB = os.path.join(HERE, "libmoe.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

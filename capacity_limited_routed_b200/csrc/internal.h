@@ -121,6 +121,10 @@ moe_status_t launch_undispatch(const Geo& g, const uint16_t* dxe, const float* g
                                cudaStream_t st);
 moe_status_t launch_bias_update(const Geo& g, const int32_t* hist, float* bias, float step, cudaStream_t st);
 
+// plan geometry and the device check, for entry points defined in other files
+const Geo& plan_geo(const moe_plan* p);
+moe_status_t device_check();
+
 // stats buffer layout (int32 words)
 constexpr int kStatsHead = 8;  // moe_stats_t
 inline int stats_hist(const Geo& g) { return kStatsHead; }

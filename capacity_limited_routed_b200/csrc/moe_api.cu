@@ -314,6 +314,11 @@ moe_status_t run_experts(const moe_plan& p, const uint16_t* w1, const uint16_t* 
 
 }  // namespace
 
+namespace moe {
+const Geo& plan_geo(const moe_plan* p) { return p->g; }
+moe_status_t device_check() { return device_ok(); }
+}  // namespace moe
+
 extern "C" {
 
 const char* moe_last_error(void) { return g_last_error.c_str(); }

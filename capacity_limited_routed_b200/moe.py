@@ -15,7 +15,7 @@ LIB_PATH = os.path.join(HERE, "libmoe.so")
 
 # the symbols include/moe.h declares
 EXPORTS = (
-    "moe_plan_create", "moe_plan_destroy", "moe_plan_info", "moe_route", "moe_dispatch",
+    "moe_plan_create", "moe_plan_destroy", "moe_plan_info", "moe_route", "moe_dispatch", "moe_dispatch_noalloc",
     "moe_expert_ffn", "moe_combine", "moe_forward", "moe_backward", "moe_bias_update",
     "moe_saved_view", "moe_gemm_bf16", "moe_profile_start", "moe_profile_stop", "moe_kernel_launches",
     "moe_last_error",
@@ -82,6 +82,7 @@ def _load():
         "moe_plan_info": [P, ctypes.POINTER(moe_plan_info_t)],
         "moe_route": [P, P, P, P, P, P, P],
         "moe_dispatch": [P, P, P, P, P, P, P, S, P],
+        "moe_dispatch_noalloc": [P, P, P, P, P, P, P],
         "moe_expert_ffn": [P, ctypes.POINTER(moe_expert_weights_t), P, P, P, P, S, P],
         "moe_combine": [P, P, P, P, P, P, P],
         "moe_forward": [P, ctypes.POINTER(moe_weights_t), P, P, P, P, P, P, P, S, P],
@@ -192,6 +193,12 @@ def moe_route(plan: Plan, logits, bias, topk_idx, topk_gate, hist, stream=None):
 def moe_dispatch(plan: Plan, z, topk_idx, pools, slot, stats, ws, stream=None):
     _check(_lib.moe_dispatch(plan.handle, _ptr(z), _ptr(topk_idx), _ptr(pools), _ptr(slot), _ptr(stats), _ptr(ws),
                              ws.numel() * ws.element_size(), _stream(stream)), "moe_dispatch")
+
+
+def moe_dispatch_noalloc(plan: Plan, z, topk_idx, pools, slot, stats, stream=None):
+    """moe_dispatch without a workspace (scan scratch in the library's static array)."""
+    _check(_lib.moe_dispatch_noalloc(plan.handle, _ptr(z), _ptr(topk_idx), _ptr(pools), _ptr(slot), _ptr(stats),
+                                     _stream(stream)), "moe_dispatch_noalloc")
 
 
 def moe_expert_ffn(plan: Plan, w1, w3, w2, pools, expert_out, expert_rows, ws, stream=None):

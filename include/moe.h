@@ -188,6 +188,26 @@ MOE_API moe_status_t moe_dispatch(moe_plan_t plan, const uint16_t* z, const int3
                           uint16_t* pools, int32_t* slot, void* stats,
                           void* ws, size_t ws_bytes, void* stream);
 
+/* moe_dispatch for callers that cannot allocate device memory.  Some callers have no
+ * allocator of their own: a plugin inside a host program that owns the whole
+ * device-memory budget, or code whose buffers are laid out before the block's sizes
+ * are known.  This variant takes no workspace: the counters of its slot scan live in
+ * a static array inside the library (2^21 int32 words, 8 MiB, held on every GPU that
+ * loads the library until the process exits).  Inputs and outputs are those of
+ * moe_dispatch, with the same results.
+ *   - Plans whose scan needs more than 2^21 words (T/32 * (D*W + E) + D*W) are
+ *     rejected with MOE_ERR_UNSUPPORTED; use moe_dispatch for them.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any stream
+ *     capture.
+ *   - Every call uses the same array.  Calls whose work overlaps on the GPU (other
+ *     streams, other threads) race on it; order them on one stream.  Nothing in the
+ *     array has to start at zero: each call writes every word it reads.
+ * It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * The source pages have no counterpart of this entry point. */
+MOE_API moe_status_t moe_dispatch_noalloc(moe_plan_t plan, const uint16_t* z, const int32_t* topk_idx,
+                                          uint16_t* pools, int32_t* slot, void* stats, void* stream);
+
 /* Receiver side and the routed experts: unpack each pool by the packed expert ids
  * (first C_r rows per expert in pool order), then the grouped SwiGLU GEMMs.
  *   pools as written by moe_dispatch; expert_out [E][C_r][d_latent] bf16 device

@@ -1,0 +1,85 @@
+"""moe_dispatch_noalloc: the dispatch for callers that cannot allocate device memory.
+
+Some callers have no allocator of their own (a plugin inside a host program that owns
+the whole device-memory budget, for instance), so they cannot hand moe_dispatch a
+workspace.  moe_dispatch_noalloc keeps the scan's scratch in a static array inside the
+library.  Its results must be those of moe_dispatch, bit for bit, call after call:
+the array is shared by every call and keeps the previous call's contents.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from capacity_limited_routed_b200 import synth
+
+
+def _idx(T, E, k, seed, skew):
+    """k distinct experts per token, skewed towards low ids (input generation only)."""
+    rng = np.random.default_rng(seed)
+    scores = rng.standard_normal((T, E)) - skew * np.log1p(np.arange(E))[None, :]
+    return np.argsort(-scores, axis=1, kind="stable")[:, :k].astype(np.int32)
+
+
+def _run_both(M, shape, seed, skew):
+    dev = torch.device("cuda:0")
+    plan = M.Plan.from_shape(shape)
+    info = plan.info
+    T, k, dl = shape.T, shape.top_k, shape.d_latent
+    z = torch.from_numpy(np.random.default_rng(seed + 1).standard_normal((T, dl), dtype=np.float32)).to(dev)
+    z = z.to(torch.bfloat16)
+    idx = torch.from_numpy(_idx(T, shape.n_experts, k, seed, skew)).to(dev)
+    outs = []
+    for use_static in (False, True):
+        pools = torch.zeros(info.pools_bytes // 2, dtype=torch.int16, device=dev)
+        slot = torch.full((T, k, 2), -9, dtype=torch.int32, device=dev)
+        stats = torch.zeros(info.stats_bytes // 4, dtype=torch.int32, device=dev)
+        if use_static:
+            M.moe_dispatch_noalloc(plan, z, idx, pools, slot, stats)
+        else:
+            ws = torch.empty(info.workspace_bytes, dtype=torch.uint8, device=dev)
+            M.moe_dispatch(plan, z, idx, pools, slot, stats, ws)
+        torch.cuda.synchronize()
+        outs.append((pools.cpu().numpy(), slot.cpu().numpy(), stats.cpu().numpy()))
+    return outs
+
+
+def _pool_rows_used(shape, plan, stats):
+    """Rows of each pool that hold a row (the rest carry only the empty header)."""
+    E = shape.n_experts
+    return stats[8 + 4 * E:8 + 4 * E + plan.info.n_pools]
+
+
+@pytest.mark.gpu
+def test_noalloc_dispatch_matches_dispatch_on_consecutive_calls():
+    from capacity_limited_routed_b200 import moe as M
+    cases = [(synth.TINY.with_(T=777, top_k=5), 3, 1.2),     # drops at both caps
+             (synth.MID, 4, 0.3)]                              # a larger scan next
+    for shape, seed, skew in cases:
+        (p_ref, s_ref, st_ref), (p_new, s_new, st_new) = _run_both(M, shape, seed, skew)
+        assert np.array_equal(s_new, s_ref)
+        assert np.array_equal(st_new[:8], st_ref[:8])
+        E = shape.n_experts
+        assert np.array_equal(st_new[8 + E:], st_ref[8 + E:])   # per-expert and per-pool counters
+        plan = M.Plan.from_shape(shape)
+        rows = p_ref.reshape(plan.info.n_pools, plan.info.cap_send, shape.d_latent + 8)
+        rows_new = p_new.reshape(rows.shape)
+        assert np.array_equal(rows_new[:, :, shape.d_latent:], rows[:, :, shape.d_latent:])  # headers
+        fill = _pool_rows_used(shape, plan, st_ref)
+        for p in range(plan.info.n_pools):
+            assert np.array_equal(rows_new[p, :fill[p]], rows[p, :fill[p]])
+        assert st_ref[1] + st_ref[2] > 0 or skew < 1.0
+
+
+def test_noalloc_dispatch_rejects_plans_beyond_its_static_scratch():
+    """A plan whose scan needs more than the static array holds is refused, with a
+    message that names both sizes, before anything touches a device."""
+    from capacity_limited_routed_b200 import moe as M
+    plan = M.Plan(T=1 << 20, d_model=64, d_latent=64, n_experts=1024, top_k=2, n_dest=32,
+                  hidden_routed=128, n_shared=1, hidden_shared=128, n_waves=1)
+    fake = ctypes.c_void_p(0x1000)
+    code = M.lib().moe_dispatch_noalloc(plan.handle, fake, fake, fake, fake, fake, None)
+    assert code == 2
+    msg = M.moe_last_error()
+    assert "static array holds 2097152" in msg and "moe_dispatch" in msg
