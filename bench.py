@@ -45,7 +45,7 @@ def load_peaks():
 def workload_shape(name):
     from capacity_limited_routed_b200 import synth
     return {"train": synth.TRAIN, "full": synth.FULL, "mid": synth.MID, "skewed": synth.SKEWED,
-            "tiny": synth.TINY.with_(backward=True)}[name]
+            "tiny": synth.TINY.with_(backward=True), "profile": synth.PROFILE}[name]
 
 
 def describe(s):
@@ -84,7 +84,26 @@ def step_work(s, kept):
         "bwd.wgrad_lat_down_shared": 2 * T * dm * (dl + 2 * SH),
     }
     A = T * k
+    w_routed = E * h * dl * 2           # one routed weight tensor, bf16
     b = {
+        # GEMMs: operands read once, results written once (bf16 unless noted)
+        "fwd.lat_down": T * dm * 2 + dl * dm * 2 + T * dl * 2,
+        "fwd.router": T * dl * 2 + E * dl * 2 + T * E * 4,
+        "experts.gate_up": 2 * w_routed + kept * dl * 2 + 3 * kept * h * 2,
+        "experts.down": w_routed + kept * h * 2 + kept * dl * 2,
+        "fwd.shared_gate_up": T * dm * 2 + 2 * SH * dm * 2 + 3 * T * SH * 2,
+        "fwd.lat_up_shared_down": T * (dl + SH) * 2 + dm * (dl + SH) * 2 + T * dm * 4,
+        "bwd.dr": T * dm * 2 + dm * dl * 2 + T * dl * 2,
+        "bwd.shared_dgrad_swiglu": T * dm * 2 + dm * SH * 2 + 4 * T * SH * 2,
+        "bwd.wgrad_lat_up_shared_down": T * dm * 2 + T * (dl + SH) * 2 + dm * (dl + SH) * 4,
+        "bwd.experts_dgrad_down": kept * dl * 2 + w_routed + 4 * kept * h * 2,
+        "bwd.experts_wgrad_down": kept * dl * 2 + kept * h * 2 + E * dl * h * 4,
+        "bwd.experts_dgrad_gate_up": 2 * kept * h * 2 + 2 * w_routed + kept * dl * 2,
+        "bwd.experts_wgrad_gate_up": 2 * kept * h * 2 + kept * dl * 2 + 2 * E * h * dl * 4,
+        "bwd.router_dgrad": T * E * 2 + E * dl * 2 + T * dl * 4 + T * dl * 2,
+        "bwd.router_wgrad": T * E * 2 + T * dl * 2 + E * dl * 4,
+        "bwd.dx": T * (dl + 2 * SH) * 2 + dm * (dl + 2 * SH) * 2 + T * dm * 4,
+        "bwd.wgrad_lat_down_shared": T * (dl + 2 * SH) * 2 + T * dm * 2 + dm * (dl + 2 * SH) * 4,
         # logits read, idx + gate written
         "fwd.route_topk": T * E * 4 + A * 8 + E * 4,
         # z read once, every sender-kept row written with its 16-byte header
@@ -239,21 +258,21 @@ def main():
     from capacity_limited_routed_b200 import moe as M
     from capacity_limited_routed_b200 import synth
     from capacity_limited_routed_b200.block import MoEBlock
+    from capacity_limited_routed_b200.parallel import global_histogram, global_tokens
 
     peaks = load_peaks()
     inp = synth.make_inputs_device(s, device=dev, seed=s.seed + 7919 * rank)
     blk = MoEBlock(s, device=dev, training=s.backward)
     blk.load(inp)
     x, dy = inp["x"], inp.get("dy")
-    hist_plan = M.Plan.from_shape(s.with_(T=s.T * world)) if world > 1 else blk.plan
+    hist_plan = M.Plan.from_shape(s.with_(T=global_tokens(s.T))) if world > 1 else blk.plan
     stream = torch.cuda.current_stream(dev)
 
     def step():
         blk.forward(x)
         if s.backward:
             blk.backward(x, dy)
-            if world > 1:
-                dist.all_reduce(blk.hist())
+            global_histogram(blk.hist())
             M.moe_bias_update(hist_plan, blk.hist(), blk.bias, 1e-3)
 
     def barrier():
@@ -304,29 +323,35 @@ def main():
     kept = st["kept"]
     flops, bytes_ = step_work(s, kept)
     tc_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    # each step against the roofline that binds it: the larger of its tensor time at
+    # the sustained bf16 peak and its HBM time at the copy bandwidth
+    hbm = peaks["hbm_gbs"]
     kernels = {}
     for name, (tot, cnt, nl) in per.items():
         avg = tot / cnt
         e = {"ms": round(avg, 4), "share": round(tot / sum(v[0] for v in per.values()), 4)}
+        t_tc = flops[name] / (tc_peak * 1e12) if name in flops else 0.0
+        t_mem = bytes_[name] / (hbm * 1e9) if name in bytes_ else 0.0
         if name in flops:
             e["tflops"] = round(flops[name] / (avg * 1e-3) / 1e12, 1)
-            e["frac"] = round(e["tflops"] / tc_peak, 3)
-        elif name in bytes_:
+        if name in bytes_:
             e["gbs"] = round(bytes_[name] / (avg * 1e-3) / 1e9, 1)
-            e["frac"] = round(e["gbs"] / peaks["hbm_gbs"], 3)
+        if t_tc or t_mem:
+            e["bound"] = "tensor" if t_tc >= t_mem else "hbm"
+            e["frac"] = round(max(t_tc, t_mem) / (avg * 1e-3), 3)
         kernels[name] = e
     top = max(per.items(), key=lambda kv: kv[1][0])[0]
     avg_top = per[top][0] / per[top][1]
-    if top in flops:
-        achieved = flops[top] / (avg_top * 1e-3) / 1e12
-        roof = {"kernel": top, "bound": "tensor", "achieved": round(achieved, 1), "peak": tc_peak,
-                "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 3), "traffic": None,
+    kt = kernels[top]
+    if kt.get("bound") == "tensor":
+        roof = {"kernel": top, "bound": "tensor", "achieved": kt["tflops"], "peak": tc_peak,
+                "unit": "TFLOP/s", "frac": round(kt["tflops"] / tc_peak, 3), "traffic": None,
                 "peak_kind": f"bf16_tflops_sustained ({peaks['_source']}): kernel timed inside a long step",
                 "flops_per_launch": flops[top]}
     else:
-        achieved = bytes_.get(top, 0) / (avg_top * 1e-3) / 1e9
-        roof = {"kernel": top, "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 3), "traffic": None}
+        roof = {"kernel": top, "bound": "hbm", "achieved": kt.get("gbs"), "peak": hbm,
+                "unit": "GB/s", "frac": round((kt.get("gbs") or 0) / hbm, 3), "traffic": None,
+                "peak_kind": f"hbm_gbs ({peaks['_source']})", "bytes_per_launch": bytes_.get(top)}
     fwd_ms = sum(v[0] for k_, v in per.items() if k_.startswith("fwd.") or k_.startswith("experts.")) / args.steps
     step_ms = ms_max / args.steps
     value = world * s.T / (step_ms * 1e-3)
@@ -351,8 +376,7 @@ def main():
             blk.forward(xs)
             if s.backward:
                 blk.backward(xs, dys)
-                if world > 1:
-                    dist.all_reduce(blk.hist())
+                global_histogram(blk.hist())
                 M.moe_bias_update(hist_plan, blk.hist(), blk.bias, 1e-3)
             out_h.copy_(blk.stats[:8], non_blocking=True)
         e1.record(stream)

@@ -33,6 +33,10 @@ struct TmaMaps {
   CUtensorMap a[3];
   CUtensorMap b[3];
   CUtensorMap bv;
+  CUtensorMap out;    // float32 / bf16 output: 32 rows x 128 bytes; SwiGLU outputs: 32 x 64 bytes
+  CUtensorMap out2;   // SwiGLU backward: dB
+  CUtensorMap aux_a;  // SwiGLU: saved gate pre-activation (store); backward: a (load)
+  CUtensorMap aux_b;  // SwiGLU: saved value pre-activation (store); backward: b (load)
 };
 
 struct KParams {
@@ -60,20 +64,36 @@ constexpr int kBK = 64;
 constexpr int kThreads = 192;
 constexpr int kMaxGroups = 1024;
 
-template <int BN>
+// WRITE_BOUND: the weight-gradient instance (both operands MN-major).  Its K is the
+// few rows an expert received, so a tile's main loop is short and its output (128 x
+// 256 float32 = 128 KB) weighs as much as its operands: it gets a ring of two staging
+// buffers per epilogue warp so stores stream without waiting.  It never runs with
+// ragged rows, so it needs no tile-prefix array.
+template <int BN, bool WRITE_BOUND = false, bool SWIGLU = false>
 struct Cfg {
   static constexpr int kABytes = kBM * kBK * 2;  // 16 KB
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStage = kABytes + kBBytes;
   static constexpr int kStages = (BN == 256) ? 4 : 6;
   static constexpr int kTmemCols = 2 * BN;
-  static constexpr int kBarBytes = 8 * (2 * kStages + 5) + 16;
-  static constexpr int kSmem = 1024 + kStages * kStage + kBarBytes + 4 * (kMaxGroups + 1);
+  static constexpr int kBufs = WRITE_BOUND ? 2 : 1;          // staging buffers per epilogue warp
+  // a buffer holds 32 rows x 128 bytes (float32 / bf16 outputs, or two 32 x 64-byte
+  // bf16 tiles); the forward SwiGLU stages three 32 x 64-byte tiles (H, a, b)
+  static constexpr int kBufBytes = SWIGLU ? 6144 : 4096;
+  static constexpr int kStaging = 4 * kBufs * kBufBytes;
+  static constexpr int kBarBytes = 8 * (2 * kStages + 5 + 4) + 16;
+  static constexpr int kPrefixInts = WRITE_BOUND ? 0 : kMaxGroups + 1;
+  static constexpr int kSmem = 1024 + kStages * kStage + kStaging + kBarBytes + 4 * kPrefixInts;
+  static_assert(kSmem <= 232448, "shared memory budget");
 };
 
 __device__ __forceinline__ void record_status(int32_t* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);
 }
+
+struct Tile {
+  int g, m, n, kb;
+};
 
 // Tile bookkeeping shared by the three roles; all of them walk the same list.
 template <int BN, int EPI>
@@ -116,6 +136,19 @@ struct Sched {
     }
   }
 
+  // everything a role needs about tile t (g = -1 past the end)
+  __device__ Tile tile(int t) const {
+    Tile r;
+    if (t >= total) {
+      r.g = -1;
+      r.m = r.n = r.kb = 0;
+      return r;
+    }
+    decode(t, r.g, r.m, r.n);
+    r.kb = k_blocks(r.g);
+    return r;
+  }
+
   __device__ int k_blocks(int g) const {
     if (p.ragged == 2) {
       int r = p.group_rows[g];
@@ -129,17 +162,19 @@ struct Sched {
 template <int BN, bool A_MN, bool B_MN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ TmaMaps maps, const KParams p) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, A_MN && B_MN, EPI == EPI_SWIGLU>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStage);
+  uint8_t* staging = smem + C::kStages * C::kStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + C::kStaging);
   uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* ebar = drain + 1;  // one per epilogue warp: its own TMA loads (SwiGLU backward)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ebar + 4);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-  int* prefix = reinterpret_cast<int*>(smem + C::kStages * C::kStage + C::kBarBytes);
+  int* prefix = reinterpret_cast<int*>(staging + C::kStaging + C::kBarBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -154,6 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tempty[a], 128);
     }
     mbar_init(drain, 1);
+    for (int w = 0; w < 4; ++w) mbar_init(&ebar[w], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -168,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   // tiles per group and their prefix (ragged rows only)
-  if (p.ragged == 1) {
+  if (C::kPrefixInts > 0 && p.ragged == 1) {
     const int out_cols = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
     const int nt = (p.N + out_cols - 1) / out_cols;
     const int per = (p.groups + kThreads - 1) / kThreads;
@@ -222,10 +258,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int armed_phase[C::kStages];
       for (int s = 0; s < C::kStages; ++s) armed_phase[s] = -1;
       bool ok = true;
+      Tile nxt = sc.tile(blockIdx.x);
       for (int t = blockIdx.x; ok && t < sc.total; t += gridDim.x) {
-        int g, mt, ntile;
-        sc.decode(t, g, mt, ntile);
-        const int kb_total = sc.k_blocks(g);
+        const Tile cur = nxt;
+        nxt = sc.tile(t + gridDim.x);  // issued a tile ahead: its count load overlaps this tile
+        const int g = cur.g, mt = cur.m, ntile = cur.n, kb_total = cur.kb;
         for (int kb = 0; kb < kb_total; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_v)) {
             ok = false;
@@ -285,10 +322,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       bool issued = false;
+      Tile nxt = sc.tile(blockIdx.x);
       for (int t = blockIdx.x; ok && t < sc.total; t += gridDim.x) {
-        int g, mt, ntile;
-        sc.decode(t, g, mt, ntile);
-        const int kb_total = sc.k_blocks(g);
+        const Tile cur = nxt;
+        nxt = sc.tile(t + gridDim.x);
+        const int kb_total = cur.kb;
         if (kb_total == 0) continue;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_v)) {
           ok = false;
@@ -340,10 +378,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     int acc = 0;
     uint32_t acc_phase = 0;
+    int ring = 0;        // next staging buffer of this warp
+    uint32_t eph = 0;    // phase of this warp's load barrier
+    Tile nxt = sc.tile(blockIdx.x);
     for (int t = blockIdx.x; t < sc.total; t += gridDim.x) {
-      int g, mt, ntile;
-      sc.decode(t, g, mt, ntile);
-      const int kb_total = sc.k_blocks(g);
+      const Tile cur = nxt;
+      nxt = sc.tile(t + gridDim.x);
+      const int g = cur.g, mt = cur.m, ntile = cur.n, kb_total = cur.kb;
       const int row = mt * kBM + row_in_tile;
       const bool row_ok = row < p.M;
       if (kb_total == 0) {
@@ -375,38 +416,166 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tbase = tmem_base + lane_off + static_cast<uint32_t>(acc * BN);
 
       if constexpr (EPI == EPI_SWIGLU) {
+        // per chunk of 32 output columns: H, a, b as three 32 x 64-byte tiles (64-byte
+        // swizzle: 16-byte piece j of row r at j ^ ((r >> 1) & 3)), three TMA stores
         const int n_out0 = ntile * (BN / 2);
+        const int row0 = mt * kBM + q * 32;
+        uint8_t* buf = staging + (warp - 2) * C::kBufBytes;
+        const uint32_t rbase = smem_u32(buf) + lane * 64;
+        const int sw = (lane >> 1) & 3;
 #pragma unroll 1
         for (int c = 0; c < BN / 2; c += 32) {
           float gv[32], uv[32];
           __syncwarp();
           tmem_ld_32cols(tbase + c, gv);
           tmem_ld_32cols(tbase + BN / 2 + c, uv);
-          const int col = n_out0 + c;
-          if (row_ok && col < p.N) {
-            const long long off = g * p.out_gs + (long long)row * p.ldo + col;
-            uint32_t h[16];
+          uint32_t h[16], ga[16], gb[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float a0 = gv[2 * i], a1 = gv[2 * i + 1];
+            const float s0 = a0 / (1.0f + expf(-a0)), s1 = a1 / (1.0f + expf(-a1));
+            h[i] = pack_bf16x2(s0 * uv[2 * i], s1 * uv[2 * i + 1]);
+            ga[i] = pack_bf16x2(a0, a1);
+            gb[i] = pack_bf16x2(uv[2 * i], uv[2 * i + 1]);
+          }
+          if (lane == 0) bulk_wait_read<0>();  // the previous chunk's stores have read the buffer
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t off = ((j ^ sw) << 4);
+            st_shared_v4(rbase + off, h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
+            st_shared_v4(rbase + 2048 + off, ga[4 * j], ga[4 * j + 1], ga[4 * j + 2], ga[4 * j + 3]);
+            st_shared_v4(rbase + 4096 + off, gb[4 * j], gb[4 * j + 1], gb[4 * j + 2], gb[4 * j + 3]);
+          }
+          fence_async_shared();
+          __syncwarp();
+          const int col0 = n_out0 + c;
+          if (lane == 0 && col0 < p.N && row0 < p.M) {
+            tma_store_3d(&maps.out, buf, col0, row0, g);
+            if (p.save_a != nullptr) {
+              tma_store_3d(&maps.aux_a, buf + 2048, col0, row0, g);
+              tma_store_3d(&maps.aux_b, buf + 4096, col0, row0, g);
+            }
+            bulk_commit();
+          }
+        }
+      } else if constexpr (EPI == EPI_F32 || EPI == EPI_BF16) {
+        // stage 32 rows x 128 bytes in shared memory (128-byte swizzle: 16-byte piece j
+        // of row r at j ^ (r & 7)), then one TMA tensor store per chunk; rows past M and
+        // columns past N are clipped by the tensor map
+        constexpr int kChunk = (EPI == EPI_F32) ? 32 : 64;
+        const int row0 = mt * kBM + q * 32;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += kChunk) {
+          uint8_t* buf = staging + ((warp - 2) * C::kBufs + ring) * C::kBufBytes;
+          if (++ring == C::kBufs) ring = 0;
+          const uint32_t row_addr = smem_u32(buf) + lane * 128;
+          uint32_t w[32];
+          __syncwarp();
+          if constexpr (EPI == EPI_F32) {
+            float v[32];
+            tmem_ld_32cols(tbase + c, v);
+            const int col0 = ntile * BN + c;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              float x = v[i];
+              if (p.col_add != nullptr && col0 + i < p.N) x += p.col_add[col0 + i];
+              w[i] = __float_as_uint(x);
+            }
+          } else {
+            float v0[32], v1[32];
+            tmem_ld_32cols(tbase + c, v0);
+            tmem_ld_32cols(tbase + c + 32, v1);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float a0 = gv[2 * i], a1 = gv[2 * i + 1];
-              const float s0 = a0 / (1.0f + expf(-a0)), s1 = a1 / (1.0f + expf(-a1));
-              h[i] = pack_bf16x2(s0 * uv[2 * i], s1 * uv[2 * i + 1]);
-            }
-            uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + off);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) o[v] = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
-            if (p.save_a != nullptr) {
-              uint4* oa = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.save_a) + off);
-              uint4* ob = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.save_b) + off);
-#pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                oa[v] = make_uint4(pack_bf16x2(gv[8 * v], gv[8 * v + 1]), pack_bf16x2(gv[8 * v + 2], gv[8 * v + 3]),
-                                   pack_bf16x2(gv[8 * v + 4], gv[8 * v + 5]), pack_bf16x2(gv[8 * v + 6], gv[8 * v + 7]));
-                ob[v] = make_uint4(pack_bf16x2(uv[8 * v], uv[8 * v + 1]), pack_bf16x2(uv[8 * v + 2], uv[8 * v + 3]),
-                                   pack_bf16x2(uv[8 * v + 4], uv[8 * v + 5]), pack_bf16x2(uv[8 * v + 6], uv[8 * v + 7]));
-              }
+              w[i] = pack_bf16x2(v0[2 * i], v0[2 * i + 1]);
+              w[16 + i] = pack_bf16x2(v1[2 * i], v1[2 * i + 1]);
             }
           }
+          // the store that last used this buffer (kBufs chunks ago) has read it
+          if (lane == 0) bulk_wait_read<C::kBufs - 1>();
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4(row_addr + ((j ^ (lane & 7)) << 4), w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          fence_async_shared();
+          __syncwarp();
+          const int col0 = ntile * BN + c;
+          if (lane == 0 && col0 < p.N && row0 < p.M) {
+            tma_store_3d(&maps.out, buf, col0, row0, g);
+            bulk_commit();
+          }
+        }
+      } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+        // per chunk of 32 columns: TMA-load a and b (32 x 64-byte tiles, 64-byte swizzle)
+        // while the accumulator chunk comes out of TMEM, form dA and dB in place, and
+        // TMA-store them
+        const int row0 = mt * kBM + q * 32;
+        const int wi = warp - 2;
+        uint8_t* buf = staging + wi * C::kBufBytes;
+        const uint32_t rbase = smem_u32(buf) + lane * 64;
+        const int sw = (lane >> 1) & 3;
+        bool ok = true;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          const int col0 = ntile * BN + c;
+          const bool live = col0 < p.N && row0 < p.M;
+          if (lane == 0) {
+            bulk_wait_read<0>();  // the previous chunk's stores have read the buffer
+            if (live) {
+              mbar_arrive_expect_tx(&ebar[wi], 4096);
+              tma_load_3d(&maps.aux_a, buf, &ebar[wi], col0, row0, g);
+              tma_load_3d(&maps.aux_b, buf + 2048, &ebar[wi], col0, row0, g);
+            }
+          }
+          float v[32];
+          __syncwarp();
+          tmem_ld_32cols(tbase + c, v);
+          if (!live) continue;
+          const bool got = mbar_wait(&ebar[wi], eph, abort_v);
+          eph ^= 1u;
+          if (!__all_sync(0xffffffffu, got)) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t off = ((j ^ sw) << 4);
+            uint32_t aw[4], bw[4], da[4], db[4];
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(aw[0]), "=r"(aw[1]), "=r"(aw[2]), "=r"(aw[3]) : "r"(rbase + off));
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(bw[0]), "=r"(bw[1]), "=r"(bw[2]), "=r"(bw[3]) : "r"(rbase + 2048 + off));
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              float rda[2], rdb[2];
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                const float a = hh ? bf16_hi(aw[w]) : bf16_lo(aw[w]);
+                const float b = hh ? bf16_hi(bw[w]) : bf16_lo(bw[w]);
+                const float dh = v[8 * j + 2 * w + hh];
+                const float sg = 1.0f / (1.0f + expf(-a));
+                rda[hh] = dh * b * (sg * (1.0f + a * (1.0f - sg)));
+                rdb[hh] = dh * (a * sg);
+              }
+              da[w] = pack_bf16x2(rda[0], rda[1]);
+              db[w] = pack_bf16x2(rdb[0], rdb[1]);
+            }
+            st_shared_v4(rbase + off, da[0], da[1], da[2], da[3]);
+            st_shared_v4(rbase + 2048 + off, db[0], db[1], db[2], db[3]);
+          }
+          fence_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&maps.out, buf, col0, row0, g);
+            tma_store_3d(&maps.out2, buf + 2048, col0, row0, g);
+            bulk_commit();
+          }
+        }
+        if (!ok) {
+          *abort_flag = 1;
+          record_status(p.status, MOE_ERR_TIMEOUT);
+          break;
         }
       } else {
 #pragma unroll 1
@@ -418,23 +587,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (row_ok && col0 < p.N) {
           const long long off = g * p.out_gs + (long long)row * p.ldo + col0;
           const int nvalid = p.N - col0;  // multiple of 8
-          if constexpr (EPI == EPI_F32) {
-            float* o = static_cast<float*>(p.out) + off;
-#pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              if (i < nvalid) {
-                float4 f = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-                if (p.col_add != nullptr) {
-                  f.x += p.col_add[col0 + i];
-                  f.y += p.col_add[col0 + i + 1];
-                  f.z += p.col_add[col0 + i + 2];
-                  f.w += p.col_add[col0 + i + 3];
-                }
-                *reinterpret_cast<float4*>(o + i) = f;
-              }
-            }
-          } else if constexpr (EPI == EPI_BF16 || EPI == EPI_BF16_ADD_F32) {
-            if constexpr (EPI == EPI_BF16_ADD_F32) {
+          if constexpr (EPI == EPI_BF16_ADD_F32) {
+            {
               const float* ad = p.addend + (long long)row * p.add_ld + col0;
 #pragma unroll
               for (int i = 0; i < 32; i += 4) {
@@ -455,40 +609,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     make_uint4(pack_bf16x2(v[i], v[i + 1]), pack_bf16x2(v[i + 2], v[i + 3]),
                                pack_bf16x2(v[i + 4], v[i + 5]), pack_bf16x2(v[i + 6], v[i + 7]));
             }
-          } else if constexpr (EPI == EPI_SWIGLU_BWD) {
-            const long long aoff = g * p.aux_gs + (long long)row * p.aux_ld + col0;
-            const uint16_t* pa = static_cast<const uint16_t*>(p.aux_a) + aoff;
-            const uint16_t* pb = static_cast<const uint16_t*>(p.aux_b) + aoff;
-            uint16_t* oa = static_cast<uint16_t*>(p.out) + off;
-            uint16_t* ob = static_cast<uint16_t*>(p.out2) + off;
-#pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              if (i < nvalid) {
-                const uint4 av = *reinterpret_cast<const uint4*>(pa + i);
-                const uint4 bv = *reinterpret_cast<const uint4*>(pb + i);
-                const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
-                const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
-                uint32_t da[4], db[4];
-#pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                  float rda[2], rdb[2];
-#pragma unroll
-                  for (int h = 0; h < 2; ++h) {
-                    const float a = h ? bf16_hi(aw[w]) : bf16_lo(aw[w]);
-                    const float b = h ? bf16_hi(bw[w]) : bf16_lo(bw[w]);
-                    const float dh = v[i + 2 * w + h];
-                    const float sg = 1.0f / (1.0f + expf(-a));
-                    const float si = a * sg;
-                    rda[h] = dh * b * (sg * (1.0f + a * (1.0f - sg)));
-                    rdb[h] = dh * si;
-                  }
-                  da[w] = pack_bf16x2(rda[0], rda[1]);
-                  db[w] = pack_bf16x2(rdb[0], rdb[1]);
-                }
-                *reinterpret_cast<uint4*>(oa + i) = make_uint4(da[0], da[1], da[2], da[3]);
-                *reinterpret_cast<uint4*>(ob + i) = make_uint4(db[0], db[1], db[2], db[3]);
-              }
-            }
           }
           }  // row_ok && col0 < N
         }
@@ -499,6 +619,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    if (lane == 0) bulk_wait_all();  // every store of this warp has completed
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -527,23 +649,25 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-moe_status_t make_map(CUtensorMap* m, const Mat& t, uint32_t box_inner, uint32_t box_rows, const char* what) {
+moe_status_t make_map(CUtensorMap* m, const Mat& t, uint32_t box_inner, uint32_t box_rows, const char* what,
+                      CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, int esize = 2,
+                      CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   if (t.ptr == nullptr) return fail(MOE_ERR_INVALID_ARG, std::string("gemm operand is null: ") + what);
   if ((reinterpret_cast<uintptr_t>(t.ptr) & 15) != 0)
     return fail(MOE_ERR_INVALID_ARG, std::string("gemm operand not 16-byte aligned: ") + what);
-  if (t.inner <= 0 || t.rows <= 0 || t.groups <= 0 || t.ld < t.inner || (t.ld * 2) % 16 != 0 ||
-      (t.gs * 2) % 16 != 0)
+  if (t.inner <= 0 || t.rows <= 0 || t.groups <= 0 || t.ld < t.inner || (t.ld * esize) % 16 != 0 ||
+      (t.gs * esize) % 16 != 0)
     return fail(MOE_ERR_INVALID_ARG, std::string("gemm operand has a bad shape or stride: ") + what);
   auto fn = encode_fn();
   if (fn == nullptr) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(t.inner), static_cast<cuuint64_t>(t.rows),
                         static_cast<cuuint64_t>(t.groups)};
   const int64_t gs = t.groups > 1 ? t.gs : t.ld * t.rows;
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(t.ld * 2), static_cast<cuuint64_t>(gs * 2)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(t.ld * esize), static_cast<cuuint64_t>(gs * esize)};
   cuuint32_t box[3] = {box_inner, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(t.ptr), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  CUresult r = fn(m, dtype, 3, const_cast<void*>(t.ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(MOE_ERR_CUDA, std::string("cuTensorMapEncodeTiled failed for ") + what + " (" +
@@ -554,7 +678,7 @@ moe_status_t make_map(CUtensorMap* m, const Mat& t, uint32_t box_inner, uint32_t
 template <int BN, bool A_MN, bool B_MN, int EPI>
 moe_status_t launch_instance(const TmaMaps& maps, const KParams& kp, int grid, cudaStream_t st) {
   auto kern = gemm_kernel<BN, A_MN, B_MN, EPI>;
-  const int smem = Cfg<BN>::kSmem;
+  const int smem = Cfg<BN, A_MN && B_MN, EPI == EPI_SWIGLU>::kSmem;
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -589,6 +713,8 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
   if (a.epi == EPI_SWIGLU && (a.nseg != 1 || a.b_mn || a.N % (a.bn / 2) != 0))
     return fail(MOE_ERR_UNSUPPORTED, "SwiGLU gemm needs one K-major segment and N a multiple of BN/2");
   if (a.N % 8 != 0) return fail(MOE_ERR_UNSUPPORTED, "gemm N must be a multiple of 8");
+  if (a.a_mn && a.b_mn && a.ragged == 1)
+    return fail(MOE_ERR_UNSUPPORTED, "gemm with both operands MN-major takes no ragged rows");
   if (a.out == nullptr) return fail(MOE_ERR_INVALID_ARG, "gemm output is null");
 
   TmaMaps maps;
@@ -612,6 +738,44 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
   }
   if (a.epi == EPI_SWIGLU) {
     moe_status_t r = make_map(&maps.bv, a.Bv, 64, a.bn / 2, "B value");
+    if (r != MOE_OK) return r;
+  }
+  if (a.epi == EPI_SWIGLU || a.epi == EPI_SWIGLU_BWD) {
+    // 32 x 32 bf16 tiles (64-byte rows) of the element-wise operands and results
+    auto tile = [&](CUtensorMap* m, const void* ptr, int64_t ld, int64_t gs, const char* what) {
+      Mat o;
+      o.ptr = ptr;
+      o.inner = a.N;
+      o.rows = a.M;
+      o.groups = a.groups;
+      o.ld = ld;
+      o.gs = a.groups > 1 ? gs : ld * a.M;
+      return make_map(m, o, 32, 32, what, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, CU_TENSOR_MAP_SWIZZLE_64B);
+    };
+    moe_status_t r = tile(&maps.out, a.out, a.ldo, a.out_gs, "output");
+    if (r != MOE_OK) return r;
+    if (a.epi == EPI_SWIGLU && a.save_a != nullptr) {
+      if (a.save_b == nullptr) return fail(MOE_ERR_INVALID_ARG, "SwiGLU saves both pre-activations or neither");
+      if ((r = tile(&maps.aux_a, a.save_a, a.ldo, a.out_gs, "saved gate")) != MOE_OK) return r;
+      if ((r = tile(&maps.aux_b, a.save_b, a.ldo, a.out_gs, "saved value")) != MOE_OK) return r;
+    }
+    if (a.epi == EPI_SWIGLU_BWD) {
+      if ((r = tile(&maps.out2, a.out2, a.ldo, a.out_gs, "dB")) != MOE_OK) return r;
+      if ((r = tile(&maps.aux_a, a.aux_a, a.aux_ld, a.aux_gs, "a")) != MOE_OK) return r;
+      if ((r = tile(&maps.aux_b, a.aux_b, a.aux_ld, a.aux_gs, "b")) != MOE_OK) return r;
+    }
+  }
+  if (a.epi == EPI_F32 || a.epi == EPI_BF16) {
+    Mat o;
+    o.ptr = a.out;
+    o.inner = a.N;
+    o.rows = a.M;
+    o.groups = a.groups;
+    o.ld = a.ldo;
+    o.gs = a.groups > 1 ? a.out_gs : a.ldo * a.M;
+    moe_status_t r = a.epi == EPI_F32
+                         ? make_map(&maps.out, o, 32, 32, "output", CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4)
+                         : make_map(&maps.out, o, 64, 32, "output");
     if (r != MOE_OK) return r;
   }
   kp.m_fastest = a.m_fastest ? 1 : 0;

@@ -736,9 +736,9 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
     a.groups = p->E;
     a.ragged = 2;
     a.group_rows = c.rows;
+    a.m_fastest = false;  // concurrent tiles write whole rows of dW
     a.A[0] = mat(dye, dl, Cr, E);
     a.B[0] = mat(c.he, h, Cr, E);
-    a.m_fastest = true;
     a.out = gr->w2;
     a.ldo = h;
     a.out_gs = dl * h;
@@ -776,9 +776,9 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
     a.groups = p->E;
     a.ragged = 2;
     a.group_rows = c.rows;
+    a.m_fastest = false;  // concurrent tiles write whole rows of dW
     a.A[0] = mat(dae, h, Cr, E);
     a.B[0] = mat(c.xe, dl, Cr, E);
-    a.m_fastest = true;
     a.out = gr->w1;
     a.ldo = dl;
     a.out_gs = h * dl;

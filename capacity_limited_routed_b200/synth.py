@@ -69,6 +69,11 @@ TRAIN = FULL.with_(name="train", backward=True, seed=4)
 
 WORKLOADS = {1: TINY, 2: MID, 3: FULL, 4: SKEWED, 5: TRAIN}
 
+# A small case of the full-width kernels for profiler captures: full widths, 24 experts
+# over 4 destinations and T=1024, so each expert still receives ~341 of C_r=393 rows
+# as in the full layer, with ~4.5 GB on the device instead of ~50 GB.
+PROFILE = TRAIN.with_(name="profile", T=1024, n_experts=24, n_dest=4, seed=5)
+
 
 def to_bf16_bits(a: np.ndarray) -> np.ndarray:
     """float32 -> bfloat16 bit patterns (uint16), round to nearest even."""
