@@ -59,6 +59,15 @@ struct KParams {
   int32_t* status;
 };
 
+// Tuning of the weight-gradient (write-bound) instance: pipeline stages and staging
+// buffers per epilogue warp.
+#ifndef MOE_WB_STAGES
+#define MOE_WB_STAGES 4
+#endif
+#ifndef MOE_WB_BUFS
+#define MOE_WB_BUFS 2
+#endif
+
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kThreads = 192;
@@ -74,9 +83,9 @@ struct Cfg {
   static constexpr int kABytes = kBM * kBK * 2;  // 16 KB
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStage = kABytes + kBBytes;
-  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  static constexpr int kStages = WRITE_BOUND ? MOE_WB_STAGES : ((BN == 256) ? 4 : 6);
   static constexpr int kTmemCols = 2 * BN;
-  static constexpr int kBufs = WRITE_BOUND ? 2 : 1;          // staging buffers per epilogue warp
+  static constexpr int kBufs = WRITE_BOUND ? MOE_WB_BUFS : 1;  // staging buffers per epilogue warp
   // a buffer holds 32 rows x 128 bytes (float32 / bf16 outputs, or two 32 x 64-byte
   // bf16 tiles); the forward SwiGLU stages three 32 x 64-byte tiles (H, a, b)
   static constexpr int kBufBytes = SWIGLU ? 6144 : 4096;
@@ -414,6 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const uint32_t tbase = tmem_base + lane_off + static_cast<uint32_t>(acc * BN);
+      bool released = false;  // accumulator handed back to the MMA warp early
 
       if constexpr (EPI == EPI_SWIGLU) {
         // per chunk of 32 output columns: H, a, b as three 32 x 64-byte tiles (64-byte
@@ -424,19 +434,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t rbase = smem_u32(buf) + lane * 64;
         const int sw = (lane >> 1) & 3;
 #pragma unroll 1
-        for (int c = 0; c < BN / 2; c += 32) {
-          float gv[32], uv[32];
+        for (int c2 = 0; c2 < BN / 2; c2 += 64) {
+          // two chunks of gate and value columns (four TMEM loads) per wait
+          uint32_t rg[2][32], ru[2][32];
           __syncwarp();
-          tmem_ld_32cols(tbase + c, gv);
-          tmem_ld_32cols(tbase + BN / 2 + c, uv);
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            tmem_ld_32cols_async(tbase + c2 + 32 * i, rg[i]);
+            tmem_ld_32cols_async(tbase + BN / 2 + c2 + 32 * i, ru[i]);
+          }
+          tmem_wait_ld();
+          if (c2 + 64 >= BN / 2) {
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+            released = true;
+          }
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+          const int c = c2 + 32 * i;
           uint32_t h[16], ga[16], gb[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float a0 = gv[2 * i], a1 = gv[2 * i + 1];
+          for (int e2 = 0; e2 < 16; ++e2) {
+            const float a0 = __uint_as_float(rg[i][2 * e2]), a1 = __uint_as_float(rg[i][2 * e2 + 1]);
+            const float u0 = __uint_as_float(ru[i][2 * e2]), u1 = __uint_as_float(ru[i][2 * e2 + 1]);
             const float s0 = a0 / (1.0f + expf(-a0)), s1 = a1 / (1.0f + expf(-a1));
-            h[i] = pack_bf16x2(s0 * uv[2 * i], s1 * uv[2 * i + 1]);
-            ga[i] = pack_bf16x2(a0, a1);
-            gb[i] = pack_bf16x2(uv[2 * i], uv[2 * i + 1]);
+            h[e2] = pack_bf16x2(s0 * u0, s1 * u1);
+            ga[e2] = pack_bf16x2(a0, a1);
+            gb[e2] = pack_bf16x2(u0, u1);
           }
           if (lane == 0) bulk_wait_read<0>();  // the previous chunk's stores have read the buffer
           __syncwarp();
@@ -458,15 +482,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             bulk_commit();
           }
+          }
         }
-      } else if constexpr (EPI == EPI_F32 || EPI == EPI_BF16) {
-        // stage 32 rows x 128 bytes in shared memory (128-byte swizzle: 16-byte piece j
-        // of row r at j ^ (r & 7)), then one TMA tensor store per chunk; rows past M and
-        // columns past N are clipped by the tensor map
+      } else if constexpr ((EPI == EPI_F32 || EPI == EPI_BF16) && (A_MN && B_MN)) {
+        // Weight gradients: one 32-column chunk at a time (a compact loop measured
+        // fastest for these short contractions), each staged as 32 rows x 128 bytes
+        // (128-byte swizzle: 16-byte piece j of row r at j ^ (r & 7)) and written with
+        // one TMA tensor store; rows past M and columns past N are clipped by the map.
         constexpr int kChunk = (EPI == EPI_F32) ? 32 : 64;
         const int row0 = mt * kBM + q * 32;
 #pragma unroll 1
         for (int c = 0; c < BN; c += kChunk) {
+          // a chunk wholly outside the output touches no staging buffer: every buffer
+          // write must be followed by a committed store, or the ring's wait-group count
+          // no longer covers the store that last read the buffer
+          if (ntile * BN + c >= p.N || row0 >= p.M) break;
           uint8_t* buf = staging + ((warp - 2) * C::kBufs + ring) * C::kBufBytes;
           if (++ring == C::kBufs) ring = 0;
           const uint32_t row_addr = smem_u32(buf) + lane * 128;
@@ -475,13 +505,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (EPI == EPI_F32) {
             float v[32];
             tmem_ld_32cols(tbase + c, v);
-            const int col0 = ntile * BN + c;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              float x = v[i];
-              if (p.col_add != nullptr && col0 + i < p.N) x += p.col_add[col0 + i];
-              w[i] = __float_as_uint(x);
-            }
+            for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(v[i]);
           } else {
             float v0[32], v1[32];
             tmem_ld_32cols(tbase + c, v0);
@@ -500,10 +525,67 @@ __global__ void __launch_bounds__(kThreads, 1)
             st_shared_v4(row_addr + ((j ^ (lane & 7)) << 4), w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
           fence_async_shared();
           __syncwarp();
-          const int col0 = ntile * BN + c;
-          if (lane == 0 && col0 < p.N && row0 < p.M) {
-            tma_store_3d(&maps.out, buf, col0, row0, g);
+          if (lane == 0) {
+            tma_store_3d(&maps.out, buf, ntile * BN + c, row0, g);
             bulk_commit();
+          }
+        }
+      } else if constexpr (EPI == EPI_F32 || EPI == EPI_BF16) {
+        // Four TMEM loads (128 columns) in flight before one wait, then the 128 columns
+        // leave through shared memory: 32 rows x 128 bytes per staging buffer (128-byte
+        // swizzle: 16-byte piece j of row r at j ^ (r & 7)), one TMA tensor store each.
+        // Rows past M and columns past N are clipped by the tensor map.  The accumulator
+        // is released as soon as the whole tile is in registers.
+        constexpr int kChunk = (EPI == EPI_F32) ? 32 : 64;  // columns per 128-byte row
+        const int row0 = mt * kBM + q * 32;
+#pragma unroll 1
+        for (int half = 0; half < BN; half += 128) {
+          uint32_t r[4][32];
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) tmem_ld_32cols_async(tbase + half + 32 * i, r[i]);
+          tmem_wait_ld();
+          if (half + 128 >= BN) {
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+            released = true;
+          }
+#pragma unroll
+          for (int cc = 0; cc < 128 / kChunk; ++cc) {
+            uint32_t w[32];
+            const int col0 = ntile * BN + half + cc * kChunk;
+            // see the weight-gradient path: no buffer write without a committed store
+            if (col0 >= p.N || row0 >= p.M) continue;
+            if constexpr (EPI == EPI_F32) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                float x = __uint_as_float(r[cc][i]);
+                if (p.col_add != nullptr && col0 + i < p.N) x += p.col_add[col0 + i];
+                w[i] = __float_as_uint(x);
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                w[i] = pack_bf16x2(__uint_as_float(r[2 * cc][2 * i]), __uint_as_float(r[2 * cc][2 * i + 1]));
+                w[16 + i] =
+                    pack_bf16x2(__uint_as_float(r[2 * cc + 1][2 * i]), __uint_as_float(r[2 * cc + 1][2 * i + 1]));
+              }
+            }
+            uint8_t* buf = staging + ((warp - 2) * C::kBufs + ring) * C::kBufBytes;
+            if (++ring == C::kBufs) ring = 0;
+            const uint32_t row_addr = smem_u32(buf) + lane * 128;
+            // the store that last used this buffer (kBufs chunks ago) has read it
+            if (lane == 0) bulk_wait_read<C::kBufs - 1>();
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              st_shared_v4(row_addr + ((j ^ (lane & 7)) << 4), w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+            fence_async_shared();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&maps.out, buf, col0, row0, g);
+              bulk_commit();
+            }
           }
         }
       } else if constexpr (EPI == EPI_SWIGLU_BWD) {
@@ -614,8 +696,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncwarp();
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      if (!released) {
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }

@@ -26,8 +26,8 @@ struct moe_plan {
     size_t z, logits, idx, gate, slot, rows, xe, ae, be, he, ye, r, as, bs, hsh, bytes;
   } saved, infer;
   // scratch layouts
-  size_t ws_scan, ws_pools, ws_ctx, ws_fwd_bytes;                        // forward
-  size_t ws_ffn_xe, ws_ffn_he, ws_ffn_rows, ws_ffn_bytes;                // moe_expert_ffn alone
+  size_t ws_scan, ws_pools, ws_rowmap, ws_ctx, ws_fwd_bytes;             // forward
+  size_t ws_ffn_xe, ws_ffn_he, ws_ffn_rows, ws_ffn_rowmap, ws_ffn_bytes;  // moe_expert_ffn alone
   size_t b_dr, b_das, b_dbs, b_dye, b_dg, b_dae, b_dbe, b_dxe, b_dlog, b_dzr, b_dz, ws_bwd_bytes;
   size_t pools_bytes, expert_out_bytes, slot_bytes, stats_bytes, ws_bytes;
 };
@@ -152,12 +152,14 @@ void layout(moe_plan& p) {
   size_t off = 0;
   p.ws_scan = take(off, scan_scratch_ints(p.g) * 4);
   p.ws_pools = take(off, p.pools_bytes);
+  p.ws_rowmap = take(off, unpack_scratch_ints(p.g) * 4);
   p.ws_ctx = take(off, p.infer.bytes);  // used only when the forward keeps no context
   p.ws_fwd_bytes = off;
   off = 0;
   p.ws_ffn_xe = take(off, E * Cr * dl * 2);
   p.ws_ffn_he = take(off, E * Cr * h * 2);
   p.ws_ffn_rows = take(off, E * 4);
+  p.ws_ffn_rowmap = take(off, unpack_scratch_ints(p.g) * 4);
   p.ws_ffn_bytes = off;
   off = 0;
   p.b_dr = take(off, T * dl * 2);
@@ -261,12 +263,12 @@ CtxPtrs ctx_ptrs(const moe_plan& p, void* base, bool training) {
 
 // receiver unpack + grouped SwiGLU experts (shared by moe_expert_ffn and moe_forward)
 moe_status_t run_experts(const moe_plan& p, const uint16_t* w1, const uint16_t* w3, const uint16_t* w2,
-                         const uint16_t* pools, uint16_t* xe, int32_t* rows, uint16_t* ae, uint16_t* be, uint16_t* he,
-                         uint16_t* ye, int32_t* status, cudaStream_t st) {
+                         const uint16_t* pools, uint16_t* xe, int32_t* rows, int32_t* row_map, uint16_t* ae,
+                         uint16_t* be, uint16_t* he, uint16_t* ye, int32_t* status, cudaStream_t st) {
   const Geo& g = p.g;
   {
     ProfScope ps("experts.unpack", st);
-    MOE_TRY(launch_unpack(g, pools, xe, rows, status, st));
+    MOE_TRY(launch_unpack(g, pools, xe, rows, row_map, status, st));
     MOE_TRY(launch_zero_tail_rows(g, xe, p.dl, rows, st));
   }
   GemmArgs a;
@@ -479,8 +481,9 @@ moe_status_t moe_expert_ffn(moe_plan_t p, const moe_expert_weights_t* w, const u
   MOE_TRY(device_ok());
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int32_t* rows = expert_rows ? expert_rows : at<int32_t>(ws, p->ws_ffn_rows);
-  return run_experts(*p, w->w1, w->w3, w->w2, pools, at<uint16_t>(ws, p->ws_ffn_xe), rows, nullptr, nullptr,
-                     at<uint16_t>(ws, p->ws_ffn_he), expert_out, nullptr, st);
+  return run_experts(*p, w->w1, w->w3, w->w2, pools, at<uint16_t>(ws, p->ws_ffn_xe), rows,
+                     at<int32_t>(ws, p->ws_ffn_rowmap), nullptr, nullptr, at<uint16_t>(ws, p->ws_ffn_he), expert_out,
+                     nullptr, st);
 }
 
 moe_status_t moe_combine(moe_plan_t p, const uint16_t* expert_out, const float* topk_gate, const int32_t* topk_idx,
@@ -558,7 +561,8 @@ moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const uint16_t* x
     ProfScope ps("fwd.dispatch_pack", st);
     MOE_TRY(launch_pack(g, c.z, c.idx, c.slot, s, pools, st));
   }
-  MOE_TRY(run_experts(*p, w->w1, w->w3, w->w2, pools, c.xe, c.rows, c.ae, c.be, c.he, c.ye, status, st));
+  MOE_TRY(run_experts(*p, w->w1, w->w3, w->w2, pools, c.xe, c.rows, at<int32_t>(ws, p->ws_rowmap), c.ae, c.be,
+                      c.he, c.ye, status, st));
   {
     ProfScope ps("fwd.combine", st);
     MOE_TRY(launch_combine(g, c.ye, c.gate, c.idx, c.slot, c.r, st));

@@ -332,11 +332,18 @@ __global__ void pack_kernel(const uint16_t* __restrict__ z, const int32_t* __res
     }
     __syncwarp();
     const uint4* src = reinterpret_cast<const uint4*>(z + static_cast<long long>(t) * dl);
-    for (int v = lane; v < nvec; v += 32) {
-      const uint4 val = src[v];
+    for (int v0 = lane; v0 < nvec; v0 += 32 * 8) {
+      uint4 val[8];  // up to 8 vectors of the row in flight per lane, then k copies
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (v0 + 32 * u < nvec) val[u] = src[v0 + 32 * u];
       for (int j = 0; j < k; ++j) {
         const long long d = s_dst[wib][j];
-        if (d >= 0) reinterpret_cast<uint4*>(pools + d)[v] = val;
+        if (d < 0) continue;
+        uint4* dst = reinterpret_cast<uint4*>(pools + d);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = val[u];
       }
     }
     if (lane < k && s_j >= 0 && s_j < Cs && e_j >= 0 && e_j < E) {
@@ -360,15 +367,14 @@ __global__ void pack_empty_headers(const int32_t* __restrict__ pool_fill, int NP
   }
 }
 
-// receiver: one block per pool.  Rows are visited in pool order in tiles of the block
-// size; a row whose packed id names local expert q of this pool gets the next slot of
-// q; the first C_r rows of each expert are gathered into xe[e][slot].
-__global__ void unpack_kernel(const uint16_t* __restrict__ pools, int Cs, int Cr, int dl, int L, int P, int W,
-                              uint16_t* __restrict__ xe, int32_t* __restrict__ rows_out,
-                              int32_t* __restrict__ status) {
+// receiver, pass 1: one block per pool.  Rows are visited in pool order in tiles of the
+// block size; a row whose packed id names local expert q of this pool gets the next slot
+// of q.  The first C_r rows of each expert are mapped to their receive-buffer row
+// (e * C_r + slot) in row_map; other rows map to -1.
+__global__ void unpack_rank_kernel(const uint16_t* __restrict__ pools, int Cs, int Cr, int dl, int L, int P, int W,
+                                   int32_t* __restrict__ row_map, int32_t* __restrict__ rows_out,
+                                   int32_t* __restrict__ status) {
   constexpr int kTile = 256;
-  __shared__ int s_slot[kTile];
-  __shared__ int s_exp[kTile];
   __shared__ int s_warp_cnt[kTile / 32][32];
   __shared__ int s_run[32];
   const int pool = blockIdx.x;
@@ -403,26 +409,43 @@ __global__ void unpack_kernel(const uint16_t* __restrict__ pools, int Cs, int Cr
       for (int w = 0; w < warp; ++w) before += s_warp_cnt[w][q];
       slot = before + rank;
     }
-    s_slot[threadIdx.x] = (slot >= 0 && slot < Cr) ? slot : -1;
-    s_exp[threadIdx.x] = q >= 0 ? e_first + q : -1;
+    if (r < Cs)
+      row_map[static_cast<long long>(pool) * Cs + r] =
+          (slot >= 0 && slot < Cr) ? (e_first + q) * Cr + slot : -1;
     __syncthreads();
     if (threadIdx.x < P) {
       int tot = 0;
       for (int w = 0; w < kTile / 32; ++w) tot += s_warp_cnt[w][threadIdx.x];
       s_run[threadIdx.x] += tot;
     }
-    // gather the kept rows of this tile: one warp per row
-    const int nvec = dl / 8;
-    for (int i = warp; i < kTile && r0 + i < Cs; i += kTile / 32) {
-      const int sl = s_slot[i];
-      if (sl < 0) continue;
-      const uint4* src = reinterpret_cast<const uint4*>(pbase + (r0 + i) * row_elems);
-      uint4* dst = reinterpret_cast<uint4*>(xe + (static_cast<long long>(s_exp[i]) * Cr + sl) * dl);
-      for (int v = lane; v < nvec; v += 32) dst[v] = src[v];
-    }
     __syncthreads();
   }
   if (threadIdx.x < P) rows_out[e_first + threadIdx.x] = min(s_run[threadIdx.x], Cr);
+}
+
+// receiver, pass 2: one warp per pool row, up to 8 vectors per lane in flight
+__global__ void unpack_copy_kernel(const uint16_t* __restrict__ pools, const int32_t* __restrict__ row_map,
+                                   long long n_rows, int dl, uint16_t* __restrict__ xe) {
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  const long long row_elems = dl + 8;
+  const int nvec = dl / 8;
+  for (long long r = static_cast<long long>(blockIdx.x) * warps + (threadIdx.x >> 5); r < n_rows;
+       r += static_cast<long long>(gridDim.x) * warps) {
+    const int d = row_map[r];
+    if (d < 0) continue;
+    const uint4* src = reinterpret_cast<const uint4*>(pools + r * row_elems);
+    uint4* dst = reinterpret_cast<uint4*>(xe + static_cast<long long>(d) * dl);
+    for (int v0 = lane; v0 < nvec; v0 += 32 * 8) {
+      uint4 val[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (v0 + 32 * u < nvec) val[u] = src[v0 + 32 * u];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = val[u];
+    }
+  }
 }
 
 // rows [n_e, min(round_up(n_e, 128), C_r)) of each expert's buffer become zero, so that
@@ -480,13 +503,22 @@ __global__ void combine_kernel(const uint16_t* __restrict__ ye, const float* __r
       s_g[wib][lane] = ok ? gate[a] : 0.0f;
     }
     __syncwarp();
-    for (int v = lane; v < nvec; v += 32) {
-      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int v = lane; v < nvec; v += 64) {
+      const bool two = v + 32 < nvec;
+      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0}, acc2[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll 4
       for (int j = 0; j < k; ++j) {
         const long long rj = s_row[wib][j];
-        if (rj >= 0) acc8(acc, reinterpret_cast<const uint4*>(ye + rj * dl)[v], s_g[wib][j]);
+        if (rj < 0) continue;
+        const uint4* yrow = reinterpret_cast<const uint4*>(ye + rj * dl);
+        const uint4 a = yrow[v];
+        const uint4 b = two ? yrow[v + 32] : make_uint4(0, 0, 0, 0);
+        acc8(acc, a, s_g[wib][j]);
+        acc8(acc2, b, s_g[wib][j]);
       }
-      reinterpret_cast<uint4*>(r + static_cast<long long>(t) * dl)[v] = pack8(acc);
+      uint4* out = reinterpret_cast<uint4*>(r + static_cast<long long>(t) * dl);
+      out[v] = pack8(acc);
+      if (two) out[v + 32] = pack8(acc2);
     }
     __syncwarp();
   }
@@ -561,15 +593,27 @@ __global__ void undispatch_kernel(const uint16_t* __restrict__ dxe, const float*
       s_row[wib][lane] = (rs >= 0 && rs < Cr && e_j >= 0) ? static_cast<long long>(e_j) * Cr + rs : -1;
     }
     __syncwarp();
-    for (int v = lane; v < nvec; v += 32) {
-      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int v = lane; v < nvec; v += 64) {
+      const bool two = v + 32 < nvec;
+      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0}, acc2[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll 4
       for (int j = 0; j < k; ++j) {
         const long long rj = s_row[wib][j];
-        if (rj >= 0) acc8(acc, reinterpret_cast<const uint4*>(dxe + rj * dl)[v], 1.0f);
+        if (rj < 0) continue;
+        const uint4* xrow = reinterpret_cast<const uint4*>(dxe + rj * dl);
+        const uint4 a = xrow[v];
+        const uint4 b = two ? xrow[v + 32] : make_uint4(0, 0, 0, 0);
+        acc8(acc, a, 1.0f);
+        acc8(acc2, b, 1.0f);
       }
       float4* o = reinterpret_cast<float4*>(dz + static_cast<long long>(t) * dl + 8 * v);
       o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
       o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      if (two) {
+        float4* o2 = reinterpret_cast<float4*>(dz + static_cast<long long>(t) * dl + 8 * (v + 32));
+        o2[0] = make_float4(acc2[0], acc2[1], acc2[2], acc2[3]);
+        o2[1] = make_float4(acc2[4], acc2[5], acc2[6], acc2[7]);
+      }
     }
     // softmax backward: dl_j = g_j (dg_j - sum_i g_i dg_i)
     float s = lane < k ? g_j * dg_j : 0.0f;
@@ -700,11 +744,16 @@ moe_status_t launch_pack(const Geo& g, const uint16_t* z, const int32_t* idx, co
   return cuda_check(cudaGetLastError(), "pack");
 }
 
-moe_status_t launch_unpack(const Geo& g, const uint16_t* pools, uint16_t* xe, int32_t* rows, int32_t* status,
-                           cudaStream_t st) {
+size_t unpack_scratch_ints(const Geo& g) { return static_cast<size_t>(g.NP) * g.Cs; }
+
+moe_status_t launch_unpack(const Geo& g, const uint16_t* pools, uint16_t* xe, int32_t* rows, int32_t* row_map,
+                           int32_t* status, cudaStream_t st) {
   if (g.P > 32) return fail(MOE_ERR_UNSUPPORTED, "more than 32 experts per wave");
-  unpack_kernel<<<g.NP, 256, 0, st>>>(pools, g.Cs, g.Cr, g.dl, g.L, g.P, g.W, xe, rows, status);
-  count_launch();
+  unpack_rank_kernel<<<g.NP, 256, 0, st>>>(pools, g.Cs, g.Cr, g.dl, g.L, g.P, g.W, row_map, rows, status);
+  const long long n_rows = static_cast<long long>(g.NP) * g.Cs;
+  const int warps = 8;
+  unpack_copy_kernel<<<blocks_for(n_rows, warps), 32 * warps, 0, st>>>(pools, row_map, n_rows, g.dl, xe);
+  count_launch(2);
   return cuda_check(cudaGetLastError(), "unpack");
 }
 

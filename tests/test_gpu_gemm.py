@@ -66,3 +66,22 @@ def test_gemm_single_tile_exact_small_integers(M):
     D = torch.zeros((m, n), dtype=torch.float32, device=dev())
     M.moe_gemm_bf16(m, n, k, a.to(dev()), 0, b.to(dev()), 0, D)
     assert torch.equal(D.double().cpu(), ref)
+
+
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 1), (1, 0)])
+@pytest.mark.parametrize("n", [96, 160])
+def test_gemm_partial_tiles_many(M, a_mn, b_mn, n):
+    """Output widths that leave most of each 256-wide tile empty, over many tiles and a
+    short contraction: the epilogue's staging buffers must never be rewritten while a
+    store still reads them."""
+    m, k = 4096, 64
+    a, b = _operands(m, n, k, seed=n + 2 * a_mn + b_mn)
+    ref = a.double() @ b.double().T
+    A = (a.T.contiguous() if a_mn else a).to(dev())
+    B = (b.T.contiguous() if b_mn else b).to(dev())
+    for _ in range(3):
+        D = torch.full((m, n), float("nan"), dtype=torch.float32, device=dev())
+        M.moe_gemm_bf16(m, n, k, A, a_mn, B, b_mn, D)
+        torch.cuda.synchronize()
+        err = (D.double().cpu() - ref).abs().max().item()
+        assert err <= 1e-4 * rms(ref.numpy()), err
