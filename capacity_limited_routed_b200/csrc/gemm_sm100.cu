@@ -65,12 +65,21 @@ struct KParams {
 #define MOE_WB_STAGES 4
 #endif
 #ifndef MOE_WB_BUFS
-#define MOE_WB_BUFS 2
+#define MOE_WB_BUFS 1
 #endif
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kThreads = 192;
+constexpr int kThreads = 192;  // producer warp, MMA warp, four epilogue warps
+
+// Epilogue warps of an instance: the weight-gradient instance (both operands
+// MN-major) drains 128 x 256 float32 per short tile and gets two warps per TMEM
+// lane quarter, each taking half of the tile's columns.
+template <bool WRITE_BOUND>
+struct Roles {
+  static constexpr int kEpiWarps = WRITE_BOUND ? 8 : 4;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+};
 constexpr int kMaxGroups = 1024;
 
 // WRITE_BOUND: the weight-gradient instance (both operands MN-major).  Its K is the
@@ -86,10 +95,11 @@ struct Cfg {
   static constexpr int kStages = WRITE_BOUND ? MOE_WB_STAGES : ((BN == 256) ? 4 : 6);
   static constexpr int kTmemCols = 2 * BN;
   static constexpr int kBufs = WRITE_BOUND ? MOE_WB_BUFS : 1;  // staging buffers per epilogue warp
+  static constexpr int kEpiWarps = Roles<WRITE_BOUND>::kEpiWarps;
   // a buffer holds 32 rows x 128 bytes (float32 / bf16 outputs, or two 32 x 64-byte
   // bf16 tiles); the forward SwiGLU stages three 32 x 64-byte tiles (H, a, b)
   static constexpr int kBufBytes = SWIGLU ? 6144 : 4096;
-  static constexpr int kStaging = 4 * kBufs * kBufBytes;
+  static constexpr int kStaging = kEpiWarps * kBufs * kBufBytes;
   static constexpr int kBarBytes = 8 * (2 * kStages + 5 + 4) + 16;
   static constexpr int kPrefixInts = WRITE_BOUND ? 0 : kMaxGroups + 1;
   static constexpr int kSmem = 1024 + kStages * kStage + kStaging + kBarBytes + 4 * kPrefixInts;
@@ -169,7 +179,7 @@ struct Sched {
 };
 
 template <int BN, bool A_MN, bool B_MN, int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
     gemm_kernel(const __grid_constant__ TmaMaps maps, const KParams p) {
   using C = Cfg<BN, A_MN && B_MN, EPI == EPI_SWIGLU>;
   extern __shared__ uint8_t smem_raw[];
@@ -195,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 32 * C::kEpiWarps);
     }
     mbar_init(drain, 1);
     for (int w = 0; w < 4; ++w) mbar_init(&ebar[w], 1);
@@ -384,6 +394,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int row_in_tile = q * 32 + lane;
+    const int ew = warp - 2;  // epilogue warp index
+    // with eight epilogue warps, warps 2..5 take columns [0, BN/2), warps 6..9 the rest
+    const int col_lo = (C::kEpiWarps == 8) ? (ew >> 2) * (BN / 2) : 0;
+    const int col_hi = (C::kEpiWarps == 8) ? col_lo + BN / 2 : BN;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -399,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (kb_total == 0) {
         // an empty contraction (group with no rows): the product is zero
         if (row_ok && (EPI == EPI_BF16 || EPI == EPI_F32)) {
-          for (int c = 0; c < BN; c += 8) {
+          for (int c = col_lo; c < col_hi; c += 8) {
             const int col = ntile * BN + c;
             if (col >= p.N) break;
             if (EPI == EPI_BF16) {
@@ -430,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // swizzle: 16-byte piece j of row r at j ^ ((r >> 1) & 3)), three TMA stores
         const int n_out0 = ntile * (BN / 2);
         const int row0 = mt * kBM + q * 32;
-        uint8_t* buf = staging + (warp - 2) * C::kBufBytes;
+        uint8_t* buf = staging + ew * C::kBufBytes;
         const uint32_t rbase = smem_u32(buf) + lane * 64;
         const int sw = (lane >> 1) & 3;
 #pragma unroll 1
@@ -485,21 +499,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else if constexpr ((EPI == EPI_F32 || EPI == EPI_BF16) && (A_MN && B_MN)) {
-        // Weight gradients: one 32-column chunk at a time (a compact loop measured
-        // fastest for these short contractions), each staged as 32 rows x 128 bytes
-        // (128-byte swizzle: 16-byte piece j of row r at j ^ (r & 7)) and written with
-        // one TMA tensor store; rows past M and columns past N are clipped by the map.
+        // Weight gradients: each tile's short main loop is worth less than its 128 KB
+        // result, and TMA stores would queue the next tile's operand loads behind them.
+        // The result leaves through the load/store path instead: one 32-column chunk at
+        // a time, staged as 32 rows x 128 bytes (128-byte swizzle: 16-byte piece j of
+        // row r at j ^ (r & 7)) and read back four rows per instruction, so every store
+        // instruction writes four whole 128-byte lines.
         constexpr int kChunk = (EPI == EPI_F32) ? 32 : 64;
+        constexpr int kEsz = (EPI == EPI_F32) ? 4 : 2;
         const int row0 = mt * kBM + q * 32;
+        uint8_t* buf = staging + ew * C::kBufs * C::kBufBytes;
+        const uint32_t sbase = smem_u32(buf);
+        const int piece = lane & 7;    // 16-byte piece of a row this lane reads back
+        const int rsub = lane >> 3;    // row within each group of four
+        char* obase = static_cast<char*>(p.out) + static_cast<long long>(g) * p.out_gs * kEsz;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += kChunk) {
-          // a chunk wholly outside the output touches no staging buffer: every buffer
-          // write must be followed by a committed store, or the ring's wait-group count
-          // no longer covers the store that last read the buffer
-          if (ntile * BN + c >= p.N || row0 >= p.M) break;
-          uint8_t* buf = staging + ((warp - 2) * C::kBufs + ring) * C::kBufBytes;
-          if (++ring == C::kBufs) ring = 0;
-          const uint32_t row_addr = smem_u32(buf) + lane * 128;
+        for (int c = col_lo; c < col_hi; c += kChunk) {
+          const int col0 = ntile * BN + c;
+          if (col0 >= p.N || row0 >= p.M) break;
           uint32_t w[32];
           __syncwarp();
           if constexpr (EPI == EPI_F32) {
@@ -517,17 +534,23 @@ __global__ void __launch_bounds__(kThreads, 1)
               w[16 + i] = pack_bf16x2(v1[2 * i], v1[2 * i + 1]);
             }
           }
-          // the store that last used this buffer (kBufs chunks ago) has read it
-          if (lane == 0) bulk_wait_read<C::kBufs - 1>();
-          __syncwarp();
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            st_shared_v4(row_addr + ((j ^ (lane & 7)) << 4), w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-          fence_async_shared();
+            st_shared_v4(sbase + lane * 128 + ((j ^ (lane & 7)) << 4), w[4 * j], w[4 * j + 1], w[4 * j + 2],
+                         w[4 * j + 3]);
           __syncwarp();
-          if (lane == 0) {
-            tma_store_3d(&maps.out, buf, ntile * BN + c, row0, g);
-            bulk_commit();
+          const int col = col0 + piece * (16 / kEsz);
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int r = it * 4 + rsub;
+            uint32_t a0, a1, a2, a3;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
+                         : "r"(sbase + r * 128 + ((piece ^ (r & 7)) << 4)));
+            const int row = row0 + r;
+            if (row < p.M && col < p.N)
+              *reinterpret_cast<uint4*>(obase + (static_cast<long long>(row) * p.ldo + col) * kEsz) =
+                  make_uint4(a0, a1, a2, a3);
           }
         }
       } else if constexpr (EPI == EPI_F32 || EPI == EPI_BF16) {
@@ -571,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     pack_bf16x2(__uint_as_float(r[2 * cc + 1][2 * i]), __uint_as_float(r[2 * cc + 1][2 * i + 1]));
               }
             }
-            uint8_t* buf = staging + ((warp - 2) * C::kBufs + ring) * C::kBufBytes;
+            uint8_t* buf = staging + (ew * C::kBufs + ring) * C::kBufBytes;
             if (++ring == C::kBufs) ring = 0;
             const uint32_t row_addr = smem_u32(buf) + lane * 128;
             // the store that last used this buffer (kBufs chunks ago) has read it
@@ -769,7 +792,7 @@ moe_status_t launch_instance(const TmaMaps& maps, const KParams& kp, int grid, c
     if (e != cudaSuccess) return cuda_check(e, "cudaFuncSetAttribute(gemm)");
     attr_set = true;
   }
-  kern<<<grid, kThreads, smem, st>>>(maps, kp);
+  kern<<<grid, Roles<A_MN && B_MN>::kThreads, smem, st>>>(maps, kp);
   count_launch();
   return cuda_check(cudaGetLastError(), "gemm launch");
 }
