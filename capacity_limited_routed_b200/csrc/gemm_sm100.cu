@@ -739,6 +739,292 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
   }
 }
 
+
+// ====================================================================== weight gradients on CTA pairs
+//
+// dW = A^T B with both operands MN-major and a float32 result, on a pair of CTAs (one
+// cluster of two, cta_group::2): 256 x 256 output tiles, each CTA loading 128 rows of A
+// and 128 of B's 256 columns per k-block, the leader issuing M=256 tcgen05.mma that read
+// both CTAs' shared memory, each CTA draining its 128 accumulator rows.  Per output
+// element this reads a third fewer operand bytes than the single-CTA kernel, which is
+// what bounds these short (rows-per-expert) contractions.
+constexpr int kPairEpiWarps = 8;
+constexpr int kPairThreads = 64 + 32 * kPairEpiWarps;
+
+struct PairCfg {
+  static constexpr int kABytes = 128 * kBK * 2;
+  static constexpr int kBBytes = 128 * kBK * 2;
+  static constexpr int kStage = kABytes + kBBytes;  // 32 KB per CTA
+  static constexpr int kStages = 6;
+  static constexpr int kTmemCols = 512;             // two 256-column accumulators
+  static constexpr int kStaging = kPairEpiWarps * 4096;
+  static constexpr int kBarBytes = 8 * (2 * kStages + 5) + 16;
+  static constexpr int kSmem = 1024 + kStages * kStage + kStaging + kBarBytes;
+  static_assert(kSmem <= 232448, "shared memory budget");
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+    gemm_pair_wgrad_kernel(const __grid_constant__ TmaMaps maps, const KParams p) {
+  using C = PairCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* staging = smem + C::kStages * C::kStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + C::kStaging);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * 32 * kPairEpiWarps);  // both CTAs' epilogue threads
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&maps.a[0]);
+    tma_prefetch_desc(&maps.b[0]);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, C::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before either touches the other's
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const volatile int* abort_v = abort_flag;
+
+  const int mt_n = (p.M + 255) / 256;
+  const int nt_n = (p.N + 255) / 256;
+  const int per_group = mt_n * nt_n;
+  const int total = p.groups * per_group;
+  auto k_blocks = [&](int g) {
+    if (p.ragged == 2) {
+      const int r = p.group_rows[g];
+      return r > 0 ? (r + kBK - 1) / kBK : 0;
+    }
+    return p.seg_kb[0];
+  };
+  // n fastest: the pairs working at one time write whole rows of the result.  Every role
+  // fetches a tile one step ahead, so the load of a group's row count overlaps the tile
+  // before it instead of stalling the pipeline at each tile boundary.
+  struct PairTile {
+    int g, m, n, kb;
+  };
+  auto fetch = [&](int t) {
+    PairTile r{0, 0, 0, 0};
+    if (t < total) {
+      r.g = t / per_group;
+      const int l = t - r.g * per_group;
+      r.n = l % nt_n;
+      r.m = l / nt_n;
+      r.kb = k_blocks(r.g);
+    }
+    return r;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int armed_phase[C::kStages];
+      for (int s = 0; s < C::kStages; ++s) armed_phase[s] = -1;
+      bool ok = true;
+      PairTile nxt = fetch(pair);
+      for (int t = pair; ok && t < total; t += npairs) {
+        const PairTile cur = nxt;
+        nxt = fetch(t + npairs);
+        const int g = cur.g, mt = cur.m, ntile = cur.n, kb_total = cur.kb;
+        const int m0 = mt * 256 + 128 * static_cast<int>(rank);
+        const int n0 = ntile * 256 + 128 * static_cast<int>(rank);
+        for (int kb = 0; kb < kb_total; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_v)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kStage);
+          armed_phase[stage] = static_cast<int>(phase);
+          const uint32_t bar = leader_addr(smem_u32(&full[stage]));
+          uint8_t* sa = smem + stage * C::kStage;
+          uint8_t* sb = sa + C::kABytes;
+          const int k0 = kb * kBK;
+          tma_load_3d_pair(&maps.a[0], sa, bar, m0, k0, g);
+          tma_load_3d_pair(&maps.a[0], sa + 8192, bar, m0 + 64, k0, g);
+          tma_load_3d_pair(&maps.b[0], sb, bar, n0, k0, g);
+          tma_load_3d_pair(&maps.b[0], sb + 8192, bar, n0 + 64, k0, g);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_status(p.status, MOE_ERR_TIMEOUT);
+        // the leader's full barriers count both CTAs' bytes: let every armed load land
+        if (leader)
+          for (int s = 0; s < C::kStages; ++s)
+            if (armed_phase[s] >= 0)
+              mbar_wait(&full[s], static_cast<uint32_t>(armed_phase[s]), nullptr, 50000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = idesc_bf16_f32(256, 256, true, true);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      bool issued = false;
+      PairTile nxt = fetch(pair);
+      for (int t = pair; ok && t < total; t += npairs) {
+        const PairTile cur = nxt;
+        nxt = fetch(t + npairs);
+        const int g = cur.g, mt = cur.m, ntile = cur.n, kb_total = cur.kb;
+        if (kb_total == 0) continue;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_v)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
+        for (int kb = 0; kb < kb_total; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_v)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * C::kStage);
+          const uint32_t b_addr = a_addr + C::kABytes;
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t ad = smem_desc_sw128(a_addr + k * 2048, 8192, 1024);
+            const uint64_t bd = smem_desc_sw128(b_addr + k * 2048, 8192, 1024);
+            mma_bf16_ss_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          issued = true;
+          mma_commit_pair(&empty[stage]);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_status(p.status, MOE_ERR_TIMEOUT);
+        if (issued) {
+          mma_commit_pair(drain);
+          mbar_wait(drain, 0, nullptr, 50000000ull);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const int ew = warp - 2;
+    const int col_lo = (ew >> 2) * 128;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    uint8_t* buf = staging + ew * 4096;  // one 32 x 32 float32 chunk, rows swizzled as the TMA expects
+    const uint32_t row_addr = smem_u32(buf) + lane * 128;
+    uint32_t tempty_leader;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(tempty_leader) : "r"(smem_u32(&tempty[0])), "r"(0));
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    PairTile nxt = fetch(pair);
+    for (int t = pair; t < total; t += npairs) {
+      const PairTile cur = nxt;
+      nxt = fetch(t + npairs);
+      const int g = cur.g, mt = cur.m, ntile = cur.n, kb_total = cur.kb;
+      const int row0 = mt * 256 + 128 * static_cast<int>(rank) + q * 32;
+      float* obase = static_cast<float*>(p.out) + static_cast<long long>(g) * p.out_gs;
+      if (kb_total == 0) {
+        // an empty contraction: the product is zero
+        const int row = row0 + lane;
+        if (row < p.M)
+          for (int c = col_lo; c < col_lo + 128; c += 4) {
+            const int col = ntile * 256 + c;
+            if (col >= p.N) break;
+            *reinterpret_cast<float4*>(obase + static_cast<long long>(row) * p.ldo + col) =
+                make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        continue;
+      }
+      const bool got = mbar_wait(&tfull[acc], acc_phase, abort_v);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, got)) {
+        *abort_flag = 1;
+        record_status(p.status, MOE_ERR_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + lane_off + static_cast<uint32_t>(acc * 256);
+      // per 32-column chunk: TMEM -> registers -> staging -> one TMA store (the copy
+      // engine clips rows and columns past the output's edge)
+#pragma unroll 1
+      for (int c = col_lo; c < col_lo + 128; c += 32) {
+        const int col0 = ntile * 256 + c;
+        if (col0 >= p.N || row0 >= p.M) break;
+        float v[32];
+        if (lane == 0) bulk_wait_read<0>();  // the previous chunk's store has read the buffer
+        __syncwarp();
+        tmem_ld_32cols(tbase + c, v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          st_shared_v4(row_addr + ((j ^ (lane & 7)) << 4), __float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
+                       __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
+        fence_async_shared();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&maps.out, buf, col0, row0, g);
+          bulk_commit();
+        }
+      }
+      __syncwarp();
+      tc_fence_before();
+      // hand the accumulator back to the leader's MMA warp
+      mbar_arrive_cluster(tempty_leader + static_cast<uint32_t>(acc * 8));
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  if (warp >= 2 && lane == 0) bulk_wait_all();  // every store has landed before the CTA exits
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // neither CTA leaves while the other may still touch its memory
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::kTmemCols);
+  }
+}
+
 // ====================================================================== host side
 
 namespace {
@@ -901,6 +1187,32 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
   kp.add_ld = a.add_ld;
   kp.status = a.status;
 
+  if (a.a_mn && a.b_mn && a.epi == EPI_F32 && a.nseg == 1 && a.ragged != 1 && a.bn == 256) {
+    const long long pair_tiles =
+        static_cast<long long>(a.groups) * ((a.M + 255) / 256) * ((a.N + 255) / 256);
+    static int max_pairs = 0;  // pairs that fit on the device at once
+    if (max_pairs == 0) {
+      cudaError_t e = cudaFuncSetAttribute(gemm_pair_wgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           PairCfg::kSmem);
+      if (e != cudaSuccess) return cuda_check(e, "cudaFuncSetAttribute(pair gemm)");
+      cudaLaunchConfig_t cfg;
+      memset(&cfg, 0, sizeof(cfg));
+      cfg.gridDim = dim3(2 * (device_sm_count() / 2));
+      cfg.blockDim = dim3(kPairThreads);
+      cfg.dynamicSmemBytes = PairCfg::kSmem;
+      int nc = 0;
+      if (cudaOccupancyMaxActiveClusters(&nc, gemm_pair_wgrad_kernel, &cfg) != cudaSuccess || nc <= 0) {
+        (void)cudaGetLastError();
+        nc = device_sm_count() / 2;
+      }
+      max_pairs = std::min(nc, device_sm_count() / 2);
+    }
+    const int pairs = static_cast<int>(std::min<long long>(pair_tiles, max_pairs));
+    if (pairs <= 0) return MOE_OK;
+    gemm_pair_wgrad_kernel<<<2 * pairs, kPairThreads, PairCfg::kSmem, st>>>(maps, kp);
+    count_launch();
+    return cuda_check(cudaGetLastError(), "pair gemm launch");
+  }
   const int out_cols = a.epi == EPI_SWIGLU ? a.bn / 2 : a.bn;
   const long long tiles = static_cast<long long>(a.groups) * ((a.M + kBM - 1) / kBM) * ((a.N + out_cols - 1) / out_cols);
   const int grid = static_cast<int>(std::min<long long>(tiles, device_sm_count()));

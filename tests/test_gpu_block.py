@@ -115,3 +115,32 @@ def test_empty_batch_is_a_no_op():
     assert y.shape == (0, s.d_model) and dx.shape == (0, s.d_model)
     assert all(int(g.abs().max().item()) == 0 for g in blk.grads.values())
     assert blk.stats_dict()["kept"] == 0
+
+
+def test_backward_idle_experts_get_zero_gradients():
+    """A batch too small to reach every expert: the weight gradients of experts that
+    received no rows must come out exactly zero (the contraction over their rows is empty),
+    whatever the gradient buffers held before."""
+    s = RAGGED.with_(T=12, backward=True, seed=21)
+    inp = synth.make_inputs(s)
+    from capacity_limited_routed_b200.block import MoEBlock
+    blk = MoEBlock(s, training=True)
+    blk.load(inp)
+    x = bf16_dev(inp["x"])
+    blk.forward(x)
+    for t in blk.grads.values():
+        t.fill_(float("nan"))
+    blk.backward(x, bf16_dev(inp["dy"]))
+    torch.cuda.synchronize()
+    rows = blk.saved_views()["expert_rows"].cpu().numpy()
+    idle = rows == 0
+    assert idle.sum() >= s.n_experts // 2
+    y_o, ctx = O.forward(inp["x"], inp["weights"], inp["bias"], s, logit_offset=inp["logit_offset"])
+    _, grads_o, _ = O.backward(inp["dy"], inp["weights"], ctx)
+    _, affected = _routing_agreement(blk.saved_views(), ctx)
+    for name in ("w1", "w3", "w2"):
+        got = host64(blk.grads[name])
+        assert np.all(got[idle] == 0.0), name
+        assert np.isfinite(got).all(), name
+        busy = ~idle & np.array([e not in affected for e in range(s.n_experts)])
+        assert_close_rms(got[busy], grads_o[name][busy], tol=ROUTED_GRAD_TOL, what=f"d{name}")
