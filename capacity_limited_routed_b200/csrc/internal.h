@@ -106,7 +106,7 @@ size_t scan_scratch_ints(const Geo& g);
 moe_status_t launch_slot_scan(const Geo& g, const int32_t* idx, int32_t* slot, int32_t* stats, int32_t* scratch,
                               cudaStream_t st);
 moe_status_t launch_pack(const Geo& g, const uint16_t* z, const int32_t* idx, const int32_t* slot,
-                         const int32_t* stats, uint16_t* pools, cudaStream_t st);
+                         int32_t* stats, uint16_t* pools, cudaStream_t st);
 // scratch ints needed by the receiver's row map
 size_t unpack_scratch_ints(const Geo& g);
 moe_status_t launch_unpack(const Geo& g, const uint16_t* pools, uint16_t* xe, int32_t* rows, int32_t* row_map,

@@ -21,7 +21,10 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace moe {
 
@@ -352,6 +355,87 @@ __global__ void pack_kernel(const uint16_t* __restrict__ z, const int32_t* __res
     }
     __syncwarp();
   }
+}
+
+// Dispatch through the copy engine.  Each warp owns two row buffers in shared memory.
+// Lane 0 brings token t's latent row in with one bulk copy and sends it to each of the
+// token's kept pool rows with one bulk store per row, while the next token's row is
+// already loading into the other buffer; lane j writes the 16-byte header of
+// assignment j.  Whole-row bulk stores keep many full lines in flight per SM.
+constexpr int kPackWarps = 8;
+
+__global__ void __launch_bounds__(32 * kPackWarps)
+    pack_bulk_kernel(const uint16_t* __restrict__ z, const int32_t* __restrict__ idx,
+                     const int32_t* __restrict__ slot, int T, int k, int dl, int L, int P, int W, int Cs, int E,
+                     uint16_t* __restrict__ pools, int32_t* __restrict__ status) {
+  extern __shared__ __align__(128) uint8_t pack_smem[];
+  __shared__ uint64_t s_bar[kPackWarps][2];
+  __shared__ long long s_dst[kPackWarps][32];
+  const int lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
+  const uint32_t row_bytes = static_cast<uint32_t>(dl) * 2u;
+  uint8_t* buf[2] = {pack_smem + static_cast<size_t>(wib) * 2 * row_bytes,
+                     pack_smem + static_cast<size_t>(wib) * 2 * row_bytes + row_bytes};
+  if (lane == 0) {
+    mbar_init(&s_bar[wib][0], 1);
+    mbar_init(&s_bar[wib][1], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  const long long row_elems = dl + 8;
+  const int nw = gridDim.x * (blockDim.x >> 5);
+  const int t0 = blockIdx.x * (blockDim.x >> 5) + wib;
+  bool armed[2] = {false, false};
+  if (lane == 0 && t0 < T) {
+    mbar_arrive_expect_tx(&s_bar[wib][0], row_bytes);
+    bulk_load_g2s(buf[0], z + static_cast<long long>(t0) * dl, row_bytes, &s_bar[wib][0]);
+    armed[0] = true;
+  }
+  int i = 0;
+  for (int t = t0; t < T; t += nw, ++i) {
+    const int b = i & 1;
+    int e_j = -1, s_j = -1;
+    bool ok_j = false;
+    if (lane < k) {
+      e_j = idx[static_cast<long long>(t) * k + lane];
+      s_j = slot[2LL * (static_cast<long long>(t) * k + lane)];
+      ok_j = s_j >= 0 && s_j < Cs && e_j >= 0 && e_j < E;
+      s_dst[wib][lane] = ok_j ? (static_cast<long long>(pool_of(e_j, L, P, W)) * Cs + s_j) * row_elems : -1;
+    }
+    __syncwarp();
+    bool got = true;
+    if (lane == 0) {
+      const int tn = t + nw;
+      if (tn < T) {
+        bulk_wait_read<0>();  // the previous token's stores have read the other buffer
+        mbar_arrive_expect_tx(&s_bar[wib][b ^ 1], row_bytes);
+        bulk_load_g2s(buf[b ^ 1], z + static_cast<long long>(tn) * dl, row_bytes, &s_bar[wib][b ^ 1]);
+        armed[b ^ 1] = true;
+      }
+      got = mbar_wait(&s_bar[wib][b], static_cast<uint32_t>((i >> 1) & 1), nullptr);
+      armed[b] = false;
+      if (got) {
+        fence_proxy_async_shared();
+        for (int j = 0; j < k; ++j) {
+          const long long d = s_dst[wib][j];
+          if (d >= 0) bulk_store_s2g(pools + d, buf[b], row_bytes);
+        }
+        bulk_commit();
+      }
+    }
+    got = __shfl_sync(0xffffffffu, got, 0);
+    if (!got) {
+      if (lane == 0) {
+        record_status_i32(status, MOE_ERR_TIMEOUT);
+        // let a row load still in flight land before the warp leaves
+        if (armed[b ^ 1]) mbar_wait(&s_bar[wib][b ^ 1], static_cast<uint32_t>(((i + 1) >> 1) & 1), nullptr);
+      }
+      break;
+    }
+    if (ok_j) *reinterpret_cast<int4*>(pools + s_dst[wib][lane] + dl) = make_int4(e_j, 0, 0, 0);
+    __syncwarp();
+  }
+  if (lane == 0) bulk_wait_all();
 }
 
 // header -1 for the rows of each pool past its fill
@@ -728,11 +812,29 @@ moe_status_t launch_slot_scan(const Geo& g, const int32_t* idx, int32_t* slot, i
 }
 
 moe_status_t launch_pack(const Geo& g, const uint16_t* z, const int32_t* idx, const int32_t* slot,
-                         const int32_t* stats, uint16_t* pools, cudaStream_t st) {
+                         int32_t* stats, uint16_t* pools, cudaStream_t st) {
   if (g.T > 0) {
-    const int warps = 8;
-    pack_kernel<<<blocks_for(g.T, warps), 32 * warps, 0, st>>>(z, idx, slot, g.T, g.k, g.dl, g.L, g.P, g.W, g.Cs,
-                                                               g.E, pools);
+    // two row buffers per warp; rows too wide for that take the register path
+    const size_t smem = static_cast<size_t>(kPackWarps) * 2 * g.dl * 2;
+    if (g.k <= 32 && smem <= 200 * 1024) {
+      static bool attr_set = false;
+      if (!attr_set) {
+        const moe_status_t r = cuda_check(
+            cudaFuncSetAttribute(pack_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024),
+            "cudaFuncSetAttribute(pack)");
+        if (r != MOE_OK) return r;
+        attr_set = true;
+      }
+      const int per_sm = smem <= 100 * 1024 ? 2 : 1;
+      const int grid = static_cast<int>(std::min<long long>((g.T + kPackWarps - 1) / kPackWarps,
+                                                            static_cast<long long>(device_sm_count()) * per_sm));
+      pack_bulk_kernel<<<grid, 32 * kPackWarps, smem, st>>>(z, idx, slot, g.T, g.k, g.dl, g.L, g.P, g.W, g.Cs, g.E,
+                                                            pools, stats + 3);
+    } else {
+      const int warps = 8;
+      pack_kernel<<<blocks_for(g.T, warps), 32 * warps, 0, st>>>(z, idx, slot, g.T, g.k, g.dl, g.L, g.P, g.W, g.Cs,
+                                                                 g.E, pools);
+    }
     count_launch();
   }
   const long long rows = static_cast<long long>(g.NP) * g.Cs;

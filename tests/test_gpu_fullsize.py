@@ -51,7 +51,8 @@ def test_route_and_dispatch_bit_exact_full_size(M, shape):
     np.testing.assert_allclose(gate.cpu().numpy(), gate_o, rtol=2e-6, atol=1e-7)
     slots = O.assign_slots(idx_o, g)
     info = plan.info
-    z = torch.zeros((s.T, s.d_latent), dtype=torch.bfloat16, device=dev())
+    gen = torch.Generator(device=dev()).manual_seed(11)
+    z = torch.randn((s.T, s.d_latent), generator=gen, device=dev()).to(torch.bfloat16)
     pools = torch.empty(info.pools_bytes // 2, dtype=torch.int16, device=dev())
     slot = torch.empty((s.T, s.top_k, 2), dtype=torch.int32, device=dev())
     stats = torch.zeros(info.stats_bytes // 4, dtype=torch.int32, device=dev())
@@ -64,6 +65,18 @@ def test_route_and_dispatch_bit_exact_full_size(M, shape):
     E = s.n_experts
     assert np.array_equal(st[8 + E:8 + 4 * E], np.concatenate(
         [slots["expert_kept"], slots["expert_dropped_sender"], slots["expert_dropped_receiver"]]))
+    # pool rows of sampled kept assignments hold the token's latent row bit for bit, and
+    # their headers the packed expert id
+    pl = O.placement(g)
+    rows = pools[: g.n_pools * g.C_s * (s.d_latent + 8)].view(g.n_pools, g.C_s, s.d_latent + 8)
+    t_all, j_all = np.nonzero(slots["sslot"] >= 0)
+    pick = np.random.default_rng(6).choice(t_all.size, size=min(512, t_all.size), replace=False)
+    t_s, j_s = t_all[pick], j_all[pick]
+    e_s = idx_o[t_s, j_s]
+    got = rows[torch.from_numpy(pl["pool"][e_s]).to(dev()), torch.from_numpy(slots["sslot"][t_s, j_s]).to(dev())]
+    assert torch.equal(got[:, : s.d_latent], z.view(torch.int16)[torch.from_numpy(t_s).to(dev())])
+    hdr = got[:, s.d_latent:].cpu().numpy().copy().view(np.int32)[:, 0]
+    assert np.array_equal(hdr, e_s)
     print(f"\n[{s.name}] drops: sender {slots['dropped_sender']}, receiver {slots['dropped_receiver']} "
           f"of {s.T * s.top_k}")
 
