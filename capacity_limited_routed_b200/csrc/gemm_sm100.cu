@@ -763,6 +763,44 @@ struct PairCfg {
   static_assert(kSmem <= 232448, "shared memory budget");
 };
 
+// An epilogue warp's share of a pair tile: 32 rows (row0..) x 128 columns (col_lo..) of
+// this CTA's accumulator half, per 32-column chunk TMEM -> registers -> staging -> one
+// TMA store (the copy engine clips rows and columns past the output's edge).
+__device__ __forceinline__ void pair_drain(const TmaMaps& maps, const KParams& p, uint32_t tbase, int col_lo,
+                                           int ntile, int row0, int g, uint8_t* buf, uint32_t row_addr, int lane) {
+#pragma unroll 1
+  for (int c = col_lo; c < col_lo + 128; c += 32) {
+    const int col0 = ntile * 256 + c;
+    if (col0 >= p.N || row0 >= p.M) break;
+    float v[32];
+    if (lane == 0) bulk_wait_read<0>();  // the previous chunk's store has read the buffer
+    __syncwarp();
+    tmem_ld_32cols(tbase + c, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      st_shared_v4(row_addr + ((j ^ (lane & 7)) << 4), __float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
+                   __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
+    fence_async_shared();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_3d(&maps.out, buf, col0, row0, g);
+      bulk_commit();
+    }
+  }
+}
+
+// the same share of a tile whose contraction is empty: zeros
+__device__ __forceinline__ void pair_zero(const KParams& p, int col_lo, int ntile, int row0, int g, int lane) {
+  float* obase = static_cast<float*>(p.out) + static_cast<long long>(g) * p.out_gs;
+  const int row = row0 + lane;
+  if (row < p.M)
+    for (int c = col_lo; c < col_lo + 128; c += 4) {
+      const int col = ntile * 256 + c;
+      if (col >= p.N) break;
+      *reinterpret_cast<float4*>(obase + static_cast<long long>(row) * p.ldo + col) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     gemm_pair_wgrad_kernel(const __grid_constant__ TmaMaps maps, const KParams p) {
   using C = PairCfg;
@@ -962,17 +1000,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       nxt = fetch(t + npairs);
       const int g = cur.g, mt = cur.m, ntile = cur.n, kb_total = cur.kb;
       const int row0 = mt * 256 + 128 * static_cast<int>(rank) + q * 32;
-      float* obase = static_cast<float*>(p.out) + static_cast<long long>(g) * p.out_gs;
       if (kb_total == 0) {
-        // an empty contraction: the product is zero
-        const int row = row0 + lane;
-        if (row < p.M)
-          for (int c = col_lo; c < col_lo + 128; c += 4) {
-            const int col = ntile * 256 + c;
-            if (col >= p.N) break;
-            *reinterpret_cast<float4*>(obase + static_cast<long long>(row) * p.ldo + col) =
-                make_float4(0.f, 0.f, 0.f, 0.f);
-          }
+        pair_zero(p, col_lo, ntile, row0, g, lane);
         continue;
       }
       const bool got = mbar_wait(&tfull[acc], acc_phase, abort_v);
@@ -983,28 +1012,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t tbase = tmem_base + lane_off + static_cast<uint32_t>(acc * 256);
-      // per 32-column chunk: TMEM -> registers -> staging -> one TMA store (the copy
-      // engine clips rows and columns past the output's edge)
-#pragma unroll 1
-      for (int c = col_lo; c < col_lo + 128; c += 32) {
-        const int col0 = ntile * 256 + c;
-        if (col0 >= p.N || row0 >= p.M) break;
-        float v[32];
-        if (lane == 0) bulk_wait_read<0>();  // the previous chunk's store has read the buffer
-        __syncwarp();
-        tmem_ld_32cols(tbase + c, v);
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          st_shared_v4(row_addr + ((j ^ (lane & 7)) << 4), __float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
-                       __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
-        fence_async_shared();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_3d(&maps.out, buf, col0, row0, g);
-          bulk_commit();
-        }
-      }
+      pair_drain(maps, p, tmem_base + lane_off + static_cast<uint32_t>(acc * 256), col_lo, ntile, row0, g, buf,
+                 row_addr, lane);
       __syncwarp();
       tc_fence_before();
       // hand the accumulator back to the leader's MMA warp
@@ -1024,6 +1033,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     tmem_dealloc_pair(tmem_base, C::kTmemCols);
   }
 }
+
 
 // ====================================================================== host side
 

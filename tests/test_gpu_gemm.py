@@ -85,3 +85,20 @@ def test_gemm_partial_tiles_many(M, a_mn, b_mn, n):
         torch.cuda.synchronize()
         err = (D.double().cpu() - ref).abs().max().item()
         assert err <= 1e-4 * rms(ref.numpy()), err
+
+
+@pytest.mark.parametrize("k", [64, 130, 384, 448, 449])
+def test_gemm_weight_gradient_short_contractions(M, k):
+    """Both operands MN-major with a float32 result (the weight-gradient form) at the
+    contraction lengths of an expert's rows (a few 64-deep blocks, ragged tails), over
+    several 256-row slabs and n-tiles with ragged edges, twice in a row."""
+    m, n = 776, 520
+    a, b = _operands(m, n, k, seed=k)
+    ref = a.double() @ b.double().T
+    A, B = a.T.contiguous().to(dev()), b.T.contiguous().to(dev())
+    for _ in range(2):
+        D = torch.full((m, n), float("nan"), dtype=torch.float32, device=dev())
+        M.moe_gemm_bf16(m, n, k, A, 1, B, 1, D)
+        torch.cuda.synchronize()
+        err = (D.double().cpu() - ref).abs().max().item()
+        assert err <= 1e-4 * rms(ref.numpy()) * max(1.0, np.sqrt(k / 64)), err
