@@ -32,6 +32,38 @@ METRIC = "MoE-block tokens/s fwd & fwd+bwd on 1 B200; GEMM % BF16 peak; dispatch
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "_source": "fallback"}
 
 
+# DRAM bytes (read + write) of the dominant step, from one ncu capture (--set full,
+# --clock-control none) of its kernels on the small profiling workload (24 experts,
+# T = 1024, same widths and rows per expert), summed over the step's launches.  The
+# step's traffic scales with the expert count, so a workload with the same shape per
+# expert reports it scaled; it is reported only while the kernel sources hash to the
+# captured ones, and as null once they change.
+NCU_TRAFFIC = {
+    "bwd.experts_wgrad_gate_up": {
+        "sources_sha256": "fbeb515446d98d0705db7d00ad0608e38d53ad0713f1ced9e4b2b4feedc7e953",
+        "dram_bytes": 1918019584, "experts": 24, "tokens": 1024, "d_latent": 3072, "hidden_routed": 3072,
+    },
+}
+KERNEL_SOURCES = ("gemm_sm100.cu", "ptx.cuh", "internal.h")
+
+
+def measured_traffic(name, s):
+    rec = NCU_TRAFFIC.get(name)
+    if rec is None:
+        return None
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "capacity_limited_routed_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != rec["sources_sha256"]:
+        return None
+    if (s.d_latent, s.hidden_routed) != (rec["d_latent"], rec["hidden_routed"]) or \
+            s.T * rec["experts"] != rec["tokens"] * s.n_experts:
+        return None
+    return int(rec["dram_bytes"] * s.n_experts / rec["experts"])
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -345,12 +377,12 @@ def main():
     kt = kernels[top]
     if kt.get("bound") == "tensor":
         roof = {"kernel": top, "bound": "tensor", "achieved": kt["tflops"], "peak": tc_peak,
-                "unit": "TFLOP/s", "frac": round(kt["tflops"] / tc_peak, 3), "traffic": None,
+                "unit": "TFLOP/s", "frac": round(kt["tflops"] / tc_peak, 3), "traffic": measured_traffic(top, s),
                 "peak_kind": f"bf16_tflops_sustained ({peaks['_source']}): kernel timed inside a long step",
                 "flops_per_launch": flops[top]}
     else:
         roof = {"kernel": top, "bound": "hbm", "achieved": kt.get("gbs"), "peak": hbm,
-                "unit": "GB/s", "frac": round((kt.get("gbs") or 0) / hbm, 3), "traffic": None,
+                "unit": "GB/s", "frac": round((kt.get("gbs") or 0) / hbm, 3), "traffic": measured_traffic(top, s),
                 "peak_kind": f"hbm_gbs ({peaks['_source']})", "bytes_per_launch": bytes_.get(top)}
     fwd_ms = sum(v[0] for k_, v in per.items() if k_.startswith("fwd.") or k_.startswith("experts.")) / args.steps
     step_ms = ms_max / args.steps
