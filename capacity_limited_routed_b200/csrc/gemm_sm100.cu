@@ -96,11 +96,12 @@ struct Cfg {
   static constexpr int kTmemCols = 2 * BN;
   static constexpr int kBufs = WRITE_BOUND ? MOE_WB_BUFS : 1;  // staging buffers per epilogue warp
   static constexpr int kEpiWarps = Roles<WRITE_BOUND>::kEpiWarps;
-  // a buffer holds 32 rows x 128 bytes (float32 / bf16 outputs, or two 32 x 64-byte
-  // bf16 tiles); the forward SwiGLU stages three 32 x 64-byte tiles (H, a, b)
+  // a buffer holds 32 rows x 128 bytes (float32 / bf16 outputs); the forward SwiGLU
+  // stages three 32 x 64-byte tiles (H, a, b), its backward three slots of two 32 x
+  // 32-byte tiles (a and b in, dA and dB out in place)
   static constexpr int kBufBytes = SWIGLU ? 6144 : 4096;
   static constexpr int kStaging = kEpiWarps * kBufs * kBufBytes;
-  static constexpr int kBarBytes = 8 * (2 * kStages + 5 + 4) + 16;
+  static constexpr int kBarBytes = 8 * (2 * kStages + 5 + 12) + 16;
   static constexpr int kPrefixInts = WRITE_BOUND ? 0 : kMaxGroups + 1;
   static constexpr int kSmem = 1024 + kStages * kStage + kStaging + kBarBytes + 4 * kPrefixInts;
   static_assert(kSmem <= 232448, "shared memory budget");
@@ -181,7 +182,7 @@ struct Sched {
 template <int BN, bool A_MN, bool B_MN, int EPI>
 __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
     gemm_kernel(const __grid_constant__ TmaMaps maps, const KParams p) {
-  using C = Cfg<BN, A_MN && B_MN, EPI == EPI_SWIGLU>;
+  using C = Cfg<BN, A_MN && B_MN, EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BWD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + C::kStages * C::kStage;
@@ -190,8 +191,8 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint64_t* ebar = drain + 1;  // one per epilogue warp: its own TMA loads (SwiGLU backward)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ebar + 4);
+  uint64_t* ebar = drain + 1;  // three per epilogue warp: its own TMA loads (SwiGLU backward)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ebar + 12);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* prefix = reinterpret_cast<int*>(staging + C::kStaging + C::kBarBytes);
 
@@ -208,7 +209,7 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
       mbar_init(&tempty[a], 32 * C::kEpiWarps);
     }
     mbar_init(drain, 1);
-    for (int w = 0; w < 4; ++w) mbar_init(&ebar[w], 1);
+    for (int w = 0; w < 12; ++w) mbar_init(&ebar[w], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -402,7 +403,8 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     int ring = 0;        // next staging buffer of this warp
-    uint32_t eph = 0;    // phase of this warp's load barrier
+    uint32_t eph = 0;    // SwiGLU backward: parity of each of this warp's three load barriers
+    int eslot = 0;       // SwiGLU backward: slot of the next live chunk
     Tile nxt = sc.tile(blockIdx.x);
     for (int t = blockIdx.x; t < sc.total; t += gridDim.x) {
       const Tile cur = nxt;
@@ -428,11 +430,36 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
         }
         continue;
       }
+      // SwiGLU backward: a and b come in by TMA one 16-column chunk ahead of their use,
+      // into a ring of three slots per warp; the first chunk's load starts before the
+      // accumulator is ready
+      const int srow0 = mt * kBM + q * 32;
+      int s_live = 0;  // live 16-column chunks of this warp in this tile
+      if constexpr (EPI == EPI_SWIGLU_BWD) {
+        if (srow0 < p.M) {
+          const int left = p.N - ntile * BN;
+          s_live = left >= BN ? BN / 16 : (left + 15) / 16;
+        }
+      }
+      auto swb_issue = [&](int ch, int slot) {  // lane 0
+        uint8_t* sb = staging + (warp - 2) * C::kBufBytes + slot * 2048;
+        uint64_t* bar = &ebar[3 * (warp - 2) + slot];
+        bulk_wait_read<1>();  // the stores of the slot's previous chunk have read it
+        mbar_arrive_expect_tx(bar, 2048);
+        tma_load_3d(&maps.aux_a, sb, bar, ntile * BN + ch * 16, srow0, g);
+        tma_load_3d(&maps.aux_b, sb + 1024, bar, ntile * BN + ch * 16, srow0, g);
+      };
+      if constexpr (EPI == EPI_SWIGLU_BWD) {
+        if (lane == 0 && s_live > 0) swb_issue(0, eslot);
+      }
       const bool got = mbar_wait(&tfull[acc], acc_phase, abort_v);
       __syncwarp();
       if (!__all_sync(0xffffffffu, got)) {
         *abort_flag = 1;
         record_status(p.status, MOE_ERR_TIMEOUT);
+        if constexpr (EPI == EPI_SWIGLU_BWD) {
+          if (lane == 0 && s_live > 0) mbar_wait(&ebar[3 * (warp - 2) + eslot], (eph >> eslot) & 1u, nullptr, 50000000ull);
+        }
         break;
       }
       tc_fence_after();
@@ -471,7 +498,7 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
           for (int e2 = 0; e2 < 16; ++e2) {
             const float a0 = __uint_as_float(rg[i][2 * e2]), a1 = __uint_as_float(rg[i][2 * e2 + 1]);
             const float u0 = __uint_as_float(ru[i][2 * e2]), u1 = __uint_as_float(ru[i][2 * e2 + 1]);
-            const float s0 = a0 / (1.0f + expf(-a0)), s1 = a1 / (1.0f + expf(-a1));
+            const float s0 = __fdividef(a0, 1.0f + __expf(-a0)), s1 = __fdividef(a1, 1.0f + __expf(-a1));
             h[e2] = pack_bf16x2(s0 * u0, s1 * u1);
             ga[e2] = pack_bf16x2(a0, a1);
             gb[e2] = pack_bf16x2(u0, u1);
@@ -612,45 +639,35 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
           }
         }
       } else if constexpr (EPI == EPI_SWIGLU_BWD) {
-        // per chunk of 32 columns: TMA-load a and b (32 x 64-byte tiles, 64-byte swizzle)
-        // while the accumulator chunk comes out of TMEM, form dA and dB in place, and
-        // TMA-store them
-        const int row0 = mt * kBM + q * 32;
+        // per chunk of 16 columns: dH from TMEM, a and b from the slot loaded one chunk
+        // ago (32 x 32-byte tiles, unswizzled), dA and dB formed in place and TMA-stored
         const int wi = warp - 2;
-        uint8_t* buf = staging + wi * C::kBufBytes;
-        const uint32_t rbase = smem_u32(buf) + lane * 64;
-        const int sw = (lane >> 1) & 3;
         bool ok = true;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          const int col0 = ntile * BN + c;
-          const bool live = col0 < p.N && row0 < p.M;
-          if (lane == 0) {
-            bulk_wait_read<0>();  // the previous chunk's stores have read the buffer
-            if (live) {
-              mbar_arrive_expect_tx(&ebar[wi], 4096);
-              tma_load_3d(&maps.aux_a, buf, &ebar[wi], col0, row0, g);
-              tma_load_3d(&maps.aux_b, buf + 2048, &ebar[wi], col0, row0, g);
-            }
-          }
-          float v[32];
+        for (int ch = 0; ch < s_live; ++ch) {  // the live chunks are a prefix (warp-uniform)
+          uint32_t r[16];
           __syncwarp();
-          tmem_ld_32cols(tbase + c, v);
-          if (!live) continue;
-          const bool got = mbar_wait(&ebar[wi], eph, abort_v);
-          eph ^= 1u;
-          if (!__all_sync(0xffffffffu, got)) {
+          tmem_ld_16cols(tbase + ch * 16, r);
+          const int slot = eslot;
+          eslot = eslot == 2 ? 0 : eslot + 1;
+          if (lane == 0 && ch + 1 < s_live) swb_issue(ch + 1, eslot);
+          const bool gotc = mbar_wait(&ebar[3 * wi + slot], (eph >> slot) & 1u, abort_v);
+          eph ^= 1u << slot;
+          if (!__all_sync(0xffffffffu, gotc)) {
+            // let the next chunk's load land before leaving
+            if (lane == 0 && ch + 1 < s_live) mbar_wait(&ebar[3 * wi + eslot], (eph >> eslot) & 1u, nullptr, 50000000ull);
             ok = false;
             break;
           }
+          uint8_t* sb = staging + wi * C::kBufBytes + slot * 2048;
+          const uint32_t ra = smem_u32(sb) + lane * 32;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t off = ((j ^ sw) << 4);
+          for (int j = 0; j < 2; ++j) {
             uint32_t aw[4], bw[4], da[4], db[4];
             asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(aw[0]), "=r"(aw[1]), "=r"(aw[2]), "=r"(aw[3]) : "r"(rbase + off));
+                         : "=r"(aw[0]), "=r"(aw[1]), "=r"(aw[2]), "=r"(aw[3]) : "r"(ra + 16 * j));
             asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(bw[0]), "=r"(bw[1]), "=r"(bw[2]), "=r"(bw[3]) : "r"(rbase + 2048 + off));
+                         : "=r"(bw[0]), "=r"(bw[1]), "=r"(bw[2]), "=r"(bw[3]) : "r"(ra + 1024 + 16 * j));
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
               float rda[2], rdb[2];
@@ -658,22 +675,22 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
               for (int hh = 0; hh < 2; ++hh) {
                 const float a = hh ? bf16_hi(aw[w]) : bf16_lo(aw[w]);
                 const float b = hh ? bf16_hi(bw[w]) : bf16_lo(bw[w]);
-                const float dh = v[8 * j + 2 * w + hh];
-                const float sg = 1.0f / (1.0f + expf(-a));
+                const float dh = __uint_as_float(r[8 * j + 2 * w + hh]);
+                const float sg = __fdividef(1.0f, 1.0f + __expf(-a));
                 rda[hh] = dh * b * (sg * (1.0f + a * (1.0f - sg)));
                 rdb[hh] = dh * (a * sg);
               }
               da[w] = pack_bf16x2(rda[0], rda[1]);
               db[w] = pack_bf16x2(rdb[0], rdb[1]);
             }
-            st_shared_v4(rbase + off, da[0], da[1], da[2], da[3]);
-            st_shared_v4(rbase + 2048 + off, db[0], db[1], db[2], db[3]);
+            st_shared_v4(ra + 16 * j, da[0], da[1], da[2], da[3]);
+            st_shared_v4(ra + 1024 + 16 * j, db[0], db[1], db[2], db[3]);
           }
           fence_async_shared();
           __syncwarp();
           if (lane == 0) {
-            tma_store_3d(&maps.out, buf, col0, row0, g);
-            tma_store_3d(&maps.out2, buf + 2048, col0, row0, g);
+            tma_store_3d(&maps.out, sb, ntile * BN + ch * 16, srow0, g);
+            tma_store_3d(&maps.out2, sb + 1024, ntile * BN + ch * 16, srow0, g);
             bulk_commit();
           }
         }
@@ -1081,7 +1098,7 @@ moe_status_t make_map(CUtensorMap* m, const Mat& t, uint32_t box_inner, uint32_t
 template <int BN, bool A_MN, bool B_MN, int EPI>
 moe_status_t launch_instance(const TmaMaps& maps, const KParams& kp, int grid, cudaStream_t st) {
   auto kern = gemm_kernel<BN, A_MN, B_MN, EPI>;
-  const int smem = Cfg<BN, A_MN && B_MN, EPI == EPI_SWIGLU>::kSmem;
+  const int smem = Cfg<BN, A_MN && B_MN, EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BWD>::kSmem;
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -1163,9 +1180,21 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
       if ((r = tile(&maps.aux_b, a.save_b, a.ldo, a.out_gs, "saved value")) != MOE_OK) return r;
     }
     if (a.epi == EPI_SWIGLU_BWD) {
-      if ((r = tile(&maps.out2, a.out2, a.ldo, a.out_gs, "dB")) != MOE_OK) return r;
-      if ((r = tile(&maps.aux_a, a.aux_a, a.aux_ld, a.aux_gs, "a")) != MOE_OK) return r;
-      if ((r = tile(&maps.aux_b, a.aux_b, a.aux_ld, a.aux_gs, "b")) != MOE_OK) return r;
+      // 32 rows x 16 columns (32-byte rows, unswizzled) for the chunked backward epilogue
+      auto tile16 = [&](CUtensorMap* m, const void* ptr, int64_t ld, int64_t gs, const char* what) {
+        Mat o;
+        o.ptr = ptr;
+        o.inner = a.N;
+        o.rows = a.M;
+        o.groups = a.groups;
+        o.ld = ld;
+        o.gs = a.groups > 1 ? gs : ld * a.M;
+        return make_map(m, o, 16, 32, what, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, CU_TENSOR_MAP_SWIZZLE_NONE);
+      };
+      if ((r = tile16(&maps.out, a.out, a.ldo, a.out_gs, "dA")) != MOE_OK) return r;
+      if ((r = tile16(&maps.out2, a.out2, a.ldo, a.out_gs, "dB")) != MOE_OK) return r;
+      if ((r = tile16(&maps.aux_a, a.aux_a, a.aux_ld, a.aux_gs, "a")) != MOE_OK) return r;
+      if ((r = tile16(&maps.aux_b, a.aux_b, a.aux_ld, a.aux_gs, "b")) != MOE_OK) return r;
     }
   }
   if (a.epi == EPI_F32 || a.epi == EPI_BF16) {
