@@ -568,7 +568,14 @@ __device__ __forceinline__ uint4 pack8(const float (&a)[8]) {
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-__global__ void combine_kernel(const uint16_t* __restrict__ ye, const float* __restrict__ gate,
+// r_t = sum_j g_tj Y[row_tj] over the kept assignments, fp32 in j order.  Per pass a lane
+// covers kCombVpl 16-byte vectors of the row and loads them from eight expert rows at
+// once (rows past k or dropped read as zero), so a warp keeps 8 x kCombVpl x 512 bytes
+// of loads in flight instead of walking the rows one after another.
+constexpr int kCombVpl = 2;
+constexpr int kCombRows = 8;
+
+__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ ye, const float* __restrict__ gate,
                                const int32_t* __restrict__ idx, const int32_t* __restrict__ slot, int T, int k,
                                int dl, int Cr, int E, uint16_t* __restrict__ r) {
   __shared__ long long s_row[8][32];
@@ -587,69 +594,130 @@ __global__ void combine_kernel(const uint16_t* __restrict__ ye, const float* __r
       s_g[wib][lane] = ok ? gate[a] : 0.0f;
     }
     __syncwarp();
-    for (int v = lane; v < nvec; v += 64) {
-      const bool two = v + 32 < nvec;
-      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0}, acc2[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-#pragma unroll 4
-      for (int j = 0; j < k; ++j) {
-        const long long rj = s_row[wib][j];
-        if (rj < 0) continue;
-        const uint4* yrow = reinterpret_cast<const uint4*>(ye + rj * dl);
-        const uint4 a = yrow[v];
-        const uint4 b = two ? yrow[v + 32] : make_uint4(0, 0, 0, 0);
-        acc8(acc, a, s_g[wib][j]);
-        acc8(acc2, b, s_g[wib][j]);
+    for (int v0 = lane; v0 < nvec; v0 += 32 * kCombVpl) {
+      float acc[kCombVpl][8];
+#pragma unroll
+      for (int u = 0; u < kCombVpl; ++u)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[u][i] = 0.0f;
+      for (int j0 = 0; j0 < k; j0 += kCombRows) {
+        uint4 val[kCombRows][kCombVpl];
+#pragma unroll
+        for (int jj = 0; jj < kCombRows; ++jj) {
+          const int j = j0 + jj;
+          const long long rj = j < k ? s_row[wib][j] : -1;
+          const uint4* yrow = reinterpret_cast<const uint4*>(ye + (rj >= 0 ? rj : 0) * dl);
+#pragma unroll
+          for (int u = 0; u < kCombVpl; ++u) {
+            const int v = v0 + 32 * u;
+            val[jj][u] = (rj >= 0 && v < nvec) ? yrow[v] : make_uint4(0, 0, 0, 0);
+          }
+        }
+#pragma unroll
+        for (int jj = 0; jj < kCombRows; ++jj) {
+          const int j = j0 + jj;
+          if (j >= k) break;
+          const float g = s_g[wib][j];
+#pragma unroll
+          for (int u = 0; u < kCombVpl; ++u) acc8(acc[u], val[jj][u], g);
+        }
       }
       uint4* out = reinterpret_cast<uint4*>(r + static_cast<long long>(t) * dl);
-      out[v] = pack8(acc);
-      if (two) out[v + 32] = pack8(acc2);
+#pragma unroll
+      for (int u = 0; u < kCombVpl; ++u)
+        if (v0 + 32 * u < nvec) out[v0 + 32 * u] = pack8(acc[u]);
     }
     __syncwarp();
   }
 }
 
-__global__ void combine_bwd_kernel(const uint16_t* __restrict__ dr, const uint16_t* __restrict__ ye,
+// dY[row_tj] = g_tj dr_t on kept rows, dg_tj = <dr_t, Y[row_tj]>.  Per pass a lane holds
+// kCombVpl vectors of dr_t and loads the matching vectors of eight expert rows at once;
+// the eight partial dot products stay in registers until the row is done.
+__global__ void __launch_bounds__(256) combine_bwd_kernel(const uint16_t* __restrict__ dr, const uint16_t* __restrict__ ye,
                                    const float* __restrict__ gate, const int32_t* __restrict__ idx,
                                    const int32_t* __restrict__ slot, int T, int k, int dl, int Cr, int E,
                                    uint16_t* __restrict__ dye, float* __restrict__ dg) {
+  __shared__ long long s_row[8][32];
+  __shared__ float s_g[8][32];
   const int lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
   const int warps = blockDim.x >> 5;
   const int nvec = dl / 8;
-  for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += gridDim.x * warps) {
-    const uint4* drow = reinterpret_cast<const uint4*>(dr + static_cast<long long>(t) * dl);
-    for (int j = 0; j < k; ++j) {
-      const long long a = static_cast<long long>(t) * k + j;
-      const int rs_raw = slot[2 * a + 1];
+  for (int t = blockIdx.x * warps + wib; t < T; t += gridDim.x * warps) {
+    if (lane < k) {
+      const long long a = static_cast<long long>(t) * k + lane;
+      const int rs = slot[2 * a + 1];
       const int e = idx[a];
-      const int rs = (rs_raw < Cr && e >= 0 && e < E) ? rs_raw : -1;
-      float dot = 0.0f;
-      if (rs >= 0) {
-        const float g = gate[a];
-        const long long rowo = (static_cast<long long>(e) * Cr + rs) * dl;
-        const uint4* yrow = reinterpret_cast<const uint4*>(ye + rowo);
-        uint4* out = reinterpret_cast<uint4*>(dye + rowo);
-        for (int v = lane; v < nvec; v += 32) {
-          const uint4 d = drow[v];
-          const uint4 y = yrow[v];
-          const uint32_t dw[4] = {d.x, d.y, d.z, d.w};
-          const uint32_t yw[4] = {y.x, y.y, y.z, y.w};
-          float o[8];
+      const bool ok = rs >= 0 && rs < Cr && e >= 0 && e < E;
+      s_row[wib][lane] = ok ? static_cast<long long>(e) * Cr + rs : -1;
+      s_g[wib][lane] = ok ? gate[a] : 0.0f;
+    }
+    __syncwarp();
+    const uint4* drow = reinterpret_cast<const uint4*>(dr + static_cast<long long>(t) * dl);
+    for (int j0 = 0; j0 < k; j0 += kCombRows) {
+      float dot[kCombRows];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float d0 = __uint_as_float(dw[i] << 16), d1 = __uint_as_float(dw[i] & 0xFFFF0000u);
-            const float y0 = __uint_as_float(yw[i] << 16), y1 = __uint_as_float(yw[i] & 0xFFFF0000u);
-            dot = fmaf(d0, y0, dot);
-            dot = fmaf(d1, y1, dot);
-            o[2 * i] = g * d0;
-            o[2 * i + 1] = g * d1;
+      for (int jj = 0; jj < kCombRows; ++jj) dot[jj] = 0.0f;
+      for (int v0 = lane; v0 < nvec; v0 += 32 * kCombVpl) {
+        uint4 d[kCombVpl], y[kCombRows][kCombVpl];
+#pragma unroll
+        for (int u = 0; u < kCombVpl; ++u) {
+          const int v = v0 + 32 * u;
+          d[u] = v < nvec ? drow[v] : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int jj = 0; jj < kCombRows; ++jj) {
+          const int j = j0 + jj;
+          const long long rj = j < k ? s_row[wib][j] : -1;
+          const uint4* yrow = reinterpret_cast<const uint4*>(ye + (rj >= 0 ? rj : 0) * dl);
+#pragma unroll
+          for (int u = 0; u < kCombVpl; ++u) {
+            const int v = v0 + 32 * u;
+            y[jj][u] = (rj >= 0 && v < nvec) ? yrow[v] : make_uint4(0, 0, 0, 0);
           }
-          out[v] = pack8(o);
+        }
+#pragma unroll
+        for (int jj = 0; jj < kCombRows; ++jj) {
+          const int j = j0 + jj;
+          const long long rj = j < k ? s_row[wib][j] : -1;
+          if (rj < 0) continue;
+          const float g = s_g[wib][j];
+          uint4* out = reinterpret_cast<uint4*>(dye + rj * dl);
+#pragma unroll
+          for (int u = 0; u < kCombVpl; ++u) {
+            const int v = v0 + 32 * u;
+            if (v >= nvec) continue;
+            const uint32_t dw[4] = {d[u].x, d[u].y, d[u].z, d[u].w};
+            const uint32_t yw[4] = {y[jj][u].x, y[jj][u].y, y[jj][u].z, y[jj][u].w};
+            float o[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float d0 = __uint_as_float(dw[i] << 16), d1 = __uint_as_float(dw[i] & 0xFFFF0000u);
+              const float y0 = __uint_as_float(yw[i] << 16), y1 = __uint_as_float(yw[i] & 0xFFFF0000u);
+              dot[jj] = fmaf(d0, y0, dot[jj]);
+              dot[jj] = fmaf(d1, y1, dot[jj]);
+              o[2 * i] = g * d0;
+              o[2 * i + 1] = g * d1;
+            }
+            out[v] = pack8(o);
+          }
         }
       }
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-      if (lane == 0) dg[a] = rs >= 0 ? dot : 0.0f;
+      for (int jj = 0; jj < kCombRows; ++jj) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) dot[jj] += __shfl_xor_sync(0xffffffffu, dot[jj], off);
+      }
+      if (lane < kCombRows && j0 + lane < k) {
+        float mine = 0.0f;
+#pragma unroll
+        for (int jj = 0; jj < kCombRows; ++jj)
+          if (jj == lane) mine = dot[jj];
+        dg[static_cast<long long>(t) * k + j0 + lane] = s_row[wib][j0 + lane] >= 0 ? mine : 0.0f;
+      }
     }
+    __syncwarp();
   }
 }
 
