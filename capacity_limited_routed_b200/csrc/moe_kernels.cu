@@ -367,7 +367,8 @@ constexpr int kPackWarps = 8;
 __global__ void __launch_bounds__(32 * kPackWarps)
     pack_bulk_kernel(const uint16_t* __restrict__ z, const int32_t* __restrict__ idx,
                      const int32_t* __restrict__ slot, int T, int k, int dl, int L, int P, int W, int Cs, int E,
-                     uint16_t* __restrict__ pools, int32_t* __restrict__ status) {
+                     const int32_t* __restrict__ pool_fill, int NP, uint16_t* __restrict__ pools,
+                     int32_t* __restrict__ status) {
   extern __shared__ __align__(128) uint8_t pack_smem[];
   __shared__ uint64_t s_bar[kPackWarps][2];
   __shared__ long long s_dst[kPackWarps][32];
@@ -434,6 +435,14 @@ __global__ void __launch_bounds__(32 * kPackWarps)
     }
     if (ok_j) *reinterpret_cast<int4*>(pools + s_dst[wib][lane] + dl) = make_int4(e_j, 0, 0, 0);
     __syncwarp();
+  }
+  // header -1 for the rows of each pool past its fill (slots below the fill are dense)
+  const long long n_rows = static_cast<long long>(NP) * Cs;
+  for (long long rr = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; rr < n_rows;
+       rr += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int pl = static_cast<int>(rr / Cs);
+    if (static_cast<int>(rr - static_cast<long long>(pl) * Cs) >= pool_fill[pl])
+      *reinterpret_cast<int4*>(pools + rr * row_elems + dl) = make_int4(-1, 0, 0, 0);
   }
   if (lane == 0) bulk_wait_all();
 }
@@ -897,7 +906,9 @@ moe_status_t launch_pack(const Geo& g, const uint16_t* z, const int32_t* idx, co
       const int grid = static_cast<int>(std::min<long long>((g.T + kPackWarps - 1) / kPackWarps,
                                                             static_cast<long long>(device_sm_count()) * per_sm));
       pack_bulk_kernel<<<grid, 32 * kPackWarps, smem, st>>>(z, idx, slot, g.T, g.k, g.dl, g.L, g.P, g.W, g.Cs, g.E,
-                                                            pools, stats + 3);
+                                                            stats + stats_pool_fill(g), g.NP, pools, stats + 3);
+      count_launch();
+      return cuda_check(cudaGetLastError(), "pack");
     } else {
       const int warps = 8;
       pack_kernel<<<blocks_for(g.T, warps), 32 * warps, 0, st>>>(z, idx, slot, g.T, g.k, g.dl, g.L, g.P, g.W, g.Cs,
