@@ -40,8 +40,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # captured ones, and as null once they change.
 NCU_TRAFFIC = {
     "bwd.experts_wgrad_gate_up": {
-        "sources_sha256": "fbeb515446d98d0705db7d00ad0608e38d53ad0713f1ced9e4b2b4feedc7e953",
-        "dram_bytes": 1918019584, "experts": 24, "tokens": 1024, "d_latent": 3072, "hidden_routed": 3072,
+        "sources_sha256": "15b9e7cfe34c2cad2e1facb33c0599eb3b11f831afd58701fb04566102d9a00a",
+        "dram_bytes": 1917372160, "experts": 24, "tokens": 1024, "d_latent": 3072, "hidden_routed": 3072,
     },
 }
 KERNEL_SOURCES = ("gemm_sm100.cu", "ptx.cuh", "internal.h")
