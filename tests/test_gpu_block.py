@@ -19,6 +19,11 @@ pytestmark = pytest.mark.gpu
 
 RAGGED = synth.MoEShape("ragged", T=333, d_model=192, d_latent=128, n_experts=48, top_k=3, n_dest=8,
                         hidden_routed=256, n_shared=2, hidden_shared=128, seed=9)
+# more choices per token than the combine kernels batch per pass (8), and a single one
+WIDE_K = synth.MoEShape("wide_k", T=200, d_model=192, d_latent=128, n_experts=48, top_k=12, n_dest=8,
+                        hidden_routed=256, n_shared=1, hidden_shared=128, seed=13)
+TOP1 = synth.MoEShape("top1", T=300, d_model=192, d_latent=128, n_experts=24, top_k=1, n_dest=4,
+                      hidden_routed=128, n_shared=1, hidden_shared=128, seed=14)
 
 
 def _run(shape, backward):
@@ -44,7 +49,7 @@ def _routing_agreement(views, ctx):
     return match, affected
 
 
-@pytest.mark.parametrize("shape", [synth.TINY, RAGGED, synth.MID], ids=lambda s: s.name)
+@pytest.mark.parametrize("shape", [synth.TINY, RAGGED, WIDE_K, TOP1, synth.MID], ids=lambda s: s.name)
 def test_forward_matches_oracle(shape):
     r = _run(shape, backward=False)
     s, inp, blk = r["s"], r["inp"], r["blk"]
@@ -69,7 +74,7 @@ def test_forward_matches_oracle(shape):
         assert np.array_equal(v["expert_rows"].cpu().numpy(), sl["expert_kept"])
 
 
-@pytest.mark.parametrize("shape", [synth.TINY, RAGGED, synth.MID], ids=lambda s: s.name)
+@pytest.mark.parametrize("shape", [synth.TINY, RAGGED, WIDE_K, TOP1, synth.MID], ids=lambda s: s.name)
 def test_backward_matches_oracle(shape):
     r = _run(shape, backward=True)
     s, inp, blk = r["s"], r["inp"], r["blk"]
