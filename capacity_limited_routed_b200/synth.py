@@ -47,6 +47,7 @@ class MoEShape:
     n_waves: int = 3
     cap_send: tuple = (110, 100)
     cap_recv: tuple = (115, 100)
+    dropless: bool = False       # no cap binds: every assignment kept (ragged buffers)
     # workload-only knobs (input recipe, not part of the block)
     zipf_s: float = 0.0          # >0: per-expert logit skew with Zipf(s) expected load
     window: int = 0              # >0: tokens in windows of this size share a component
@@ -73,6 +74,9 @@ WORKLOADS = {1: TINY, 2: MID, 3: FULL, 4: SKEWED, 5: TRAIN}
 # over 4 destinations and T=1024, so each expert still receives ~341 of C_r=393 rows
 # as in the full layer, with ~4.5 GB on the device instead of ~50 GB.
 PROFILE = TRAIN.with_(name="profile", T=1024, n_experts=24, n_dest=4, seed=5)
+# the dropless variant of the full-width training step and of the skewed stress
+TRAIN_DROPLESS = TRAIN.with_(name="train_dropless", dropless=True)
+SKEWED_DROPLESS = SKEWED.with_(name="skewed_dropless", dropless=True)
 
 
 def to_bf16_bits(a: np.ndarray) -> np.ndarray:

@@ -30,7 +30,8 @@ What the pages fix, and the readings taken where they are silent:
     expert; overflow assignments are dropped and counted separately ([RU] §2).
     Capacities are the expected row counts times the factor, rounded up in exact
     integer arithmetic (reading): C_s = ceil(1.10 * T*k / (D*W)),
-    C_r = ceil(1.15 * T*k / E).
+    C_r = ceil(1.15 * T*k / E).  The dropless variant ([ZH] §3.3, §7) is the same
+    assignment with no cap binding (``dropless_geometry``).
   * Sender slots are given in (token, rank) order; receiver slots are given among
     the sender-kept rows in the same order (reading).  One GPU is one source.
   * Combine: gate-weighted sum in latent space of the kept expert outputs, then
@@ -154,6 +155,21 @@ def geometry(shape) -> Geometry:
     L = E // D
     C_s, C_r = capacities(shape.T, shape.top_k, E, D, W, shape.cap_send, shape.cap_recv)
     return Geometry(T=shape.T, E=E, k=shape.top_k, D=D, W=W, L=L, P=L // W, C_s=C_s, C_r=C_r)
+
+
+def dropless_geometry(g: Geometry, idx: np.ndarray) -> Geometry:
+    """Capacities of the dropless variant for one routing ([ZH] §3.3 and §7: the run
+    later switched to a dropless ragged all-to-all).
+
+    Reading: the same slot assignment with no cap binding (C = infinity).  A rank can
+    never reach past the largest pool load or the largest expert load of the routing
+    itself, so those two numbers serve as the capacities: every assignment is kept,
+    every pool and expert holds exactly its load.
+    """
+    pool = placement(g)["pool"][np.asarray(idx)]
+    C_s = int(np.bincount(pool.ravel(), minlength=g.n_pools).max()) if pool.size else 0
+    C_r = int(np.bincount(np.asarray(idx).ravel(), minlength=g.E).max()) if pool.size else 0
+    return Geometry(T=g.T, E=g.E, k=g.k, D=g.D, W=g.W, L=g.L, P=g.P, C_s=max(C_s, 1), C_r=max(C_r, 1))
 
 
 def placement(g: Geometry) -> dict:
@@ -340,6 +356,8 @@ def forward(x, weights: dict, bias, shape, logit_offset=None, storage: str = "bf
     else:
         logits = np.asarray(logits_override, dtype=np.float32)
     idx, gate, hist = route(logits, bias, g.k)
+    if getattr(shape, "dropless", False):
+        g = dropless_geometry(g, idx)
     slots = assign_slots(idx, g)
     # routed experts on their kept rows, receiver-slot order
     T, k = idx.shape
@@ -497,6 +515,8 @@ def route_batch(x, weights, bias, shape, logit_offset=None, storage="bf16"):
         lg = lg + np.asarray(logit_offset, dtype=np.float64)[None, :]
     logits = lg.astype(np.float32) if storage == "bf16" else lg
     idx, gate, hist = route(logits, bias, g.k)
+    if getattr(shape, "dropless", False):
+        g = dropless_geometry(g, idx)
     slots = assign_slots(idx, g)
     return {"geometry": g, "storage": storage, "x": x, "z": z, "logits": logits, "idx": idx, "gate": gate,
             "hist": hist, "slots": slots, "kept": slots["rslot"] >= 0}
