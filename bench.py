@@ -1,6 +1,6 @@
 """Benchmark of the capacity-limited, pooled-wave MoE block on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload train|full|mid|skewed]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload train|full|mid|skewed|train_dropless|skewed_dropless]
                     [--impl ours|reference]
 
 A step is one pass of the whole hot path on one batch: forward (latent down-projection,
@@ -77,14 +77,17 @@ def load_peaks():
 def workload_shape(name):
     from capacity_limited_routed_b200 import synth
     return {"train": synth.TRAIN, "full": synth.FULL, "mid": synth.MID, "skewed": synth.SKEWED,
-            "tiny": synth.TINY.with_(backward=True), "profile": synth.PROFILE}[name]
+            "tiny": synth.TINY.with_(backward=True), "profile": synth.PROFILE,
+            "train_dropless": synth.TRAIN_DROPLESS, "skewed_dropless": synth.SKEWED_DROPLESS}[name]
 
 
 def describe(s):
     return (f"{s.name}: MoE block {'fwd+bwd+bias step' if s.backward else 'forward'}, T={s.T}, "
             f"d_model {s.d_model}, latent {s.d_latent}, E={s.n_experts} top-{s.top_k}, "
-            f"D={s.n_dest} x {s.n_waves} waves, caps {s.cap_send[0]/s.cap_send[1]:.2f}/"
-            f"{s.cap_recv[0]/s.cap_recv[1]:.2f}, {s.n_shared} shared x {s.hidden_shared}"
+            f"D={s.n_dest} x {s.n_waves} waves, "
+            + ("dropless (no caps)" if s.dropless else
+               f"caps {s.cap_send[0]/s.cap_send[1]:.2f}/{s.cap_recv[0]/s.cap_recv[1]:.2f}")
+            + f", {s.n_shared} shared x {s.hidden_shared}"
             + (f", Zipf({s.zipf_s}) logit skew, rho={s.rho} windows of {s.window}" if s.zipf_s else ""))
 
 

@@ -42,6 +42,7 @@ struct TmaMaps {
 struct KParams {
   int M, N, groups, ragged;
   const int32_t* group_rows;
+  const int32_t* group_off;  // ragged rows packed by group: group g starts at row group_off[g]
   int nseg;
   int seg_kb[3];
   int m_fastest;
@@ -113,6 +114,7 @@ __device__ __forceinline__ void record_status(int32_t* status, int code) {
 
 struct Tile {
   int g, m, n, kb;
+  int off;  // first row of group g in packed activation tensors (0 when not packed)
 };
 
 // Tile bookkeeping shared by the three roles; all of them walk the same list.
@@ -161,11 +163,12 @@ struct Sched {
     Tile r;
     if (t >= total) {
       r.g = -1;
-      r.m = r.n = r.kb = 0;
+      r.m = r.n = r.kb = r.off = 0;
       return r;
     }
     decode(t, r.g, r.m, r.n);
     r.kb = k_blocks(r.g);
+    r.off = p.group_off != nullptr ? p.group_off[r.g] : 0;
     return r;
   }
 
@@ -283,6 +286,10 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
         const Tile cur = nxt;
         nxt = sc.tile(t + gridDim.x);  // issued a tile ahead: its count load overlaps this tile
         const int g = cur.g, mt = cur.m, ntile = cur.n, kb_total = cur.kb;
+        // packed activations: 2-D tensors, rows offset by the group's first row
+        const int gz = p.group_off != nullptr ? 0 : g, gro = cur.off;
+        (void)gz;
+        (void)gro;
         for (int kb = 0; kb < kb_total; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_v)) {
             ok = false;
@@ -302,7 +309,7 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
           armed_phase[stage] = static_cast<int>(phase);
           const int m0 = mt * kBM;
           if (!A_MN) {
-            tma_load_3d(&maps.a[s], sa, &full[stage], k0, m0, g);
+            tma_load_3d(&maps.a[s], sa, &full[stage], k0, gro + m0, gz);
           } else {
             tma_load_3d(&maps.a[s], sa, &full[stage], m0, k0, g);
             tma_load_3d(&maps.a[s], sa + 8192, &full[stage], m0 + 64, k0, g);
@@ -410,6 +417,10 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
       const Tile cur = nxt;
       nxt = sc.tile(t + gridDim.x);
       const int g = cur.g, mt = cur.m, ntile = cur.n, kb_total = cur.kb;
+        // packed activations: 2-D tensors, rows offset by the group's first row
+        const int gz = p.group_off != nullptr ? 0 : g, gro = cur.off;
+        (void)gz;
+        (void)gro;
       const int row = mt * kBM + row_in_tile;
       const bool row_ok = row < p.M;
       if (kb_total == 0) {
@@ -446,8 +457,8 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
         uint64_t* bar = &ebar[3 * (warp - 2) + slot];
         bulk_wait_read<1>();  // the stores of the slot's previous chunk have read it
         mbar_arrive_expect_tx(bar, 2048);
-        tma_load_3d(&maps.aux_a, sb, bar, ntile * BN + ch * 16, srow0, g);
-        tma_load_3d(&maps.aux_b, sb + 1024, bar, ntile * BN + ch * 16, srow0, g);
+        tma_load_3d(&maps.aux_a, sb, bar, ntile * BN + ch * 16, gro + srow0, gz);
+        tma_load_3d(&maps.aux_b, sb + 1024, bar, ntile * BN + ch * 16, gro + srow0, gz);
       };
       if constexpr (EPI == EPI_SWIGLU_BWD) {
         if (lane == 0 && s_live > 0) swb_issue(0, eslot);
@@ -516,10 +527,10 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
           __syncwarp();
           const int col0 = n_out0 + c;
           if (lane == 0 && col0 < p.N && row0 < p.M) {
-            tma_store_3d(&maps.out, buf, col0, row0, g);
+            tma_store_3d(&maps.out, buf, col0, gro + row0, gz);
             if (p.save_a != nullptr) {
-              tma_store_3d(&maps.aux_a, buf + 2048, col0, row0, g);
-              tma_store_3d(&maps.aux_b, buf + 4096, col0, row0, g);
+              tma_store_3d(&maps.aux_a, buf + 2048, col0, gro + row0, gz);
+              tma_store_3d(&maps.aux_b, buf + 4096, col0, gro + row0, gz);
             }
             bulk_commit();
           }
@@ -633,7 +644,7 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
             fence_async_shared();
             __syncwarp();
             if (lane == 0) {
-              tma_store_3d(&maps.out, buf, col0, row0, g);
+              tma_store_3d(&maps.out, buf, col0, gro + row0, gz);
               bulk_commit();
             }
           }
@@ -689,8 +700,8 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
           fence_async_shared();
           __syncwarp();
           if (lane == 0) {
-            tma_store_3d(&maps.out, sb, ntile * BN + ch * 16, srow0, g);
-            tma_store_3d(&maps.out2, sb + 1024, ntile * BN + ch * 16, srow0, g);
+            tma_store_3d(&maps.out, sb, ntile * BN + ch * 16, gro + srow0, gz);
+            tma_store_3d(&maps.out2, sb + 1024, ntile * BN + ch * 16, gro + srow0, gz);
             bulk_commit();
           }
         }
@@ -883,15 +894,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   // before it instead of stalling the pipeline at each tile boundary.
   struct PairTile {
     int g, m, n, kb;
+    int off;  // first K row of group g in packed activation tensors (0 when not packed)
   };
   auto fetch = [&](int t) {
-    PairTile r{0, 0, 0, 0};
+    PairTile r{0, 0, 0, 0, 0};
     if (t < total) {
       r.g = t / per_group;
       const int l = t - r.g * per_group;
       r.n = l % nt_n;
       r.m = l / nt_n;
       r.kb = k_blocks(r.g);
+      r.off = p.group_off != nullptr ? p.group_off[r.g] : 0;
     }
     return r;
   };
@@ -909,6 +922,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const PairTile cur = nxt;
         nxt = fetch(t + npairs);
         const int g = cur.g, mt = cur.m, ntile = cur.n, kb_total = cur.kb;
+        // packed activations: 2-D tensors, rows offset by the group's first row
+        const int gz = p.group_off != nullptr ? 0 : g, gro = cur.off;
+        (void)gz;
+        (void)gro;
         const int m0 = mt * 256 + 128 * static_cast<int>(rank);
         const int n0 = ntile * 256 + 128 * static_cast<int>(rank);
         for (int kb = 0; kb < kb_total; ++kb) {
@@ -922,10 +939,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           uint8_t* sa = smem + stage * C::kStage;
           uint8_t* sb = sa + C::kABytes;
           const int k0 = kb * kBK;
-          tma_load_3d_pair(&maps.a[0], sa, bar, m0, k0, g);
-          tma_load_3d_pair(&maps.a[0], sa + 8192, bar, m0 + 64, k0, g);
-          tma_load_3d_pair(&maps.b[0], sb, bar, n0, k0, g);
-          tma_load_3d_pair(&maps.b[0], sb + 8192, bar, n0 + 64, k0, g);
+          tma_load_3d_pair(&maps.a[0], sa, bar, m0, gro + k0, gz);
+          tma_load_3d_pair(&maps.a[0], sa + 8192, bar, m0 + 64, gro + k0, gz);
+          tma_load_3d_pair(&maps.b[0], sb, bar, n0, gro + k0, gz);
+          tma_load_3d_pair(&maps.b[0], sb + 8192, bar, n0 + 64, gro + k0, gz);
           if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1u;
@@ -957,6 +974,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const PairTile cur = nxt;
         nxt = fetch(t + npairs);
         const int g = cur.g, mt = cur.m, ntile = cur.n, kb_total = cur.kb;
+        // packed activations: 2-D tensors, rows offset by the group's first row
+        const int gz = p.group_off != nullptr ? 0 : g, gro = cur.off;
+        (void)gz;
+        (void)gro;
         if (kb_total == 0) continue;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_v)) {
           ok = false;
@@ -1016,6 +1037,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       const PairTile cur = nxt;
       nxt = fetch(t + npairs);
       const int g = cur.g, mt = cur.m, ntile = cur.n, kb_total = cur.kb;
+        // packed activations: 2-D tensors, rows offset by the group's first row
+        const int gz = p.group_off != nullptr ? 0 : g, gro = cur.off;
+        (void)gz;
+        (void)gro;
       const int row0 = mt * 256 + 128 * static_cast<int>(rank) + q * 32;
       if (kb_total == 0) {
         pair_zero(p, col_lo, ntile, row0, g, lane);
@@ -1130,6 +1155,12 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
   if (a.nseg < 1 || a.nseg > 3) return fail(MOE_ERR_INVALID_ARG, "gemm needs 1..3 K segments");
   if (a.ragged != 0 && a.group_rows == nullptr) return fail(MOE_ERR_INVALID_ARG, "ragged gemm needs group rows");
   if (a.ragged == 2 && a.nseg != 1) return fail(MOE_ERR_INVALID_ARG, "ragged-K gemm takes one segment");
+  // packed groups: activations are 2-D (rows_total rows), weights 3-D; only the epilogues
+  // and kernels that address activation rows through tensor maps take them
+  const bool packed = a.group_off != nullptr;
+  if (packed && (a.ragged == 0 || a.rows_total <= 0 || a.epi == EPI_BF16_ADD_F32 ||
+                 (a.ragged == 2 && !(a.a_mn && a.b_mn && a.epi == EPI_F32 && a.bn == 256))))
+    return fail(MOE_ERR_UNSUPPORTED, "packed groups need ragged rows or a ragged-K weight gradient");
   if (a.epi == EPI_SWIGLU && (a.nseg != 1 || a.b_mn || a.N % (a.bn / 2) != 0))
     return fail(MOE_ERR_UNSUPPORTED, "SwiGLU gemm needs one K-major segment and N a multiple of BN/2");
   if (a.N % 8 != 0) return fail(MOE_ERR_UNSUPPORTED, "gemm N must be a multiple of 8");
@@ -1146,6 +1177,7 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
   kp.groups = a.groups;
   kp.ragged = a.ragged;
   kp.group_rows = a.group_rows;
+  kp.group_off = a.group_off;
   kp.nseg = a.nseg;
   for (int s = 0; s < a.nseg; ++s) {
     moe_status_t r;
@@ -1166,10 +1198,10 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
       Mat o;
       o.ptr = ptr;
       o.inner = a.N;
-      o.rows = a.M;
-      o.groups = a.groups;
+      o.rows = packed ? a.rows_total : a.M;
+      o.groups = packed ? 1 : a.groups;
       o.ld = ld;
-      o.gs = a.groups > 1 ? gs : ld * a.M;
+      o.gs = (a.groups > 1 && !packed) ? gs : ld * o.rows;
       return make_map(m, o, 32, 32, what, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, CU_TENSOR_MAP_SWIZZLE_64B);
     };
     moe_status_t r = tile(&maps.out, a.out, a.ldo, a.out_gs, "output");
@@ -1185,10 +1217,10 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
         Mat o;
         o.ptr = ptr;
         o.inner = a.N;
-        o.rows = a.M;
-        o.groups = a.groups;
+        o.rows = packed ? a.rows_total : a.M;
+        o.groups = packed ? 1 : a.groups;
         o.ld = ld;
-        o.gs = a.groups > 1 ? gs : ld * a.M;
+        o.gs = (a.groups > 1 && !packed) ? gs : ld * o.rows;
         return make_map(m, o, 16, 32, what, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, CU_TENSOR_MAP_SWIZZLE_NONE);
       };
       if ((r = tile16(&maps.out, a.out, a.ldo, a.out_gs, "dA")) != MOE_OK) return r;
@@ -1201,10 +1233,12 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
     Mat o;
     o.ptr = a.out;
     o.inner = a.N;
-    o.rows = a.M;
-    o.groups = a.groups;
+    // a packed ragged-row output is 2-D; a weight gradient's output stays one per group
+    const bool packed_out = packed && a.ragged == 1;
+    o.rows = packed_out ? a.rows_total : a.M;
+    o.groups = packed_out ? 1 : a.groups;
     o.ld = a.ldo;
-    o.gs = a.groups > 1 ? a.out_gs : a.ldo * a.M;
+    o.gs = (a.groups > 1 && !packed_out) ? a.out_gs : a.ldo * o.rows;
     moe_status_t r = a.epi == EPI_F32
                          ? make_map(&maps.out, o, 32, 32, "output", CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4)
                          : make_map(&maps.out, o, 64, 32, "output");

@@ -68,6 +68,11 @@ struct GemmArgs {
   int groups = 1;
   int ragged = 0;
   const int32_t* group_rows = nullptr;
+  // ragged == 1 or 2 with buffers packed by expert: group g's rows start at row
+  // group_off[g] of 2-D activation tensors (rows_total rows, groups = 1) instead of
+  // being group g of a 3-D tensor; weights (and weight gradients) stay 3-D
+  const int32_t* group_off = nullptr;
+  int64_t rows_total = 0;
   int nseg = 1;
   Mat A[3], B[3];
   Mat Bv;            // value weights paired with B[0] for EPI_SWIGLU
@@ -95,6 +100,11 @@ int device_sm_count();
 struct Geo {
   int T, E, k, D, W, L, P, NP, Cs, Cr, dl;
   int n_chunks;      // token chunks of the slot scan
+  // dropless variant: no cap binds (Cs = Cr = T*k); pools are packed back to back in
+  // pool order (pool_rows = T*k rows) and expert buffers by expert, each expert's
+  // region padded to a multiple of 128 rows (exp_rows = T*k + 127*E rows)
+  bool dropless;
+  int64_t pool_rows, exp_rows;
 };
 
 constexpr int kScanTokensPerChunk = 32;
@@ -106,21 +116,28 @@ size_t scan_scratch_ints(const Geo& g);
 moe_status_t launch_slot_scan(const Geo& g, const int32_t* idx, int32_t* slot, int32_t* stats, int32_t* scratch,
                               cudaStream_t st);
 moe_status_t launch_pack(const Geo& g, const uint16_t* z, const int32_t* idx, const int32_t* slot,
-                         int32_t* stats, uint16_t* pools, cudaStream_t st);
+                         int32_t* stats, uint16_t* pools, cudaStream_t st, const int32_t* pool_off = nullptr);
+// off[i] = sum over j < i of round_up(counts[j], align), i = 0..n (n <= 1024)
+moe_status_t launch_offsets(const int32_t* counts, int n, int align, int32_t* off, cudaStream_t st);
 // scratch ints needed by the receiver's row map
 size_t unpack_scratch_ints(const Geo& g);
+// capacity layout: pool_off = exp_off = nullptr.  Dropless: pool_off / pool_fill give
+// each pool's packed row range; exp_off (E+1 ints) is computed here from the counts.
 moe_status_t launch_unpack(const Geo& g, const uint16_t* pools, uint16_t* xe, int32_t* rows, int32_t* row_map,
-                           int32_t* status, cudaStream_t st);
+                           int32_t* status, cudaStream_t st, const int32_t* pool_off = nullptr,
+                           const int32_t* pool_fill = nullptr, int32_t* exp_off = nullptr);
 moe_status_t launch_zero_tail_rows(const Geo& g, uint16_t* buf, int64_t width, const int32_t* rows,
-                                   cudaStream_t st);
+                                   cudaStream_t st, const int32_t* exp_off = nullptr);
+// exp_off: row of each expert's first row in the expert buffers (dropless); nullptr:
+// expert e's rows start at e * C_r
 moe_status_t launch_combine(const Geo& g, const uint16_t* ye, const float* gate, const int32_t* idx,
-                            const int32_t* slot, uint16_t* r, cudaStream_t st);
+                            const int32_t* slot, uint16_t* r, cudaStream_t st, const int32_t* exp_off = nullptr);
 moe_status_t launch_combine_bwd(const Geo& g, const uint16_t* dr, const uint16_t* ye, const float* gate,
                                 const int32_t* idx, const int32_t* slot, uint16_t* dye, float* dg,
-                                cudaStream_t st);
+                                cudaStream_t st, const int32_t* exp_off = nullptr);
 moe_status_t launch_undispatch(const Geo& g, const uint16_t* dxe, const float* gate, const float* dg,
                                const int32_t* idx, const int32_t* slot, float* dz_routed, uint16_t* dlogits,
-                               cudaStream_t st);
+                               cudaStream_t st, const int32_t* exp_off = nullptr);
 moe_status_t launch_bias_update(const Geo& g, const int32_t* hist, float* bias, float step, cudaStream_t st);
 
 // plan geometry and the device check, for entry points defined in other files

@@ -23,7 +23,7 @@ struct moe_plan {
   int dm, dl, E, k, h, S, hs;
   // forward context layout (byte offsets); training adds the SwiGLU pre-activations
   struct Ctx {
-    size_t z, logits, idx, gate, slot, rows, xe, ae, be, he, ye, r, as, bs, hsh, bytes;
+    size_t z, logits, idx, gate, slot, rows, xe, ae, be, he, ye, r, as, bs, hsh, exp_off, pool_off, bytes;
   } saved, infer;
   // scratch layouts
   size_t ws_scan, ws_pools, ws_rowmap, ws_ctx, ws_fwd_bytes;             // forward
@@ -121,7 +121,10 @@ size_t take(size_t& off, size_t bytes) {
 }
 
 void layout_ctx(const moe_plan& p, bool training, moe_plan::Ctx& c) {
-  const size_t T = p.g.T, E = p.E, k = p.k, dl = p.dl, h = p.h, Cr = p.g.Cr, SH = size_t(p.S) * p.hs;
+  // expert buffers: E x C_r rows, or (dropless) every assignment packed by expert with
+  // each expert's region padded to 128 rows
+  const size_t T = p.g.T, E = p.E, k = p.k, dl = p.dl, h = p.h, SH = size_t(p.S) * p.hs;
+  const size_t R = size_t(p.g.exp_rows);
   size_t off = 0;
   c.z = take(off, T * dl * 2);
   c.logits = take(off, T * E * 4);
@@ -129,24 +132,27 @@ void layout_ctx(const moe_plan& p, bool training, moe_plan::Ctx& c) {
   c.gate = take(off, T * k * 4);
   c.slot = take(off, T * k * 8);
   c.rows = take(off, E * 4);
-  c.xe = take(off, E * Cr * dl * 2);
-  c.ae = training ? take(off, E * Cr * h * 2) : 0;
-  c.be = training ? take(off, E * Cr * h * 2) : 0;
-  c.he = take(off, E * Cr * h * 2);
-  c.ye = take(off, E * Cr * dl * 2);
+  c.xe = take(off, R * dl * 2);
+  c.ae = training ? take(off, R * h * 2) : 0;
+  c.be = training ? take(off, R * h * 2) : 0;
+  c.he = take(off, R * h * 2);
+  c.ye = take(off, R * dl * 2);
   c.r = take(off, T * dl * 2);
   c.as = training ? take(off, T * SH * 2) : 0;
   c.bs = training ? take(off, T * SH * 2) : 0;
   c.hsh = take(off, T * SH * 2);
+  c.exp_off = take(off, (E + 1) * 4);
+  c.pool_off = take(off, (size_t(p.g.NP) + 1) * 4);
   c.bytes = (off + kAlign - 1) / kAlign * kAlign;
 }
 
 void layout(moe_plan& p) {
-  const size_t T = p.g.T, E = p.E, k = p.k, dl = p.dl, h = p.h, Cr = p.g.Cr, SH = size_t(p.S) * p.hs;
+  const size_t T = p.g.T, E = p.E, k = p.k, dl = p.dl, h = p.h, SH = size_t(p.S) * p.hs;
+  const size_t R = size_t(p.g.exp_rows);
   layout_ctx(p, true, p.saved);
   layout_ctx(p, false, p.infer);
-  p.pools_bytes = size_t(p.g.NP) * p.g.Cs * (dl + 8) * 2;
-  p.expert_out_bytes = E * Cr * dl * 2;
+  p.pools_bytes = size_t(p.g.pool_rows) * (dl + 8) * 2;
+  p.expert_out_bytes = R * dl * 2;
   p.slot_bytes = T * k * 8;
   p.stats_bytes = size_t(stats_words(p.g)) * 4;
   size_t off = 0;
@@ -156,8 +162,8 @@ void layout(moe_plan& p) {
   p.ws_ctx = take(off, p.infer.bytes);  // used only when the forward keeps no context
   p.ws_fwd_bytes = off;
   off = 0;
-  p.ws_ffn_xe = take(off, E * Cr * dl * 2);
-  p.ws_ffn_he = take(off, E * Cr * h * 2);
+  p.ws_ffn_xe = take(off, R * dl * 2);
+  p.ws_ffn_he = take(off, R * h * 2);
   p.ws_ffn_rows = take(off, E * 4);
   p.ws_ffn_rowmap = take(off, unpack_scratch_ints(p.g) * 4);
   p.ws_ffn_bytes = off;
@@ -165,11 +171,11 @@ void layout(moe_plan& p) {
   p.b_dr = take(off, T * dl * 2);
   p.b_das = take(off, T * SH * 2);
   p.b_dbs = take(off, T * SH * 2);
-  p.b_dye = take(off, E * Cr * dl * 2);
+  p.b_dye = take(off, R * dl * 2);
   p.b_dg = take(off, T * k * 4);
-  p.b_dae = take(off, E * Cr * h * 2);
-  p.b_dbe = take(off, E * Cr * h * 2);
-  p.b_dxe = take(off, E * Cr * dl * 2);
+  p.b_dae = take(off, R * h * 2);
+  p.b_dbe = take(off, R * h * 2);
+  p.b_dxe = take(off, R * dl * 2);
   p.b_dlog = take(off, T * E * 2);
   p.b_dzr = take(off, T * dl * 4);
   p.b_dz = take(off, T * dl * 2);
@@ -238,6 +244,7 @@ struct CtxPtrs {
   uint16_t *z, *xe, *ae, *be, *he, *ye, *r, *as, *bs, *hsh;
   float *logits, *gate;
   int32_t *idx, *slot, *rows;
+  int32_t *exp_off, *pool_off;  // used by the dropless variant
 };
 
 CtxPtrs ctx_ptrs(const moe_plan& p, void* base, bool training) {
@@ -258,18 +265,35 @@ CtxPtrs ctx_ptrs(const moe_plan& p, void* base, bool training) {
   q.as = training ? at<uint16_t>(base, c.as) : nullptr;
   q.bs = training ? at<uint16_t>(base, c.bs) : nullptr;
   q.hsh = at<uint16_t>(base, c.hsh);
+  q.exp_off = at<int32_t>(base, c.exp_off);
+  q.pool_off = at<int32_t>(base, c.pool_off);
   return q;
+}
+
+// An expert activation buffer as a GEMM operand: E groups of C_r rows, or (dropless) one
+// 2-D tensor of exp_rows rows whose group g starts at row exp_off[g].
+Mat expert_mat(const Geo& g, const void* ptr, int64_t width) {
+  return g.dropless ? mat(ptr, width, g.exp_rows, 1) : mat(ptr, width, g.Cr, g.E);
+}
+
+void pack_groups(const Geo& g, GemmArgs& a, const int32_t* exp_off) {
+  if (!g.dropless) return;
+  a.group_off = exp_off;
+  a.rows_total = g.exp_rows;
+  if (a.ragged == 1) a.M = static_cast<int>(g.exp_rows);  // local rows never reach it
 }
 
 // receiver unpack + grouped SwiGLU experts (shared by moe_expert_ffn and moe_forward)
 moe_status_t run_experts(const moe_plan& p, const uint16_t* w1, const uint16_t* w3, const uint16_t* w2,
                          const uint16_t* pools, uint16_t* xe, int32_t* rows, int32_t* row_map, uint16_t* ae,
-                         uint16_t* be, uint16_t* he, uint16_t* ye, int32_t* status, cudaStream_t st) {
+                         uint16_t* be, uint16_t* he, uint16_t* ye, int32_t* status, cudaStream_t st,
+                         const int32_t* pool_off = nullptr, const int32_t* pool_fill = nullptr,
+                         int32_t* exp_off = nullptr) {
   const Geo& g = p.g;
   {
     ProfScope ps("experts.unpack", st);
-    MOE_TRY(launch_unpack(g, pools, xe, rows, row_map, status, st));
-    MOE_TRY(launch_zero_tail_rows(g, xe, p.dl, rows, st));
+    MOE_TRY(launch_unpack(g, pools, xe, rows, row_map, status, st, pool_off, pool_fill, exp_off));
+    MOE_TRY(launch_zero_tail_rows(g, xe, p.dl, rows, st, exp_off));
   }
   GemmArgs a;
   a.bn = 256;
@@ -279,7 +303,7 @@ moe_status_t run_experts(const moe_plan& p, const uint16_t* w1, const uint16_t* 
   a.groups = p.E;
   a.ragged = 1;
   a.group_rows = rows;
-  a.A[0] = mat(xe, p.dl, g.Cr, p.E);
+  a.A[0] = expert_mat(g, xe, p.dl);
   a.B[0] = mat(w1, p.dl, p.h, p.E);
   a.Bv = mat(w3, p.dl, p.h, p.E);
   a.K[0] = p.dl;
@@ -290,6 +314,7 @@ moe_status_t run_experts(const moe_plan& p, const uint16_t* w1, const uint16_t* 
   a.save_a = ae;
   a.save_b = be;
   a.status = status;
+  pack_groups(g, a, exp_off);
   {
     ProfScope ps("experts.gate_up", st);
     MOE_TRY(gemm_run(a, st));
@@ -302,7 +327,7 @@ moe_status_t run_experts(const moe_plan& p, const uint16_t* w1, const uint16_t* 
   d.groups = p.E;
   d.ragged = 1;
   d.group_rows = rows;
-  d.A[0] = mat(he, p.h, g.Cr, p.E);
+  d.A[0] = expert_mat(g, he, p.h);
   d.B[0] = mat(w2, p.h, p.dl, p.E);
   d.K[0] = p.h;
   d.m_fastest = true;
@@ -310,6 +335,7 @@ moe_status_t run_experts(const moe_plan& p, const uint16_t* w1, const uint16_t* 
   d.ldo = p.dl;
   d.out_gs = int64_t(g.Cr) * p.dl;
   d.status = status;
+  pack_groups(g, d, exp_off);
   ProfScope ps("experts.down", st);
   return gemm_run(d, st);
 }
@@ -364,8 +390,10 @@ moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out) {
   if (c.T < 0 || c.d_model <= 0 || c.d_latent <= 0 || c.n_experts <= 0 || c.top_k <= 0 || c.n_dest <= 0 ||
       c.n_waves <= 0 || c.hidden_routed <= 0 || c.n_shared <= 0 || c.hidden_shared <= 0)
     return fail(MOE_ERR_INVALID_ARG, "sizes must be positive (T may be 0)");
-  if (c.cap_send_num <= 0 || c.cap_send_den <= 0 || c.cap_recv_num <= 0 || c.cap_recv_den <= 0)
-    return fail(MOE_ERR_INVALID_ARG, "capacity ratios must be positive");
+  // both numerators 0: the dropless variant (no cap binds)
+  const bool dropless = c.cap_send_num == 0 && c.cap_recv_num == 0;
+  if (!dropless && (c.cap_send_num <= 0 || c.cap_send_den <= 0 || c.cap_recv_num <= 0 || c.cap_recv_den <= 0))
+    return fail(MOE_ERR_INVALID_ARG, "capacity ratios must be positive (or both numerators 0: dropless)");
   if (c.n_experts % c.n_dest != 0) return fail(MOE_ERR_UNSUPPORTED, "E must be a multiple of D");
   const int L = c.n_experts / c.n_dest;
   if (L % c.n_waves != 0) return fail(MOE_ERR_UNSUPPORTED, "E/D must be a multiple of the wave count");
@@ -397,10 +425,20 @@ moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out) {
   g.L = L;
   g.P = L / c.n_waves;
   g.NP = c.n_dest * c.n_waves;
-  g.Cs = ceil_cap(A, int64_t(c.n_dest) * c.n_waves, c.cap_send_num, c.cap_send_den);
-  g.Cr = ceil_cap(A, c.n_experts, c.cap_recv_num, c.cap_recv_den);
-  if (g.Cs < 1) g.Cs = 1;
-  if (g.Cr < 1) g.Cr = 1;
+  g.dropless = dropless;
+  if (dropless) {
+    // no slot reaches T*k, so no cap binds; buffers are packed (see Geo)
+    g.Cs = g.Cr = static_cast<int32_t>(A > 0 ? A : 1);
+    g.pool_rows = A;
+    g.exp_rows = A + int64_t(127) * c.n_experts;
+  } else {
+    g.Cs = ceil_cap(A, int64_t(c.n_dest) * c.n_waves, c.cap_send_num, c.cap_send_den);
+    g.Cr = ceil_cap(A, c.n_experts, c.cap_recv_num, c.cap_recv_den);
+    if (g.Cs < 1) g.Cs = 1;
+    if (g.Cr < 1) g.Cr = 1;
+    g.pool_rows = int64_t(g.NP) * g.Cs;
+    g.exp_rows = int64_t(c.n_experts) * g.Cr;
+  }
   g.dl = c.d_latent;
   g.n_chunks = (c.T + kScanTokensPerChunk - 1) / kScanTokensPerChunk;
   if (g.n_chunks < 1) g.n_chunks = 1;
@@ -419,8 +457,8 @@ moe_status_t moe_plan_info(moe_plan_t p, moe_plan_info_t* out) {
   out->local_experts = p->g.L;
   out->experts_per_wave = p->g.P;
   out->n_pools = p->g.NP;
-  out->cap_send = p->g.Cs;
-  out->cap_recv = p->g.Cr;
+  out->cap_send = p->g.dropless ? 0 : p->g.Cs;  // 0: no cap (dropless)
+  out->cap_recv = p->g.dropless ? 0 : p->g.Cr;
   out->pool_row_elems = p->dl + 8;
   out->pools_bytes = p->pools_bytes;
   out->expert_out_bytes = p->expert_out_bytes;
@@ -460,6 +498,8 @@ moe_status_t moe_route(moe_plan_t p, const float* logits, const float* bias, int
 moe_status_t moe_dispatch(moe_plan_t p, const uint16_t* z, const int32_t* topk_idx, uint16_t* pools, int32_t* slot,
                           void* stats, void* ws, size_t ws_bytes, void* stream) {
   if (p == nullptr) return fail(MOE_ERR_INVALID_ARG, "null plan");
+  if (p->g.dropless)
+    return fail(MOE_ERR_UNSUPPORTED, "the dropless variant runs through moe_forward / moe_backward only");
   if (!pools || !stats || !ws) return fail(MOE_ERR_INVALID_ARG, "null buffer");
   if (p->g.T > 0 && (!z || !topk_idx || !slot)) return fail(MOE_ERR_INVALID_ARG, "null buffer");
   if (!aligned16(z) || !aligned16(pools)) return fail(MOE_ERR_INVALID_ARG, "z and pools must be 16-byte aligned");
@@ -474,6 +514,8 @@ moe_status_t moe_dispatch(moe_plan_t p, const uint16_t* z, const int32_t* topk_i
 moe_status_t moe_expert_ffn(moe_plan_t p, const moe_expert_weights_t* w, const uint16_t* pools, uint16_t* expert_out,
                             int32_t* expert_rows, void* ws, size_t ws_bytes, void* stream) {
   if (p == nullptr || w == nullptr) return fail(MOE_ERR_INVALID_ARG, "null argument");
+  if (p->g.dropless)
+    return fail(MOE_ERR_UNSUPPORTED, "the dropless variant runs through moe_forward / moe_backward only");
   if (!w->w1 || !w->w3 || !w->w2 || !pools || !expert_out || !ws)
     return fail(MOE_ERR_INVALID_ARG, "null buffer");
   if (ws_bytes < p->ws_ffn_bytes) return fail(MOE_ERR_WORKSPACE, "workspace too small");
@@ -489,6 +531,8 @@ moe_status_t moe_expert_ffn(moe_plan_t p, const moe_expert_weights_t* w, const u
 moe_status_t moe_combine(moe_plan_t p, const uint16_t* expert_out, const float* topk_gate, const int32_t* topk_idx,
                          const int32_t* slot, uint16_t* r, void* stream) {
   if (p == nullptr) return fail(MOE_ERR_INVALID_ARG, "null plan");
+  if (p->g.dropless)
+    return fail(MOE_ERR_UNSUPPORTED, "the dropless variant runs through moe_forward / moe_backward only");
   if (p->g.T == 0) return MOE_OK;
   if (!expert_out || !topk_gate || !topk_idx || !slot || !r) return fail(MOE_ERR_INVALID_ARG, "null buffer");
   if (!aligned16(expert_out) || !aligned16(r)) return fail(MOE_ERR_INVALID_ARG, "buffers must be 16-byte aligned");
@@ -557,15 +601,19 @@ moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const uint16_t* x
     MOE_TRY(launch_slot_scan(g, c.idx, c.slot, s, at<int32_t>(ws, p->ws_scan), st));
   }
   uint16_t* pools = at<uint16_t>(ws, p->ws_pools);
+  // dropless: pools and expert buffers are packed; their offsets come from the counts
+  int32_t* pool_off = g.dropless ? c.pool_off : nullptr;
+  int32_t* exp_off = g.dropless ? c.exp_off : nullptr;
   {
     ProfScope ps("fwd.dispatch_pack", st);
-    MOE_TRY(launch_pack(g, c.z, c.idx, c.slot, s, pools, st));
+    if (g.dropless) MOE_TRY(launch_offsets(s + stats_pool_fill(g), g.NP, 1, pool_off, st));
+    MOE_TRY(launch_pack(g, c.z, c.idx, c.slot, s, pools, st, pool_off));
   }
   MOE_TRY(run_experts(*p, w->w1, w->w3, w->w2, pools, c.xe, c.rows, at<int32_t>(ws, p->ws_rowmap), c.ae, c.be,
-                      c.he, c.ye, status, st));
+                      c.he, c.ye, status, st, pool_off, g.dropless ? s + stats_pool_fill(g) : nullptr, exp_off));
   {
     ProfScope ps("fwd.combine", st);
-    MOE_TRY(launch_combine(g, c.ye, c.gate, c.idx, c.slot, c.r, st));
+    MOE_TRY(launch_combine(g, c.ye, c.gate, c.idx, c.slot, c.r, st, exp_off));
   }
   // shared experts: H_s = silu(x ws1^T) * (x ws3^T)
   {
@@ -634,6 +682,7 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
     return MOE_OK;
   }
   CtxPtrs c = ctx_ptrs(*p, const_cast<void*>(saved), true);
+  const int32_t* exp_off = g.dropless ? c.exp_off : nullptr;  // packed expert buffers (dropless)
   uint16_t* dr = at<uint16_t>(ws, p->b_dr);
   uint16_t* das = at<uint16_t>(ws, p->b_das);
   uint16_t* dbs = at<uint16_t>(ws, p->b_dbs);
@@ -702,8 +751,8 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
   // combine backward: dY = g dr on kept rows, dg = <dr, Y>
   {
     ProfScope ps("bwd.combine", st);
-    MOE_TRY(launch_combine_bwd(g, dr, c.ye, c.gate, c.idx, c.slot, dye, dg, st));
-    MOE_TRY(launch_zero_tail_rows(g, dye, dl, c.rows, st));
+    MOE_TRY(launch_combine_bwd(g, dr, c.ye, c.gate, c.idx, c.slot, dye, dg, st, exp_off));
+    MOE_TRY(launch_zero_tail_rows(g, dye, dl, c.rows, st, exp_off));
   }
   // routed experts: dH = dY w2 -> (dA, dB);  dw2 = dY^T H;  dX = dA w1 + dB w3;  dw1 = dA^T X, dw3 = dB^T X
   {
@@ -716,7 +765,7 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
     a.groups = p->E;
     a.ragged = 1;
     a.group_rows = c.rows;
-    a.A[0] = mat(dye, dl, Cr, E);
+    a.A[0] = expert_mat(g, dye, dl);
     a.B[0] = mat(w->w2, h, dl, E);
     a.K[0] = dl;
     a.m_fastest = true;
@@ -728,6 +777,7 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
     a.out2 = dbe;
     a.ldo = h;
     a.out_gs = Cr * h;
+    pack_groups(g, a, exp_off);
     MOE_TRY(gemm_run(a, st));
   }
   {
@@ -741,11 +791,12 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
     a.ragged = 2;
     a.group_rows = c.rows;
     a.m_fastest = false;  // concurrent tiles write whole rows of dW
-    a.A[0] = mat(dye, dl, Cr, E);
-    a.B[0] = mat(c.he, h, Cr, E);
+    a.A[0] = expert_mat(g, dye, dl);
+    a.B[0] = expert_mat(g, c.he, h);
     a.out = gr->w2;
     a.ldo = h;
     a.out_gs = dl * h;
+    pack_groups(g, a, exp_off);
     MOE_TRY(gemm_run(a, st));
   }
   {
@@ -758,16 +809,17 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
     a.ragged = 1;
     a.group_rows = c.rows;
     a.nseg = 2;
-    a.A[0] = mat(dae, h, Cr, E);
+    a.A[0] = expert_mat(g, dae, h);
     a.B[0] = mat(w->w1, dl, h, E);
     a.K[0] = h;
-    a.A[1] = mat(dbe, h, Cr, E);
+    a.A[1] = expert_mat(g, dbe, h);
     a.B[1] = mat(w->w3, dl, h, E);
     a.K[1] = h;
     a.m_fastest = true;
     a.out = dxe;
     a.ldo = dl;
     a.out_gs = Cr * dl;
+    pack_groups(g, a, exp_off);
     MOE_TRY(gemm_run(a, st));
   }
   {
@@ -781,20 +833,21 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
     a.ragged = 2;
     a.group_rows = c.rows;
     a.m_fastest = false;  // concurrent tiles write whole rows of dW
-    a.A[0] = mat(dae, h, Cr, E);
-    a.B[0] = mat(c.xe, dl, Cr, E);
+    a.A[0] = expert_mat(g, dae, h);
+    a.B[0] = expert_mat(g, c.xe, dl);
     a.out = gr->w1;
     a.ldo = dl;
     a.out_gs = h * dl;
+    pack_groups(g, a, exp_off);
     MOE_TRY(gemm_run(a, st));
-    a.A[0] = mat(dbe, h, Cr, E);
+    a.A[0] = expert_mat(g, dbe, h);
     a.out = gr->w3;
     MOE_TRY(gemm_run(a, st));
   }
   // un-dispatch and the softmax backward to the logits
   {
     ProfScope ps("bwd.undispatch", st);
-    MOE_TRY(launch_undispatch(g, dxe, c.gate, dg, c.idx, c.slot, dzr, dlog, st));
+    MOE_TRY(launch_undispatch(g, dxe, c.gate, dg, c.idx, c.slot, dzr, dlog, st, exp_off));
   }
   // dz = dlogits W_r + dz_routed;  dW_r = dlogits^T z
   {

@@ -28,6 +28,12 @@
 
 namespace moe {
 
+#define MOE_TRY_K(x)               \
+  do {                             \
+    moe_status_t _s = (x);         \
+    if (_s != MOE_OK) return _s;   \
+  } while (0)
+
 namespace {
 
 constexpr int kMaxE = 1024;
@@ -314,9 +320,19 @@ __global__ void scan_totals(int32_t* __restrict__ stats, int E, int NP, int A_to
 // ---------------------------------------------------------------------- pack / unpack
 
 // one warp per token: read z_t once, write it into every pool row it was given
+// first row of pool p: fixed-size pools at p * C_s, packed pools (dropless) at pool_off[p]
+__device__ __forceinline__ long long pool_row0(int p, int Cs, const int32_t* pool_off) {
+  return pool_off != nullptr ? static_cast<long long>(pool_off[p]) : static_cast<long long>(p) * Cs;
+}
+
+// first row of expert e in the expert buffers: e * C_r, or exp_off[e] (dropless)
+__device__ __forceinline__ long long exp_row0(int e, int Cr, const int32_t* exp_off) {
+  return exp_off != nullptr ? static_cast<long long>(exp_off[e]) : static_cast<long long>(e) * Cr;
+}
+
 __global__ void pack_kernel(const uint16_t* __restrict__ z, const int32_t* __restrict__ idx,
                             const int32_t* __restrict__ slot, int T, int k, int dl, int L, int P, int W, int Cs,
-                            int E, uint16_t* __restrict__ pools) {
+                            int E, uint16_t* __restrict__ pools, const int32_t* __restrict__ pool_off) {
   // destination row of each of the token's k assignments, staged per warp in shared
   // memory (no warp shuffle inside the lane-divergent column loop)
   __shared__ long long s_dst[8][32];
@@ -331,7 +347,7 @@ __global__ void pack_kernel(const uint16_t* __restrict__ z, const int32_t* __res
       e_j = idx[static_cast<long long>(t) * k + lane];
       s_j = slot[2LL * (static_cast<long long>(t) * k + lane)];
       const bool ok = s_j >= 0 && s_j < Cs && e_j >= 0 && e_j < E;
-      s_dst[wib][lane] = ok ? (static_cast<long long>(pool_of(e_j, L, P, W)) * Cs + s_j) * row_elems : -1;
+      s_dst[wib][lane] = ok ? (pool_row0(pool_of(e_j, L, P, W), Cs, pool_off) + s_j) * row_elems : -1;
     }
     __syncwarp();
     const uint4* src = reinterpret_cast<const uint4*>(z + static_cast<long long>(t) * dl);
@@ -350,7 +366,7 @@ __global__ void pack_kernel(const uint16_t* __restrict__ z, const int32_t* __res
       }
     }
     if (lane < k && s_j >= 0 && s_j < Cs && e_j >= 0 && e_j < E) {
-      uint16_t* dst = pools + (static_cast<long long>(pool_of(e_j, L, P, W)) * Cs + s_j) * row_elems + dl;
+      uint16_t* dst = pools + (pool_row0(pool_of(e_j, L, P, W), Cs, pool_off) + s_j) * row_elems + dl;
       *reinterpret_cast<int4*>(dst) = make_int4(e_j, 0, 0, 0);
     }
     __syncwarp();
@@ -368,7 +384,7 @@ __global__ void __launch_bounds__(32 * kPackWarps)
     pack_bulk_kernel(const uint16_t* __restrict__ z, const int32_t* __restrict__ idx,
                      const int32_t* __restrict__ slot, int T, int k, int dl, int L, int P, int W, int Cs, int E,
                      const int32_t* __restrict__ pool_fill, int NP, uint16_t* __restrict__ pools,
-                     int32_t* __restrict__ status) {
+                     int32_t* __restrict__ status, const int32_t* __restrict__ pool_off) {
   extern __shared__ __align__(128) uint8_t pack_smem[];
   __shared__ uint64_t s_bar[kPackWarps][2];
   __shared__ long long s_dst[kPackWarps][32];
@@ -401,7 +417,7 @@ __global__ void __launch_bounds__(32 * kPackWarps)
       e_j = idx[static_cast<long long>(t) * k + lane];
       s_j = slot[2LL * (static_cast<long long>(t) * k + lane)];
       ok_j = s_j >= 0 && s_j < Cs && e_j >= 0 && e_j < E;
-      s_dst[wib][lane] = ok_j ? (static_cast<long long>(pool_of(e_j, L, P, W)) * Cs + s_j) * row_elems : -1;
+      s_dst[wib][lane] = ok_j ? (pool_row0(pool_of(e_j, L, P, W), Cs, pool_off) + s_j) * row_elems : -1;
     }
     __syncwarp();
     bool got = true;
@@ -436,8 +452,9 @@ __global__ void __launch_bounds__(32 * kPackWarps)
     if (ok_j) *reinterpret_cast<int4*>(pools + s_dst[wib][lane] + dl) = make_int4(e_j, 0, 0, 0);
     __syncwarp();
   }
-  // header -1 for the rows of each pool past its fill (slots below the fill are dense)
-  const long long n_rows = static_cast<long long>(NP) * Cs;
+  // header -1 for the rows of each pool past its fill (slots below the fill are dense);
+  // packed pools (dropless) have no such rows
+  const long long n_rows = pool_off != nullptr ? 0 : static_cast<long long>(NP) * Cs;
   for (long long rr = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; rr < n_rows;
        rr += static_cast<long long>(gridDim.x) * blockDim.x) {
     const int pl = static_cast<int>(rr / Cs);
@@ -466,7 +483,8 @@ __global__ void pack_empty_headers(const int32_t* __restrict__ pool_fill, int NP
 // (e * C_r + slot) in row_map; other rows map to -1.
 __global__ void unpack_rank_kernel(const uint16_t* __restrict__ pools, int Cs, int Cr, int dl, int L, int P, int W,
                                    int32_t* __restrict__ row_map, int32_t* __restrict__ rows_out,
-                                   int32_t* __restrict__ status) {
+                                   int32_t* __restrict__ status, const int32_t* __restrict__ pool_off,
+                                   const int32_t* __restrict__ pool_fill) {
   constexpr int kTile = 256;
   __shared__ int s_warp_cnt[kTile / 32][32];
   __shared__ int s_run[32];
@@ -477,11 +495,16 @@ __global__ void unpack_rank_kernel(const uint16_t* __restrict__ pools, int Cs, i
   const long long row_elems = dl + 8;
   if (threadIdx.x < 32) s_run[threadIdx.x] = 0;
   __syncthreads();
-  const uint16_t* pbase = pools + static_cast<long long>(pool) * Cs * row_elems;
-  for (int r0 = 0; r0 < Cs; r0 += kTile) {
+  // packed pools (dropless): this pool's rows are the pool_fill[pool] rows at pool_off[pool],
+  // the row map holds the receiver slot and every row is kept
+  const bool packed = pool_off != nullptr;
+  const long long prow0 = pool_row0(pool, Cs, pool_off);
+  const int nrows = packed ? pool_fill[pool] : Cs;
+  const uint16_t* pbase = pools + prow0 * row_elems;
+  for (int r0 = 0; r0 < nrows; r0 += kTile) {
     const int r = r0 + threadIdx.x;
     int q = -1;
-    if (r < Cs) {
+    if (r < nrows) {
       const int e = *reinterpret_cast<const int*>(pbase + r * row_elems + dl);
       if (e >= 0) {
         if (e >= e_first && e < e_first + P) q = e - e_first;
@@ -502,9 +525,8 @@ __global__ void unpack_rank_kernel(const uint16_t* __restrict__ pools, int Cs, i
       for (int w = 0; w < warp; ++w) before += s_warp_cnt[w][q];
       slot = before + rank;
     }
-    if (r < Cs)
-      row_map[static_cast<long long>(pool) * Cs + r] =
-          (slot >= 0 && slot < Cr) ? (e_first + q) * Cr + slot : -1;
+    if (r < nrows)
+      row_map[prow0 + r] = packed ? slot : ((slot >= 0 && slot < Cr) ? (e_first + q) * Cr + slot : -1);
     __syncthreads();
     if (threadIdx.x < P) {
       int tot = 0;
@@ -513,22 +535,28 @@ __global__ void unpack_rank_kernel(const uint16_t* __restrict__ pools, int Cs, i
     }
     __syncthreads();
   }
-  if (threadIdx.x < P) rows_out[e_first + threadIdx.x] = min(s_run[threadIdx.x], Cr);
+  if (threadIdx.x < P) rows_out[e_first + threadIdx.x] = packed ? s_run[threadIdx.x] : min(s_run[threadIdx.x], Cr);
 }
 
 // receiver, pass 2: one warp per pool row, up to 8 vectors per lane in flight
 __global__ void unpack_copy_kernel(const uint16_t* __restrict__ pools, const int32_t* __restrict__ row_map,
-                                   long long n_rows, int dl, uint16_t* __restrict__ xe) {
+                                   long long n_rows, int dl, uint16_t* __restrict__ xe,
+                                   const int32_t* __restrict__ exp_off, int E) {
   const int lane = threadIdx.x & 31;
   const int warps = blockDim.x >> 5;
   const long long row_elems = dl + 8;
   const int nvec = dl / 8;
   for (long long r = static_cast<long long>(blockIdx.x) * warps + (threadIdx.x >> 5); r < n_rows;
        r += static_cast<long long>(gridDim.x) * warps) {
-    const int d = row_map[r];
+    long long d = row_map[r];
     if (d < 0) continue;
+    if (exp_off != nullptr) {  // packed buffers: the row map holds the slot within the expert
+      const int e = *reinterpret_cast<const int*>(pools + r * row_elems + dl);
+      if (e < 0 || e >= E) continue;
+      d += exp_off[e];
+    }
     const uint4* src = reinterpret_cast<const uint4*>(pools + r * row_elems);
-    uint4* dst = reinterpret_cast<uint4*>(xe + static_cast<long long>(d) * dl);
+    uint4* dst = reinterpret_cast<uint4*>(xe + d * dl);
     for (int v0 = lane; v0 < nvec; v0 += 32 * 8) {
       uint4 val[8];
 #pragma unroll
@@ -544,13 +572,14 @@ __global__ void unpack_copy_kernel(const uint16_t* __restrict__ pools, const int
 // rows [n_e, min(round_up(n_e, 128), C_r)) of each expert's buffer become zero, so that
 // the GEMM tiles that cover them read zeros
 __global__ void zero_tail_rows_kernel(uint16_t* __restrict__ buf, long long width, int Cr,
-                                      const int32_t* __restrict__ rows) {
+                                      const int32_t* __restrict__ rows, const int32_t* __restrict__ exp_off) {
   const int e = blockIdx.y;
   const int n = rows[e];
-  const int end = min(((n + 127) / 128) * 128, Cr);
+  // packed buffers (dropless): the expert's region is exactly round_up(n, 128) rows
+  const int end = exp_off != nullptr ? ((n + 127) / 128) * 128 : min(((n + 127) / 128) * 128, Cr);
   const long long nvec = width / 8;
   const long long total = static_cast<long long>(end - n) * nvec;
-  uint4* base = reinterpret_cast<uint4*>(buf + (static_cast<long long>(e) * Cr + n) * width);
+  uint4* base = reinterpret_cast<uint4*>(buf + (exp_row0(e, Cr, exp_off) + n) * width);
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long long>(gridDim.x) * blockDim.x)
     base[i] = make_uint4(0, 0, 0, 0);
@@ -586,7 +615,7 @@ constexpr int kCombRows = 8;
 
 __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ ye, const float* __restrict__ gate,
                                const int32_t* __restrict__ idx, const int32_t* __restrict__ slot, int T, int k,
-                               int dl, int Cr, int E, uint16_t* __restrict__ r) {
+                               int dl, int Cr, int E, uint16_t* __restrict__ r, const int32_t* __restrict__ exp_off) {
   __shared__ long long s_row[8][32];
   __shared__ float s_g[8][32];
   const int lane = threadIdx.x & 31;
@@ -599,7 +628,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
       const int rs = slot[2 * a + 1];
       const int e = idx[a];
       const bool ok = rs >= 0 && rs < Cr && e >= 0 && e < E;
-      s_row[wib][lane] = ok ? static_cast<long long>(e) * Cr + rs : -1;
+      s_row[wib][lane] = ok ? exp_row0(e, Cr, exp_off) + rs : -1;
       s_g[wib][lane] = ok ? gate[a] : 0.0f;
     }
     __syncwarp();
@@ -646,7 +675,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
 __global__ void __launch_bounds__(256) combine_bwd_kernel(const uint16_t* __restrict__ dr, const uint16_t* __restrict__ ye,
                                    const float* __restrict__ gate, const int32_t* __restrict__ idx,
                                    const int32_t* __restrict__ slot, int T, int k, int dl, int Cr, int E,
-                                   uint16_t* __restrict__ dye, float* __restrict__ dg) {
+                                   uint16_t* __restrict__ dye, float* __restrict__ dg,
+                                   const int32_t* __restrict__ exp_off) {
   __shared__ long long s_row[8][32];
   __shared__ float s_g[8][32];
   const int lane = threadIdx.x & 31;
@@ -659,7 +689,7 @@ __global__ void __launch_bounds__(256) combine_bwd_kernel(const uint16_t* __rest
       const int rs = slot[2 * a + 1];
       const int e = idx[a];
       const bool ok = rs >= 0 && rs < Cr && e >= 0 && e < E;
-      s_row[wib][lane] = ok ? static_cast<long long>(e) * Cr + rs : -1;
+      s_row[wib][lane] = ok ? exp_row0(e, Cr, exp_off) + rs : -1;
       s_g[wib][lane] = ok ? gate[a] : 0.0f;
     }
     __syncwarp();
@@ -735,7 +765,8 @@ __global__ void __launch_bounds__(256) combine_bwd_kernel(const uint16_t* __rest
 __global__ void undispatch_kernel(const uint16_t* __restrict__ dxe, const float* __restrict__ gate,
                                   const float* __restrict__ dg, const int32_t* __restrict__ idx,
                                   const int32_t* __restrict__ slot, int T, int k, int dl, int Cr, int E,
-                                  float* __restrict__ dz, uint16_t* __restrict__ dlogits) {
+                                  float* __restrict__ dz, uint16_t* __restrict__ dlogits,
+                                  const int32_t* __restrict__ exp_off) {
   __shared__ long long s_row[8][32];
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
@@ -751,7 +782,7 @@ __global__ void undispatch_kernel(const uint16_t* __restrict__ dxe, const float*
       g_j = gate[a];
       dg_j = dg[a];
       if (e_j < 0 || e_j >= E) e_j = -1;
-      s_row[wib][lane] = (rs >= 0 && rs < Cr && e_j >= 0) ? static_cast<long long>(e_j) * Cr + rs : -1;
+      s_row[wib][lane] = (rs >= 0 && rs < Cr && e_j >= 0) ? exp_row0(e_j, Cr, exp_off) + rs : -1;
     }
     __syncwarp();
     for (int v = lane; v < nvec; v += 64) {
@@ -826,6 +857,42 @@ int blocks_for(long long work, int per_block) {
 
 }  // namespace
 
+// off[i] = sum over j < i of round_up(counts[j], align), for i = 0..n; one block of 1024
+// threads, n <= 1024 (negative counts read as zero)
+__global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict__ counts, int n, int align,
+                                                       int32_t* __restrict__ off) {
+  __shared__ int s_warp[32];
+  const int i = threadIdx.x;
+  const int lane = i & 31, warp = i >> 5;
+  int v = 0;
+  if (i < n) {
+    const int c = counts[i] > 0 ? counts[i] : 0;
+    v = (c + align - 1) / align * align;
+  }
+  int incl = v;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += u;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = s_warp[lane];
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, w, d);
+      if (lane >= d) w += u;
+    }
+    s_warp[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  const int before = warp > 0 ? s_warp[warp - 1] : 0;
+  if (i < n) off[i] = before + incl - v;
+  if (i == n - 1) off[n] = before + incl;
+  if (n == 0 && i == 0) off[0] = 0;
+}
+
 // ====================================================================== launchers
 
 moe_status_t launch_route(const Geo& g, const float* logits, const float* bias, int32_t* idx, float* gate,
@@ -889,7 +956,7 @@ moe_status_t launch_slot_scan(const Geo& g, const int32_t* idx, int32_t* slot, i
 }
 
 moe_status_t launch_pack(const Geo& g, const uint16_t* z, const int32_t* idx, const int32_t* slot,
-                         int32_t* stats, uint16_t* pools, cudaStream_t st) {
+                         int32_t* stats, uint16_t* pools, cudaStream_t st, const int32_t* pool_off) {
   if (g.T > 0) {
     // two row buffers per warp; rows too wide for that take the register path
     const size_t smem = static_cast<size_t>(kPackWarps) * 2 * g.dl * 2;
@@ -906,17 +973,18 @@ moe_status_t launch_pack(const Geo& g, const uint16_t* z, const int32_t* idx, co
       const int grid = static_cast<int>(std::min<long long>((g.T + kPackWarps - 1) / kPackWarps,
                                                             static_cast<long long>(device_sm_count()) * per_sm));
       pack_bulk_kernel<<<grid, 32 * kPackWarps, smem, st>>>(z, idx, slot, g.T, g.k, g.dl, g.L, g.P, g.W, g.Cs, g.E,
-                                                            stats + stats_pool_fill(g), g.NP, pools, stats + 3);
+                                                            stats + stats_pool_fill(g), g.NP, pools, stats + 3,
+                                                            pool_off);
       count_launch();
       return cuda_check(cudaGetLastError(), "pack");
     } else {
       const int warps = 8;
       pack_kernel<<<blocks_for(g.T, warps), 32 * warps, 0, st>>>(z, idx, slot, g.T, g.k, g.dl, g.L, g.P, g.W, g.Cs,
-                                                                 g.E, pools);
+                                                                 g.E, pools, pool_off);
     }
     count_launch();
   }
-  const long long rows = static_cast<long long>(g.NP) * g.Cs;
+  const long long rows = pool_off != nullptr ? 0 : static_cast<long long>(g.NP) * g.Cs;
   if (rows > 0)
   {
     pack_empty_headers<<<blocks_for(rows, 256), 256, 0, st>>>(stats + stats_pool_fill(g), g.NP, g.Cs, g.dl, pools);
@@ -925,54 +993,70 @@ moe_status_t launch_pack(const Geo& g, const uint16_t* z, const int32_t* idx, co
   return cuda_check(cudaGetLastError(), "pack");
 }
 
-size_t unpack_scratch_ints(const Geo& g) { return static_cast<size_t>(g.NP) * g.Cs; }
+size_t unpack_scratch_ints(const Geo& g) { return static_cast<size_t>(g.pool_rows); }
+
+moe_status_t launch_offsets(const int32_t* counts, int n, int align, int32_t* off, cudaStream_t st) {
+  if (n < 0 || n > 1024 || align < 1) return fail(MOE_ERR_UNSUPPORTED, "offsets over at most 1024 counts");
+  offsets_kernel<<<1, 1024, 0, st>>>(counts, n, align, off);
+  count_launch();
+  return cuda_check(cudaGetLastError(), "offsets");
+}
 
 moe_status_t launch_unpack(const Geo& g, const uint16_t* pools, uint16_t* xe, int32_t* rows, int32_t* row_map,
-                           int32_t* status, cudaStream_t st) {
+                           int32_t* status, cudaStream_t st, const int32_t* pool_off, const int32_t* pool_fill,
+                           int32_t* exp_off) {
   if (g.P > 32) return fail(MOE_ERR_UNSUPPORTED, "more than 32 experts per wave");
-  unpack_rank_kernel<<<g.NP, 256, 0, st>>>(pools, g.Cs, g.Cr, g.dl, g.L, g.P, g.W, row_map, rows, status);
-  const long long n_rows = static_cast<long long>(g.NP) * g.Cs;
+  const bool packed = pool_off != nullptr;
+  if (packed && (pool_fill == nullptr || exp_off == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "packed pools need their fills and the expert offsets");
+  unpack_rank_kernel<<<g.NP, 256, 0, st>>>(pools, g.Cs, g.Cr, g.dl, g.L, g.P, g.W, row_map, rows, status, pool_off,
+                                           pool_fill);
+  count_launch();
+  if (packed) MOE_TRY_K(launch_offsets(rows, g.E, 128, exp_off, st));
+  const long long n_rows = g.pool_rows;
   const int warps = 8;
-  unpack_copy_kernel<<<blocks_for(n_rows, warps), 32 * warps, 0, st>>>(pools, row_map, n_rows, g.dl, xe);
-  count_launch(2);
+  unpack_copy_kernel<<<blocks_for(n_rows, warps), 32 * warps, 0, st>>>(pools, row_map, n_rows, g.dl, xe,
+                                                                       packed ? exp_off : nullptr, g.E);
+  count_launch();
   return cuda_check(cudaGetLastError(), "unpack");
 }
 
 moe_status_t launch_zero_tail_rows(const Geo& g, uint16_t* buf, int64_t width, const int32_t* rows,
-                                   cudaStream_t st) {
+                                   cudaStream_t st, const int32_t* exp_off) {
   dim3 grid(4, g.E);
-  zero_tail_rows_kernel<<<grid, 256, 0, st>>>(buf, width, g.Cr, rows);
+  zero_tail_rows_kernel<<<grid, 256, 0, st>>>(buf, width, g.Cr, rows, exp_off);
   count_launch();
   return cuda_check(cudaGetLastError(), "zero tail rows");
 }
 
 moe_status_t launch_combine(const Geo& g, const uint16_t* ye, const float* gate, const int32_t* idx,
-                            const int32_t* slot, uint16_t* r, cudaStream_t st) {
+                            const int32_t* slot, uint16_t* r, cudaStream_t st, const int32_t* exp_off) {
   if (g.T == 0) return MOE_OK;
   const int warps = 8;
-  combine_kernel<<<blocks_for(g.T, warps), 32 * warps, 0, st>>>(ye, gate, idx, slot, g.T, g.k, g.dl, g.Cr, g.E, r);
+  combine_kernel<<<blocks_for(g.T, warps), 32 * warps, 0, st>>>(ye, gate, idx, slot, g.T, g.k, g.dl, g.Cr, g.E, r,
+                                                                exp_off);
   count_launch();
   return cuda_check(cudaGetLastError(), "combine");
 }
 
 moe_status_t launch_combine_bwd(const Geo& g, const uint16_t* dr, const uint16_t* ye, const float* gate,
                                 const int32_t* idx, const int32_t* slot, uint16_t* dye, float* dg,
-                                cudaStream_t st) {
+                                cudaStream_t st, const int32_t* exp_off) {
   if (g.T == 0) return MOE_OK;
   const int warps = 8;
   combine_bwd_kernel<<<blocks_for(g.T, warps), 32 * warps, 0, st>>>(dr, ye, gate, idx, slot, g.T, g.k, g.dl,
-                                                                    g.Cr, g.E, dye, dg);
+                                                                    g.Cr, g.E, dye, dg, exp_off);
   count_launch();
   return cuda_check(cudaGetLastError(), "combine_bwd");
 }
 
 moe_status_t launch_undispatch(const Geo& g, const uint16_t* dxe, const float* gate, const float* dg,
                                const int32_t* idx, const int32_t* slot, float* dz_routed, uint16_t* dlogits,
-                               cudaStream_t st) {
+                               cudaStream_t st, const int32_t* exp_off) {
   if (g.T == 0) return MOE_OK;
   const int warps = 8;
   undispatch_kernel<<<blocks_for(g.T, warps), 32 * warps, 0, st>>>(dxe, gate, dg, idx, slot, g.T, g.k, g.dl, g.Cr,
-                                                                   g.E, dz_routed, dlogits);
+                                                                   g.E, dz_routed, dlogits, exp_off);
   count_launch();
   return cuda_check(cudaGetLastError(), "undispatch");
 }

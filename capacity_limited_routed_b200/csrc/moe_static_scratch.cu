@@ -56,6 +56,8 @@ extern "C" moe_status_t moe_dispatch_noalloc(moe_plan_t plan, const uint16_t* z,
                                              uint16_t* pools, int32_t* slot, void* stats, void* stream) {
   if (plan == nullptr) return fail(MOE_ERR_INVALID_ARG, "null plan");
   const Geo& g = plan_geo(plan);
+  if (g.dropless)
+    return fail(MOE_ERR_UNSUPPORTED, "moe_dispatch_noalloc: the dropless variant runs through moe_forward only");
   if (!pools || !stats) return fail(MOE_ERR_INVALID_ARG, "null buffer");
   if (g.T > 0 && (!z || !topk_idx || !slot)) return fail(MOE_ERR_INVALID_ARG, "null buffer");
   if ((reinterpret_cast<uintptr_t>(z) & 15) || (reinterpret_cast<uintptr_t>(pools) & 15))

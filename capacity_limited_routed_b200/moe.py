@@ -164,8 +164,10 @@ class Plan:
 
     @classmethod
     def from_shape(cls, s):
+        # both capacity numerators 0 select the dropless variant
+        cap_send, cap_recv = ((0, 1), (0, 1)) if getattr(s, "dropless", False) else (s.cap_send, s.cap_recv)
         return cls(s.T, s.d_model, s.d_latent, s.n_experts, s.top_k, s.n_dest, s.hidden_routed, s.n_shared,
-                   s.hidden_shared, s.n_waves, s.cap_send, s.cap_recv)
+                   s.hidden_shared, s.n_waves, cap_send, cap_recv)
 
     def __del__(self):
         h = getattr(self, "handle", None)

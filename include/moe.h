@@ -82,6 +82,14 @@ typedef struct {
   int32_t hidden_shared;  /* hidden width of a shared expert (3072) */
   int32_t cap_send_num, cap_send_den;  /* sender factor, 110/100 */
   int32_t cap_recv_num, cap_recv_den;  /* receiver factor, 115/100 */
+  /* cap_send_num = cap_recv_num = 0 selects the dropless variant ("Marin 535B-A23B"
+   * page on ranhao.site, §3.3 token dropping and §7: the run later switched to a
+   * dropless ragged all-to-all): no cap binds, every assignment is kept.  Pools are
+   * then packed back to back in pool order (T*k rows in all) and the expert buffers
+   * by expert, each expert's rows padded to a multiple of 128 (T*k + 127*E rows);
+   * moe_plan_info reports cap_send = cap_recv = 0 and those sizes.  The dropless
+   * variant runs through moe_forward / moe_backward; moe_dispatch, moe_expert_ffn,
+   * moe_combine and moe_dispatch_noalloc return MOE_ERR_UNSUPPORTED for it. */
 } moe_config_t;
 
 typedef struct moe_plan* moe_plan_t;
@@ -91,11 +99,11 @@ typedef struct {
   int32_t local_experts;     /* L = E / D */
   int32_t experts_per_wave;  /* P = L / W */
   int32_t n_pools;           /* D * W */
-  int32_t cap_send;          /* C_s, rows of one pool */
-  int32_t cap_recv;          /* C_r, rows of one expert */
+  int32_t cap_send;          /* C_s, rows of one pool (0: dropless) */
+  int32_t cap_recv;          /* C_r, rows of one expert (0: dropless) */
   int32_t pool_row_elems;    /* bf16 elements per pool row: d_latent payload + 8 header */
-  uint64_t pools_bytes;      /* [D*W][C_s][pool_row_elems] bf16 */
-  uint64_t expert_out_bytes; /* [E][C_r][d_latent] bf16 */
+  uint64_t pools_bytes;      /* [D*W][C_s][pool_row_elems] bf16 (dropless: [T*k][...]) */
+  uint64_t expert_out_bytes; /* [E][C_r][d_latent] bf16 (dropless: [T*k + 127*E][...]) */
   uint64_t slot_bytes;       /* [T][k][2] int32 */
   uint64_t stats_bytes;      /* moe_stats_t + per-expert and per-pool counters */
   uint64_t saved_bytes;      /* forward context for moe_backward */

@@ -101,3 +101,18 @@ def test_null_arguments_are_rejected(M):
     fake = ctypes.c_void_p(0x1000)
     # too-small workspace is reported before anything runs
     assert lib.moe_dispatch(p.handle, fake, fake, fake, fake, fake, fake, 16, None) == 3
+
+
+def test_dropless_plan_sizes(M):
+    """Both capacity numerators 0 select the dropless variant: no caps, pools packed to
+    T*k rows, expert buffers packed by expert with each expert padded to 128 rows."""
+    T, k, E, dl = 300, 3, 24, 64
+    p = M.Plan(T=T, d_model=128, d_latent=dl, n_experts=E, top_k=k, n_dest=4, hidden_routed=128,
+               n_shared=1, hidden_shared=128, cap_send=(0, 1), cap_recv=(0, 1))
+    assert p.info.cap_send == 0 and p.info.cap_recv == 0
+    assert p.info.pools_bytes == T * k * (dl + 8) * 2
+    assert p.info.expert_out_bytes == (T * k + 127 * E) * dl * 2
+    # only one numerator 0 is an error, as before
+    with pytest.raises(M.MoEError):
+        M.Plan(T=T, d_model=128, d_latent=dl, n_experts=E, top_k=k, n_dest=4, hidden_routed=128,
+               n_shared=1, hidden_shared=128, cap_send=(0, 1))
