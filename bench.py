@@ -40,8 +40,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # captured ones, and as null once they change.
 NCU_TRAFFIC = {
     "bwd.experts_wgrad_gate_up": {
-        "sources_sha256": "15b9e7cfe34c2cad2e1facb33c0599eb3b11f831afd58701fb04566102d9a00a",
-        "dram_bytes": 1917372160, "experts": 24, "tokens": 1024, "d_latent": 3072, "hidden_routed": 3072,
+        "sources_sha256": "9cd110a0465c274519fea7062452e09f82d70046afab58915fa840b1022a4aea",
+        "dram_bytes": 1918638848, "experts": 24, "tokens": 1024, "d_latent": 3072, "hidden_routed": 3072,
     },
 }
 KERNEL_SOURCES = ("gemm_sm100.cu", "ptx.cuh", "internal.h")
