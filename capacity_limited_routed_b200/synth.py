@@ -48,6 +48,7 @@ class MoEShape:
     cap_send: tuple = (110, 100)
     cap_recv: tuple = (115, 100)
     dropless: bool = False       # no cap binds: every assignment kept (ragged buffers)
+    n_sources: int = 1           # T splits into this many sources with their own sender pools
     # workload-only knobs (input recipe, not part of the block)
     zipf_s: float = 0.0          # >0: per-expert logit skew with Zipf(s) expected load
     window: int = 0              # >0: tokens in windows of this size share a component

@@ -120,11 +120,14 @@ class Geometry:
     W: int
     L: int        # local experts per destination
     P: int        # experts per wave
-    C_s: int      # sender capacity of one (destination, wave) pool
+    C_s: int      # sender capacity of one (destination, wave) pool of one source
     C_r: int      # receiver capacity of one expert
+    S: int = 1    # sources: T splits into S equal contiguous token ranges, each sending
+                  # its own pools with its own sender caps (as each GPU does under EP)
 
     @property
     def n_pools(self) -> int:
+        """(destination, wave) pools of one source."""
         return self.D * self.W
 
 
@@ -134,15 +137,16 @@ def ceil_ratio(a: int, b: int) -> int:
 
 
 def capacities(T: int, k: int, E: int, D: int, W: int,
-               cap_send=(110, 100), cap_recv=(115, 100)) -> tuple[int, int]:
+               cap_send=(110, 100), cap_recv=(115, 100), S: int = 1) -> tuple[int, int]:
     """Sender and receiver capacities ([RU] §2: factors 1.10 and 1.15).
 
-    Expected rows per (destination, wave) pool from one source are T*k/(D*W); per
-    expert T*k/E.  Each is scaled by its factor num/den and rounded up exactly.
+    Expected rows per (destination, wave) pool from one source of T/S tokens are
+    (T/S)*k/(D*W); per expert (all sources together) T*k/E.  Each is scaled by its
+    factor num/den and rounded up exactly.
     """
     ns, ds = cap_send
     nr, dr = cap_recv
-    C_s = ceil_ratio(T * k * ns, ds * D * W)
+    C_s = ceil_ratio(T * k * ns, ds * D * W * S)
     C_r = ceil_ratio(T * k * nr, dr * E)
     return C_s, C_r
 
@@ -153,8 +157,19 @@ def geometry(shape) -> Geometry:
     if E % D or (E // D) % W:
         raise ValueError("E must split into D destinations of W equal waves")
     L = E // D
-    C_s, C_r = capacities(shape.T, shape.top_k, E, D, W, shape.cap_send, shape.cap_recv)
-    return Geometry(T=shape.T, E=E, k=shape.top_k, D=D, W=W, L=L, P=L // W, C_s=C_s, C_r=C_r)
+    S = getattr(shape, "n_sources", 1)
+    if S < 1 or shape.T % S:
+        raise ValueError("T must split into S equal sources")
+    C_s, C_r = capacities(shape.T, shape.top_k, E, D, W, shape.cap_send, shape.cap_recv, S)
+    return Geometry(T=shape.T, E=E, k=shape.top_k, D=D, W=W, L=L, P=L // W, C_s=C_s, C_r=C_r, S=S)
+
+
+def source_pool(g: Geometry, idx: np.ndarray) -> np.ndarray:
+    """Pool of every assignment of idx [T][k] across sources: source * (D*W) + pool, where
+    the source of token t is t // (T/S)."""
+    idx = np.asarray(idx)
+    src = np.arange(idx.shape[0]) // (idx.shape[0] // g.S) if g.S > 1 else np.zeros(idx.shape[0], np.int64)
+    return src[:, None] * g.n_pools + placement(g)["pool"][idx]
 
 
 def dropless_geometry(g: Geometry, idx: np.ndarray) -> Geometry:
@@ -166,10 +181,10 @@ def dropless_geometry(g: Geometry, idx: np.ndarray) -> Geometry:
     itself, so those two numbers serve as the capacities: every assignment is kept,
     every pool and expert holds exactly its load.
     """
-    pool = placement(g)["pool"][np.asarray(idx)]
-    C_s = int(np.bincount(pool.ravel(), minlength=g.n_pools).max()) if pool.size else 0
+    pool = source_pool(g, idx)
+    C_s = int(np.bincount(pool.ravel(), minlength=g.S * g.n_pools).max()) if pool.size else 0
     C_r = int(np.bincount(np.asarray(idx).ravel(), minlength=g.E).max()) if pool.size else 0
-    return Geometry(T=g.T, E=g.E, k=g.k, D=g.D, W=g.W, L=g.L, P=g.P, C_s=max(C_s, 1), C_r=max(C_r, 1))
+    return Geometry(T=g.T, E=g.E, k=g.k, D=g.D, W=g.W, L=g.L, P=g.P, C_s=max(C_s, 1), C_r=max(C_r, 1), S=g.S)
 
 
 def placement(g: Geometry) -> dict:
@@ -243,16 +258,17 @@ def _running_rank(keys: np.ndarray, valid: np.ndarray) -> np.ndarray:
 def assign_slots(idx: np.ndarray, g: Geometry) -> dict:
     """Sender and receiver slots of every assignment, visited in (token, rank) order.
 
-    sslot[t][j]: position in pool(e) among this source's assignments to that pool,
-                 or -1 when it is at or past C_s (sender drop).
+    sslot[t][j]: position in pool(e) among the assignments of t's source to that
+                 pool, or -1 when it is at or past C_s (sender drop).
     rslot[t][j]: position among the sender-kept assignments of expert e, or -1 when
                  it was sender-dropped or is at or past C_r (receiver drop).
     Also returns the counters: kept, dropped_sender, dropped_receiver, per-expert
-    kept / sender-dropped / receiver-dropped, and the fill of every pool.
+    kept / sender-dropped / receiver-dropped, and the fill of every pool (source-major,
+    S * D * W pools).  The receiver sees a pool group's sources in order, so its
+    (token, rank) visiting order is the global one.
     """
-    pl = placement(g)
     e = np.asarray(idx, dtype=np.int64).ravel()
-    pool = pl["pool"][e]
+    pool = source_pool(g, idx).ravel()                  # one set of pools per source
     srank = _running_rank(pool, np.ones(e.size, dtype=bool))
     skept = srank < g.C_s
     rrank = _running_rank(e, skept)
@@ -264,7 +280,7 @@ def assign_slots(idx: np.ndarray, g: Geometry) -> dict:
     per_kept = np.bincount(e[rkept], minlength=g.E)
     per_ds = np.bincount(e[drop_s], minlength=g.E)
     per_dr = np.bincount(e[drop_r], minlength=g.E)
-    fill = np.bincount(pool[skept], minlength=g.n_pools)
+    fill = np.bincount(pool[skept], minlength=g.S * g.n_pools)
     return {
         "sslot": sslot.reshape(idx.shape).astype(np.int32),
         "rslot": rslot.reshape(idx.shape).astype(np.int32),
@@ -284,16 +300,16 @@ def pack_pools(z: np.ndarray, idx: np.ndarray, sslot: np.ndarray, g: Geometry):
     Returns (payload [D*W][C_s][d_l], header [D*W][C_s] int32): the header of a row
     holds the global expert id of the assignment stored there, -1 for an empty row.
     """
-    pl = placement(g)
     d_l = z.shape[1]
-    payload = np.zeros((g.n_pools, g.C_s, d_l), dtype=z.dtype)
-    header = np.full((g.n_pools, g.C_s), -1, dtype=np.int32)
+    payload = np.zeros((g.S * g.n_pools, g.C_s, d_l), dtype=z.dtype)
+    header = np.full((g.S * g.n_pools, g.C_s), -1, dtype=np.int32)
+    spool = source_pool(g, idx)
     T, k = idx.shape
     for t in range(T):
         for j in range(k):
             s = sslot[t, j]
             if s >= 0:
-                p = pl["pool"][idx[t, j]]
+                p = spool[t, j]
                 payload[p, s] = z[t]
                 header[p, s] = idx[t, j]
     return payload, header
@@ -302,17 +318,20 @@ def pack_pools(z: np.ndarray, idx: np.ndarray, sslot: np.ndarray, g: Geometry):
 def receive(payload: np.ndarray, header: np.ndarray, g: Geometry):
     """Receiver side: unpack each pool by the expert id in its rows.
 
-    Rows of one pool are visited in pool order; each local expert keeps its first
-    C_r rows.  Returns (rows [E] list of [n_e][d_l] arrays, counts [E]), the rows
+    The receiver of a (destination, wave) takes the pools that every source sent it,
+    sources in order, rows of each pool in pool order; each local expert keeps its
+    first C_r rows.  Returns (rows [E] list of [n_e][d_l] arrays, counts [E]), the rows
     in receiver-slot order.  Uses nothing but the pools themselves.
     """
     d_l = payload.shape[2]
     buckets = [[] for _ in range(g.E)]
     for p in range(g.n_pools):
-        for s in range(g.C_s):
-            e = int(header[p, s])
-            if e >= 0 and len(buckets[e]) < g.C_r:
-                buckets[e].append(payload[p, s])
+        for src in range(g.S):
+            q = src * g.n_pools + p
+            for s in range(g.C_s):
+                e = int(header[q, s])
+                if e >= 0 and len(buckets[e]) < g.C_r:
+                    buckets[e].append(payload[q, s])
     rows = [np.array(b, dtype=payload.dtype).reshape(len(b), d_l) for b in buckets]
     return rows, np.array([r.shape[0] for r in rows], dtype=np.int64)
 
