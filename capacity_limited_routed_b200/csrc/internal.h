@@ -100,6 +100,10 @@ int device_sm_count();
 struct Geo {
   int T, E, k, D, W, L, P, NP, Cs, Cr, dl;
   int n_chunks;      // token chunks of the slot scan
+  // virtual sources: T splits into S equal token ranges of Ts tokens (whole scan chunks),
+  // each with its own D*W pools (NP of them) and sender caps; NPS = S * NP pools in all,
+  // source-major.  S = 1 is one source.
+  int S, Ts, NPS;
   // dropless variant: no cap binds (Cs = Cr = T*k); pools are packed back to back in
   // pool order (pool_rows = T*k rows) and expert buffers by expert, each expert's
   // region padded to a multiple of 128 rows (exp_rows = T*k + 127*E rows)
@@ -117,7 +121,7 @@ moe_status_t launch_slot_scan(const Geo& g, const int32_t* idx, int32_t* slot, i
                               cudaStream_t st);
 moe_status_t launch_pack(const Geo& g, const uint16_t* z, const int32_t* idx, const int32_t* slot,
                          int32_t* stats, uint16_t* pools, cudaStream_t st, const int32_t* pool_off = nullptr);
-// off[i] = sum over j < i of round_up(counts[j], align), i = 0..n (n <= 1024)
+// off[i] = sum over j < i of round_up(counts[j], align), i = 0..n
 moe_status_t launch_offsets(const int32_t* counts, int n, int align, int32_t* off, cudaStream_t st);
 // scratch ints needed by the receiver's row map
 size_t unpack_scratch_ints(const Geo& g);
@@ -151,6 +155,6 @@ inline int stats_kept_e(const Geo& g) { return kStatsHead + g.E; }
 inline int stats_ds_e(const Geo& g) { return kStatsHead + 2 * g.E; }
 inline int stats_dr_e(const Geo& g) { return kStatsHead + 3 * g.E; }
 inline int stats_pool_fill(const Geo& g) { return kStatsHead + 4 * g.E; }
-inline int stats_words(const Geo& g) { return kStatsHead + 4 * g.E + g.NP; }
+inline int stats_words(const Geo& g) { return kStatsHead + 4 * g.E + g.NPS; }
 
 }  // namespace moe

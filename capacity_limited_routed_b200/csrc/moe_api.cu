@@ -142,7 +142,7 @@ void layout_ctx(const moe_plan& p, bool training, moe_plan::Ctx& c) {
   c.bs = training ? take(off, T * SH * 2) : 0;
   c.hsh = take(off, T * SH * 2);
   c.exp_off = take(off, (E + 1) * 4);
-  c.pool_off = take(off, (size_t(p.g.NP) + 1) * 4);
+  c.pool_off = take(off, (size_t(p.g.NPS) + 1) * 4);
   c.bytes = (off + kAlign - 1) / kAlign * kAlign;
 }
 
@@ -406,6 +406,12 @@ moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out) {
   if (L / c.n_waves > 32) return fail(MOE_ERR_UNSUPPORTED, "at most 32 experts per wave");
   const int64_t A = int64_t(c.T) * c.top_k;
   if (A > (int64_t(1) << 30)) return fail(MOE_ERR_UNSUPPORTED, "T * top_k too large");
+  // virtual sources (0 reads as 1): each source's tokens are whole chunks of the slot scan
+  const int S = c.n_sources > 0 ? c.n_sources : 1;
+  if (c.n_sources < 0) return fail(MOE_ERR_INVALID_ARG, "n_sources must be >= 0");
+  if (S > 1 && (c.T % S != 0 || (c.T / S) % kScanTokensPerChunk != 0))
+    return fail(MOE_ERR_UNSUPPORTED, "with several sources T/S must be a multiple of " +
+                                         std::to_string(kScanTokensPerChunk));
   moe_plan* p = new moe_plan();
   std::memset(static_cast<void*>(p), 0, sizeof(*p));
   p->cfg = c;
@@ -425,6 +431,9 @@ moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out) {
   g.L = L;
   g.P = L / c.n_waves;
   g.NP = c.n_dest * c.n_waves;
+  g.S = S;
+  g.Ts = S > 1 ? c.T / S : (c.T > 0 ? c.T : 1);
+  g.NPS = S * g.NP;
   g.dropless = dropless;
   if (dropless) {
     // no slot reaches T*k, so no cap binds; buffers are packed (see Geo)
@@ -432,11 +441,12 @@ moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out) {
     g.pool_rows = A;
     g.exp_rows = A + int64_t(127) * c.n_experts;
   } else {
-    g.Cs = ceil_cap(A, int64_t(c.n_dest) * c.n_waves, c.cap_send_num, c.cap_send_den);
+    // a source's pool expects (T/S)*k/(D*W) rows
+    g.Cs = ceil_cap(A, int64_t(c.n_dest) * c.n_waves * S, c.cap_send_num, c.cap_send_den);
     g.Cr = ceil_cap(A, c.n_experts, c.cap_recv_num, c.cap_recv_den);
     if (g.Cs < 1) g.Cs = 1;
     if (g.Cr < 1) g.Cr = 1;
-    g.pool_rows = int64_t(g.NP) * g.Cs;
+    g.pool_rows = int64_t(g.NPS) * g.Cs;
     g.exp_rows = int64_t(c.n_experts) * g.Cr;
   }
   g.dl = c.d_latent;
@@ -456,7 +466,7 @@ moe_status_t moe_plan_info(moe_plan_t p, moe_plan_info_t* out) {
   if (p == nullptr || out == nullptr) return fail(MOE_ERR_INVALID_ARG, "null argument");
   out->local_experts = p->g.L;
   out->experts_per_wave = p->g.P;
-  out->n_pools = p->g.NP;
+  out->n_pools = p->g.NPS;  // every source's D*W pools, source-major
   out->cap_send = p->g.dropless ? 0 : p->g.Cs;  // 0: no cap (dropless)
   out->cap_recv = p->g.dropless ? 0 : p->g.Cr;
   out->pool_row_elems = p->dl + 8;
@@ -606,7 +616,7 @@ moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const uint16_t* x
   int32_t* exp_off = g.dropless ? c.exp_off : nullptr;
   {
     ProfScope ps("fwd.dispatch_pack", st);
-    if (g.dropless) MOE_TRY(launch_offsets(s + stats_pool_fill(g), g.NP, 1, pool_off, st));
+    if (g.dropless) MOE_TRY(launch_offsets(s + stats_pool_fill(g), g.NPS, 1, pool_off, st));
     MOE_TRY(launch_pack(g, c.z, c.idx, c.slot, s, pools, st, pool_off));
   }
   MOE_TRY(run_experts(*p, w->w1, w->w3, w->w2, pools, c.xe, c.rows, at<int32_t>(ws, p->ws_rowmap), c.ae, c.be,

@@ -164,19 +164,22 @@ __global__ void scan_count_pools(const int32_t* __restrict__ idx, int A_total, i
   for (int p = threadIdx.x; p < NP; p += blockDim.x) cnt_pool[static_cast<long long>(p) * n_chunks + c] = sh[p];
 }
 
-// exclusive scan of each row of a [rows][n] int array, one block per row; writes the
-// row total to totals[row] (optional), clamped at cap into clamp_out[row] (optional)
+// exclusive scan of each row of a [rows][n] int array, one block per row, restarted every
+// seg elements (seg divides n; seg = n: one segment).  Segment s of row r: its total goes
+// to totals[s * rows + r] (optional), clamped at cap into clamp_out[s * rows + r] (optional).
 __global__ void scan_rows(int32_t* __restrict__ data, int n, int32_t* __restrict__ totals, int cap,
-                          int32_t* __restrict__ clamp_out) {
+                          int32_t* __restrict__ clamp_out, int seg) {
   __shared__ int warp_tot[32];
   __shared__ int carry;
   int32_t* row = data + static_cast<long long>(blockIdx.x) * n;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
+  for (int s0 = 0; s0 < n; s0 += seg) {
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
-  for (int base = 0; base < n; base += blockDim.x) {
+  const int s1 = min(n, s0 + seg);
+  for (int base = s0; base < s1; base += blockDim.x) {
     const int i = base + threadIdx.x;
-    const int v = i < n ? row[i] : 0;
+    const int v = i < s1 ? row[i] : 0;
     int incl = v;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -187,15 +190,18 @@ __global__ void scan_rows(int32_t* __restrict__ data, int n, int32_t* __restrict
     __syncthreads();
     int before = carry;
     for (int w = 0; w < warp; ++w) before += warp_tot[w];
-    if (i < n) row[i] = before + incl - v;
+    if (i < s1) row[i] = before + incl - v;
     __syncthreads();
     if (threadIdx.x == blockDim.x - 1) carry = before + incl;
     __syncthreads();
     (void)nwarp;
   }
   if (threadIdx.x == 0) {
-    if (totals) totals[blockIdx.x] = carry;
-    if (clamp_out) clamp_out[blockIdx.x] = carry < cap ? carry : cap;
+    const long long o = static_cast<long long>(s0 / seg) * gridDim.x + blockIdx.x;
+    if (totals) totals[o] = carry;
+    if (clamp_out) clamp_out[o] = carry < cap ? carry : cap;
+  }
+  __syncthreads();
   }
 }
 
@@ -320,6 +326,12 @@ __global__ void scan_totals(int32_t* __restrict__ stats, int E, int NP, int A_to
 // ---------------------------------------------------------------------- pack / unpack
 
 // one warp per token: read z_t once, write it into every pool row it was given
+// pool of assignment (token t, expert e) across sources: source t / Ts owns the NP pools
+// [source * NP, source * NP + NP), source-major
+__device__ __forceinline__ int src_pool(int t, int Ts, int NP, int e, int L, int P, int W) {
+  return (t / Ts) * NP + pool_of(e, L, P, W);
+}
+
 // first row of pool p: fixed-size pools at p * C_s, packed pools (dropless) at pool_off[p]
 __device__ __forceinline__ long long pool_row0(int p, int Cs, const int32_t* pool_off) {
   return pool_off != nullptr ? static_cast<long long>(pool_off[p]) : static_cast<long long>(p) * Cs;
@@ -332,7 +344,8 @@ __device__ __forceinline__ long long exp_row0(int e, int Cr, const int32_t* exp_
 
 __global__ void pack_kernel(const uint16_t* __restrict__ z, const int32_t* __restrict__ idx,
                             const int32_t* __restrict__ slot, int T, int k, int dl, int L, int P, int W, int Cs,
-                            int E, uint16_t* __restrict__ pools, const int32_t* __restrict__ pool_off) {
+                            int E, uint16_t* __restrict__ pools, const int32_t* __restrict__ pool_off, int Ts,
+                            int NPsrc) {
   // destination row of each of the token's k assignments, staged per warp in shared
   // memory (no warp shuffle inside the lane-divergent column loop)
   __shared__ long long s_dst[8][32];
@@ -347,7 +360,7 @@ __global__ void pack_kernel(const uint16_t* __restrict__ z, const int32_t* __res
       e_j = idx[static_cast<long long>(t) * k + lane];
       s_j = slot[2LL * (static_cast<long long>(t) * k + lane)];
       const bool ok = s_j >= 0 && s_j < Cs && e_j >= 0 && e_j < E;
-      s_dst[wib][lane] = ok ? (pool_row0(pool_of(e_j, L, P, W), Cs, pool_off) + s_j) * row_elems : -1;
+      s_dst[wib][lane] = ok ? (pool_row0(src_pool(t, Ts, NPsrc, e_j, L, P, W), Cs, pool_off) + s_j) * row_elems : -1;
     }
     __syncwarp();
     const uint4* src = reinterpret_cast<const uint4*>(z + static_cast<long long>(t) * dl);
@@ -366,7 +379,7 @@ __global__ void pack_kernel(const uint16_t* __restrict__ z, const int32_t* __res
       }
     }
     if (lane < k && s_j >= 0 && s_j < Cs && e_j >= 0 && e_j < E) {
-      uint16_t* dst = pools + (pool_row0(pool_of(e_j, L, P, W), Cs, pool_off) + s_j) * row_elems + dl;
+      uint16_t* dst = pools + (pool_row0(src_pool(t, Ts, NPsrc, e_j, L, P, W), Cs, pool_off) + s_j) * row_elems + dl;
       *reinterpret_cast<int4*>(dst) = make_int4(e_j, 0, 0, 0);
     }
     __syncwarp();
@@ -384,7 +397,7 @@ __global__ void __launch_bounds__(32 * kPackWarps)
     pack_bulk_kernel(const uint16_t* __restrict__ z, const int32_t* __restrict__ idx,
                      const int32_t* __restrict__ slot, int T, int k, int dl, int L, int P, int W, int Cs, int E,
                      const int32_t* __restrict__ pool_fill, int NP, uint16_t* __restrict__ pools,
-                     int32_t* __restrict__ status, const int32_t* __restrict__ pool_off) {
+                     int32_t* __restrict__ status, const int32_t* __restrict__ pool_off, int Ts, int NPsrc) {
   extern __shared__ __align__(128) uint8_t pack_smem[];
   __shared__ uint64_t s_bar[kPackWarps][2];
   __shared__ long long s_dst[kPackWarps][32];
@@ -417,7 +430,7 @@ __global__ void __launch_bounds__(32 * kPackWarps)
       e_j = idx[static_cast<long long>(t) * k + lane];
       s_j = slot[2LL * (static_cast<long long>(t) * k + lane)];
       ok_j = s_j >= 0 && s_j < Cs && e_j >= 0 && e_j < E;
-      s_dst[wib][lane] = ok_j ? (pool_row0(pool_of(e_j, L, P, W), Cs, pool_off) + s_j) * row_elems : -1;
+      s_dst[wib][lane] = ok_j ? (pool_row0(src_pool(t, Ts, NPsrc, e_j, L, P, W), Cs, pool_off) + s_j) * row_elems : -1;
     }
     __syncwarp();
     bool got = true;
@@ -484,11 +497,12 @@ __global__ void pack_empty_headers(const int32_t* __restrict__ pool_fill, int NP
 __global__ void unpack_rank_kernel(const uint16_t* __restrict__ pools, int Cs, int Cr, int dl, int L, int P, int W,
                                    int32_t* __restrict__ row_map, int32_t* __restrict__ rows_out,
                                    int32_t* __restrict__ status, const int32_t* __restrict__ pool_off,
-                                   const int32_t* __restrict__ pool_fill) {
+                                   const int32_t* __restrict__ pool_fill, int S) {
   constexpr int kTile = 256;
   __shared__ int s_warp_cnt[kTile / 32][32];
   __shared__ int s_run[32];
-  const int pool = blockIdx.x;
+  const int pool = blockIdx.x;  // (destination, wave); its pools from every source, in order
+  const int NPsrc = gridDim.x;
   const int dest = pool / W, wave = pool % W;
   const int e_first = dest * L + wave * P;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -498,8 +512,10 @@ __global__ void unpack_rank_kernel(const uint16_t* __restrict__ pools, int Cs, i
   // packed pools (dropless): this pool's rows are the pool_fill[pool] rows at pool_off[pool],
   // the row map holds the receiver slot and every row is kept
   const bool packed = pool_off != nullptr;
-  const long long prow0 = pool_row0(pool, Cs, pool_off);
-  const int nrows = packed ? pool_fill[pool] : Cs;
+  for (int src = 0; src < S; ++src) {
+  const int qpool = src * NPsrc + pool;
+  const long long prow0 = pool_row0(qpool, Cs, pool_off);
+  const int nrows = packed ? pool_fill[qpool] : Cs;
   const uint16_t* pbase = pools + prow0 * row_elems;
   for (int r0 = 0; r0 < nrows; r0 += kTile) {
     const int r = r0 + threadIdx.x;
@@ -535,6 +551,7 @@ __global__ void unpack_rank_kernel(const uint16_t* __restrict__ pools, int Cs, i
     }
     __syncthreads();
   }
+  }  // sources
   if (threadIdx.x < P) rows_out[e_first + threadIdx.x] = packed ? s_run[threadIdx.x] : min(s_run[threadIdx.x], Cr);
 }
 
@@ -858,39 +875,46 @@ int blocks_for(long long work, int per_block) {
 }  // namespace
 
 // off[i] = sum over j < i of round_up(counts[j], align), for i = 0..n; one block of 1024
-// threads, n <= 1024 (negative counts read as zero)
+// threads walking the counts 1024 at a time (negative counts read as zero)
 __global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict__ counts, int n, int align,
                                                        int32_t* __restrict__ off) {
   __shared__ int s_warp[32];
-  const int i = threadIdx.x;
-  const int lane = i & 31, warp = i >> 5;
-  int v = 0;
-  if (i < n) {
-    const int c = counts[i] > 0 ? counts[i] : 0;
-    v = (c + align - 1) / align * align;
-  }
-  int incl = v;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, incl, d);
-    if (lane >= d) incl += u;
-  }
-  if (lane == 31) s_warp[warp] = incl;
+  __shared__ int s_carry;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) s_carry = 0;
   __syncthreads();
-  if (warp == 0) {
-    int w = s_warp[lane];
+  for (int base = 0; base < n; base += 1024) {
+    const int i = base + threadIdx.x;
+    int v = 0;
+    if (i < n) {
+      const int c = counts[i] > 0 ? counts[i] : 0;
+      v = (c + align - 1) / align * align;
+    }
+    int incl = v;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, w, d);
-      if (lane >= d) w += u;
+      const int u = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += u;
     }
-    s_warp[lane] = w;  // inclusive over warps
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int w = s_warp[lane];
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, w, d);
+        if (lane >= d) w += u;
+      }
+      s_warp[lane] = w;  // inclusive over warps
+    }
+    __syncthreads();
+    const int before = s_carry + (warp > 0 ? s_warp[warp - 1] : 0);
+    if (i < n) off[i] = before + incl - v;
+    __syncthreads();
+    if (threadIdx.x == 1023) s_carry = before + incl;
+    __syncthreads();
   }
-  __syncthreads();
-  const int before = warp > 0 ? s_warp[warp - 1] : 0;
-  if (i < n) off[i] = before + incl - v;
-  if (i == n - 1) off[n] = before + incl;
-  if (n == 0 && i == 0) off[0] = 0;
+  if (threadIdx.x == 0) off[n] = s_carry;
 }
 
 // ====================================================================== launchers
@@ -919,7 +943,7 @@ moe_status_t launch_route(const Geo& g, const float* logits, const float* bias, 
 }
 
 size_t scan_scratch_ints(const Geo& g) {
-  return static_cast<size_t>(g.n_chunks) * (g.NP + g.E) + g.NP;
+  return static_cast<size_t>(g.n_chunks) * (g.NP + g.E) + g.NPS;
 }
 
 moe_status_t launch_slot_scan(const Geo& g, const int32_t* idx, int32_t* slot, int32_t* stats, int32_t* scratch,
@@ -928,28 +952,30 @@ moe_status_t launch_slot_scan(const Geo& g, const int32_t* idx, int32_t* slot, i
   const int chunk_assign = kScanTokensPerChunk * g.k;
   int32_t* cnt_pool = scratch;                                        // [NP][n_chunks]
   int32_t* cnt_exp = scratch + static_cast<size_t>(g.n_chunks) * g.NP;  // [E][n_chunks]
-  int32_t* pool_tot = cnt_exp + static_cast<size_t>(g.n_chunks) * g.E;  // [NP]
+  int32_t* pool_tot = cnt_exp + static_cast<size_t>(g.n_chunks) * g.E;  // [S][NP]
   // counters of this call start at zero (hist is left to the router)
   cudaError_t e = cudaMemsetAsync(stats + stats_kept_e(g), 0, sizeof(int32_t) * 3 * g.E, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(stats, 0, sizeof(int32_t) * 3, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(stats + 4, 0, sizeof(int32_t) * 3, st);
   if (e != cudaSuccess) return cuda_check(e, "slot scan memset");
   if (A == 0) {
-    e = cudaMemsetAsync(stats + stats_pool_fill(g), 0, sizeof(int32_t) * g.NP, st);
+    e = cudaMemsetAsync(stats + stats_pool_fill(g), 0, sizeof(int32_t) * g.NPS, st);
     return cuda_check(e, "slot scan memset");
   }
   scan_count_pools<<<g.n_chunks, 256, g.NP * sizeof(int), st>>>(idx, A, chunk_assign, g.n_chunks, g.L, g.P, g.W,
                                                                  g.NP, g.E, cnt_pool);
-  scan_rows<<<g.NP, 256, 0, st>>>(cnt_pool, g.n_chunks, pool_tot, g.Cs, stats + stats_pool_fill(g));
+  // sender slots count per (source, pool): the scan restarts at each source's first chunk
+  scan_rows<<<g.NP, 256, 0, st>>>(cnt_pool, g.n_chunks, pool_tot, g.Cs, stats + stats_pool_fill(g),
+                                  g.n_chunks / g.S);
   const int wpb = 4;
   const int grid = (g.n_chunks + wpb - 1) / wpb;
   scan_sender_slots<<<grid, 32 * wpb, wpb * (g.NP + g.E) * sizeof(int), st>>>(
       idx, A, chunk_assign, g.n_chunks, g.L, g.P, g.W, g.NP, g.E, g.Cs, cnt_pool, slot, cnt_exp, stats + 3);
-  scan_rows<<<g.E, 256, 0, st>>>(cnt_exp, g.n_chunks, nullptr, 0, nullptr);
+  scan_rows<<<g.E, 256, 0, st>>>(cnt_exp, g.n_chunks, nullptr, 0, nullptr, g.n_chunks);
   scan_receiver_slots<<<grid, 32 * wpb, wpb * g.E * sizeof(int), st>>>(
       idx, A, chunk_assign, g.n_chunks, g.E, g.Cr, cnt_exp, slot, stats + stats_kept_e(g), stats + stats_ds_e(g),
       stats + stats_dr_e(g));
-  scan_totals<<<1, 256, 0, st>>>(stats, g.E, g.NP, A, stats_kept_e(g), stats_ds_e(g), stats_dr_e(g),
+  scan_totals<<<1, 256, 0, st>>>(stats, g.E, g.NPS, A, stats_kept_e(g), stats_ds_e(g), stats_dr_e(g),
                                  stats_pool_fill(g));
   count_launch(6);
   return cuda_check(cudaGetLastError(), "slot scan");
@@ -973,21 +999,21 @@ moe_status_t launch_pack(const Geo& g, const uint16_t* z, const int32_t* idx, co
       const int grid = static_cast<int>(std::min<long long>((g.T + kPackWarps - 1) / kPackWarps,
                                                             static_cast<long long>(device_sm_count()) * per_sm));
       pack_bulk_kernel<<<grid, 32 * kPackWarps, smem, st>>>(z, idx, slot, g.T, g.k, g.dl, g.L, g.P, g.W, g.Cs, g.E,
-                                                            stats + stats_pool_fill(g), g.NP, pools, stats + 3,
-                                                            pool_off);
+                                                            stats + stats_pool_fill(g), g.NPS, pools, stats + 3,
+                                                            pool_off, g.Ts, g.NP);
       count_launch();
       return cuda_check(cudaGetLastError(), "pack");
     } else {
       const int warps = 8;
       pack_kernel<<<blocks_for(g.T, warps), 32 * warps, 0, st>>>(z, idx, slot, g.T, g.k, g.dl, g.L, g.P, g.W, g.Cs,
-                                                                 g.E, pools, pool_off);
+                                                                 g.E, pools, pool_off, g.Ts, g.NP);
     }
     count_launch();
   }
-  const long long rows = pool_off != nullptr ? 0 : static_cast<long long>(g.NP) * g.Cs;
+  const long long rows = pool_off != nullptr ? 0 : static_cast<long long>(g.NPS) * g.Cs;
   if (rows > 0)
   {
-    pack_empty_headers<<<blocks_for(rows, 256), 256, 0, st>>>(stats + stats_pool_fill(g), g.NP, g.Cs, g.dl, pools);
+    pack_empty_headers<<<blocks_for(rows, 256), 256, 0, st>>>(stats + stats_pool_fill(g), g.NPS, g.Cs, g.dl, pools);
     count_launch();
   }
   return cuda_check(cudaGetLastError(), "pack");
@@ -996,7 +1022,7 @@ moe_status_t launch_pack(const Geo& g, const uint16_t* z, const int32_t* idx, co
 size_t unpack_scratch_ints(const Geo& g) { return static_cast<size_t>(g.pool_rows); }
 
 moe_status_t launch_offsets(const int32_t* counts, int n, int align, int32_t* off, cudaStream_t st) {
-  if (n < 0 || n > 1024 || align < 1) return fail(MOE_ERR_UNSUPPORTED, "offsets over at most 1024 counts");
+  if (n < 0 || align < 1) return fail(MOE_ERR_INVALID_ARG, "offsets need n >= 0 and align >= 1");
   offsets_kernel<<<1, 1024, 0, st>>>(counts, n, align, off);
   count_launch();
   return cuda_check(cudaGetLastError(), "offsets");
@@ -1010,7 +1036,7 @@ moe_status_t launch_unpack(const Geo& g, const uint16_t* pools, uint16_t* xe, in
   if (packed && (pool_fill == nullptr || exp_off == nullptr))
     return fail(MOE_ERR_INVALID_ARG, "packed pools need their fills and the expert offsets");
   unpack_rank_kernel<<<g.NP, 256, 0, st>>>(pools, g.Cs, g.Cr, g.dl, g.L, g.P, g.W, row_map, rows, status, pool_off,
-                                           pool_fill);
+                                           pool_fill, g.S);
   count_launch();
   if (packed) MOE_TRY_K(launch_offsets(rows, g.E, 128, exp_off, st));
   const long long n_rows = g.pool_rows;

@@ -34,7 +34,8 @@ class MoEError(RuntimeError):
 class moe_config_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "T", "d_model", "d_latent", "n_experts", "top_k", "n_dest", "n_waves", "hidden_routed",
-        "n_shared", "hidden_shared", "cap_send_num", "cap_send_den", "cap_recv_num", "cap_recv_den")]
+        "n_shared", "hidden_shared", "cap_send_num", "cap_send_den", "cap_recv_num", "cap_recv_den",
+        "n_sources")]
 
 
 class moe_plan_info_t(ctypes.Structure):
@@ -152,9 +153,10 @@ class Plan:
     """Owns a moe_plan_t for one block shape."""
 
     def __init__(self, T, d_model, d_latent, n_experts, top_k, n_dest, hidden_routed, n_shared, hidden_shared,
-                 n_waves=3, cap_send=(110, 100), cap_recv=(115, 100)):
+                 n_waves=3, cap_send=(110, 100), cap_recv=(115, 100), n_sources=1):
         self.cfg = moe_config_t(T, d_model, d_latent, n_experts, top_k, n_dest, n_waves, hidden_routed,
-                                n_shared, hidden_shared, cap_send[0], cap_send[1], cap_recv[0], cap_recv[1])
+                                n_shared, hidden_shared, cap_send[0], cap_send[1], cap_recv[0], cap_recv[1],
+                                n_sources)
         h = ctypes.c_void_p()
         _check(_lib.moe_plan_create(ctypes.byref(self.cfg), ctypes.byref(h)), "moe_plan_create")
         self.handle = h
@@ -167,7 +169,7 @@ class Plan:
         # both capacity numerators 0 select the dropless variant
         cap_send, cap_recv = ((0, 1), (0, 1)) if getattr(s, "dropless", False) else (s.cap_send, s.cap_recv)
         return cls(s.T, s.d_model, s.d_latent, s.n_experts, s.top_k, s.n_dest, s.hidden_routed, s.n_shared,
-                   s.hidden_shared, s.n_waves, cap_send, cap_recv)
+                   s.hidden_shared, s.n_waves, cap_send, cap_recv, getattr(s, "n_sources", 1))
 
     def __del__(self):
         h = getattr(self, "handle", None)

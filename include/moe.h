@@ -90,6 +90,13 @@ typedef struct {
    * moe_plan_info reports cap_send = cap_recv = 0 and those sizes.  The dropless
    * variant runs through moe_forward / moe_backward; moe_dispatch, moe_expert_ffn,
    * moe_combine and moe_dispatch_noalloc return MOE_ERR_UNSUPPORTED for it. */
+  int32_t n_sources;      /* virtual sources S (0 or 1: one).  T splits into S equal,
+                           * contiguous token ranges, each sending its own D*W pools with
+                           * its own sender cap C_s = ceil(1.10 * (T/S)*k / (D*W)), as each
+                           * GPU does under expert parallelism ("Marin 535B-A23B" page on
+                           * ranhao.site, §3.1 topology; lamjinlab.com §2 caps per pool).
+                           * Pools are source-major; a destination's receiver reads its
+                           * pools source by source.  T/S must be a multiple of 32. */
 } moe_config_t;
 
 typedef struct moe_plan* moe_plan_t;
@@ -98,7 +105,7 @@ typedef struct moe_plan* moe_plan_t;
 typedef struct {
   int32_t local_experts;     /* L = E / D */
   int32_t experts_per_wave;  /* P = L / W */
-  int32_t n_pools;           /* D * W */
+  int32_t n_pools;           /* pools in the buffer: S * D * W (source-major) */
   int32_t cap_send;          /* C_s, rows of one pool (0: dropless) */
   int32_t cap_recv;          /* C_r, rows of one expert (0: dropless) */
   int32_t pool_row_elems;    /* bf16 elements per pool row: d_latent payload + 8 header */

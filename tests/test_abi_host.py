@@ -116,3 +116,19 @@ def test_dropless_plan_sizes(M):
     with pytest.raises(M.MoEError):
         M.Plan(T=T, d_model=128, d_latent=dl, n_experts=E, top_k=k, n_dest=4, hidden_routed=128,
                n_shared=1, hidden_shared=128, cap_send=(0, 1))
+
+
+def test_plan_with_sources(M):
+    """S sources: per-source sender caps, S*D*W pools; T/S must be whole scan chunks."""
+    base = dict(T=512, d_model=128, d_latent=64, n_experts=24, top_k=2, n_dest=4, hidden_routed=128,
+                n_shared=1, hidden_shared=128)
+    for S in (1, 2, 4, 16):
+        p = M.Plan(**base, n_sources=S)
+        assert p.info.n_pools == S * 4 * 3
+        assert p.info.cap_send == -(-512 * 2 * 110 // (100 * 12 * S))
+        assert p.info.cap_recv == -(-512 * 2 * 115 // (100 * 24))
+        assert p.info.pools_bytes == S * 12 * p.info.cap_send * (64 + 8) * 2
+    with pytest.raises(M.MoEError):
+        M.Plan(**base, n_sources=3)    # 512 / 3 is not whole
+    with pytest.raises(M.MoEError):
+        M.Plan(**base, n_sources=32)   # 16 tokens per source: not whole 32-token chunks

@@ -1,0 +1,99 @@
+"""Multiple virtual sources on the GPU against the oracle: per-source sender pools and
+caps (source-major), the receiver reading a destination's pools source by source."""
+import numpy as np
+import pytest
+import torch
+
+from _helpers import (ROUTED_GRAD_FRO, ROUTED_GRAD_TOL, assert_close_rms, assert_fro_close, bf16_dev, dev,
+                      host64, i32_dev)
+from capacity_limited_routed_b200 import synth
+from oracle import moe_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def M():
+    from capacity_limited_routed_b200 import moe
+    return moe
+
+
+@pytest.mark.parametrize("S,skew", [(4, 1.5), (16, 0.5), (2, 0.0)])
+def test_dispatch_bit_exact_with_sources(M, S, skew):
+    s = synth.TINY.with_(n_sources=S)
+    g = O.geometry(s)
+    plan = M.Plan.from_shape(s)
+    logits = synth.make_logits(s.T, s.n_experts, 3)
+    logits = (logits - np.float32(skew) * np.log1p(np.arange(s.n_experts, dtype=np.float32))[None, :])
+    idx_o = O.route(logits.astype(np.float32), np.zeros(s.n_experts, np.float32), s.top_k)[0]
+    sl = O.assign_slots(idx_o, g)
+    z = synth._bf16(np.random.default_rng(4).standard_normal((s.T, s.d_latent), dtype=np.float32))
+    payload, header = O.pack_pools(z, idx_o, sl["sslot"], g)
+    info = plan.info
+    assert info.n_pools == S * g.n_pools and info.cap_send == g.C_s
+    pools = torch.full((info.pools_bytes // 2,), 0x7FC0, dtype=torch.int16, device=dev()).view(torch.bfloat16)
+    slot = torch.full((s.T, s.top_k, 2), -5, dtype=torch.int32, device=dev())
+    stats = torch.zeros(info.stats_bytes // 4, dtype=torch.int32, device=dev())
+    ws = torch.empty(info.workspace_bytes, dtype=torch.uint8, device=dev())
+    M.moe_dispatch(plan, bf16_dev(z), i32_dev(idx_o), pools, slot, stats, ws)
+    torch.cuda.synchronize()
+    got = slot.cpu().numpy()
+    assert np.array_equal(got[..., 0], sl["sslot"]) and np.array_equal(got[..., 1], sl["rslot"])
+    st = stats.cpu().numpy()
+    E, NPS = s.n_experts, S * g.n_pools
+    assert (st[0], st[1], st[2], st[3]) == (sl["kept"], sl["dropped_sender"], sl["dropped_receiver"], 0)
+    assert np.array_equal(st[8 + 4 * E:8 + 4 * E + NPS], sl["pool_fill"])
+    rows = pools.view(torch.int16).cpu().numpy().reshape(NPS, g.C_s, s.d_latent + 8)
+    hdr = rows[:, :, s.d_latent:].copy().view(np.int32)[:, :, 0]
+    assert np.array_equal(hdr, header)
+    filled = header >= 0
+    assert np.array_equal(rows[:, :, :s.d_latent].view(np.uint16)[filled],
+                          synth.to_bf16_bits(payload.astype(np.float32))[filled])
+    # the expert path unpacks the source-major pools in the receiver's order
+    w1 = synth._bf16(np.random.default_rng(5).standard_normal((E, s.hidden_routed, s.d_latent), dtype=np.float32) * 0.1)
+    w3 = synth._bf16(np.random.default_rng(6).standard_normal((E, s.hidden_routed, s.d_latent), dtype=np.float32) * 0.1)
+    w2 = synth._bf16(np.random.default_rng(7).standard_normal((E, s.d_latent, s.hidden_routed), dtype=np.float32) * 0.1)
+    out = torch.zeros(info.expert_out_bytes // 2, dtype=torch.bfloat16, device=dev())
+    rows_dev = torch.empty(E, dtype=torch.int32, device=dev())
+    M.moe_expert_ffn(plan, bf16_dev(w1), bf16_dev(w3), bf16_dev(w2), pools, out, rows_dev, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(rows_dev.cpu().numpy(), sl["expert_kept"])
+
+
+@pytest.mark.parametrize("S", [4, 8])
+@pytest.mark.parametrize("dropless", [False, True])
+def test_block_with_sources_matches_oracle(S, dropless):
+    from capacity_limited_routed_b200.block import MoEBlock
+    s = synth.TINY.with_(n_sources=S, dropless=dropless, backward=True, zipf_s=0.8, seed=17)
+    inp = synth.make_inputs(s)
+    blk = MoEBlock(s, training=True)
+    blk.load(inp)
+    x = bf16_dev(inp["x"])
+    y = blk.forward(x)
+    dx = blk.backward(x, bf16_dev(inp["dy"]))
+    torch.cuda.synchronize()
+    y_o, ctx = O.forward(inp["x"], inp["weights"], inp["bias"], s, logit_offset=inp["logit_offset"])
+    dx_o, grads_o, _ = O.backward(inp["dy"], inp["weights"], ctx)
+    st = blk.stats_dict()
+    assert st["status"] == 0
+    v = blk.saved_views()
+    idx_g = v["topk_idx"].cpu().numpy()
+    match = (idx_g == ctx["idx"]).all(axis=1)
+    assert 1 - match.mean() <= 0.01
+    if match.all():
+        sl = ctx["slots"]
+        assert (st["kept"], st["dropped_sender"], st["dropped_receiver"]) == (
+            sl["kept"], sl["dropped_sender"], sl["dropped_receiver"])
+        assert np.array_equal(st["pool_fill"], sl["pool_fill"])
+        assert np.array_equal(v["slot"][..., 0].cpu().numpy(), sl["sslot"])
+        assert np.array_equal(v["slot"][..., 1].cpu().numpy(), sl["rslot"])
+    print(f"\n[S={S} dropless={dropless}] kept {st['kept']} of {s.T * s.top_k}, sender drops "
+          f"{st['dropped_sender']}, receiver drops {st['dropped_receiver']}")
+    assert_close_rms(host64(y)[match], y_o[match], what="y")
+    assert_close_rms(host64(dx)[match], dx_o[match], what="dx")
+    affected = set(np.unique(idx_g[~match]).tolist()) | set(np.unique(ctx["idx"][~match]).tolist())
+    keep_e = np.array([e not in affected for e in range(s.n_experts)])
+    for name in ("w1", "w3", "w2"):
+        got, want = host64(blk.grads[name])[keep_e], grads_o[name][keep_e]
+        assert_close_rms(got, want, tol=ROUTED_GRAD_TOL, what=f"d{name}")
+        assert_fro_close(got, want, ROUTED_GRAD_FRO, what=f"d{name}")
