@@ -23,6 +23,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -322,8 +323,9 @@ def main():
         raise RuntimeError(f"kernel status {st0['status']} after warm-up")
 
     # ---------------- timed region: K steps, device-resident inputs
-    clocks = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
-                          if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/clocks_rank{rank}.csv")
+    # the raw clock samples go to MOE_BENCH_CLOCKS_DIR (default: the system temp directory)
+    clocks_dir = os.environ.get("MOE_BENCH_CLOCKS_DIR") or tempfile.gettempdir()
+    clocks = ClockSampler(local, os.path.join(clocks_dir, f"clocks_rank{rank}.csv"))
     launches0 = M.moe_kernel_launches()
     M.moe_profile_start()
     ev0 = torch.cuda.Event(enable_timing=True)
