@@ -174,34 +174,34 @@ __global__ void scan_rows(int32_t* __restrict__ data, int n, int32_t* __restrict
   int32_t* row = data + static_cast<long long>(blockIdx.x) * n;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
   for (int s0 = 0; s0 < n; s0 += seg) {
-  if (threadIdx.x == 0) carry = 0;
-  __syncthreads();
-  const int s1 = min(n, s0 + seg);
-  for (int base = s0; base < s1; base += blockDim.x) {
-    const int i = base + threadIdx.x;
-    const int v = i < s1 ? row[i] : 0;
-    int incl = v;
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+    const int s1 = min(n, s0 + seg);
+    for (int base = s0; base < s1; base += blockDim.x) {
+      const int i = base + threadIdx.x;
+      const int v = i < s1 ? row[i] : 0;
+      int incl = v;
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += o;
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      if (lane == 31) warp_tot[warp] = incl;
+      __syncthreads();
+      int before = carry;
+      for (int w = 0; w < warp; ++w) before += warp_tot[w];
+      if (i < s1) row[i] = before + incl - v;
+      __syncthreads();
+      if (threadIdx.x == blockDim.x - 1) carry = before + incl;
+      __syncthreads();
+      (void)nwarp;
     }
-    if (lane == 31) warp_tot[warp] = incl;
+    if (threadIdx.x == 0) {
+      const long long o = static_cast<long long>(s0 / seg) * gridDim.x + blockIdx.x;
+      if (totals) totals[o] = carry;
+      if (clamp_out) clamp_out[o] = carry < cap ? carry : cap;
+    }
     __syncthreads();
-    int before = carry;
-    for (int w = 0; w < warp; ++w) before += warp_tot[w];
-    if (i < s1) row[i] = before + incl - v;
-    __syncthreads();
-    if (threadIdx.x == blockDim.x - 1) carry = before + incl;
-    __syncthreads();
-    (void)nwarp;
-  }
-  if (threadIdx.x == 0) {
-    const long long o = static_cast<long long>(s0 / seg) * gridDim.x + blockIdx.x;
-    if (totals) totals[o] = carry;
-    if (clamp_out) clamp_out[o] = carry < cap ? carry : cap;
-  }
-  __syncthreads();
   }
 }
 
@@ -513,44 +513,44 @@ __global__ void unpack_rank_kernel(const uint16_t* __restrict__ pools, int Cs, i
   // the row map holds the receiver slot and every row is kept
   const bool packed = pool_off != nullptr;
   for (int src = 0; src < S; ++src) {
-  const int qpool = src * NPsrc + pool;
-  const long long prow0 = pool_row0(qpool, Cs, pool_off);
-  const int nrows = packed ? pool_fill[qpool] : Cs;
-  const uint16_t* pbase = pools + prow0 * row_elems;
-  for (int r0 = 0; r0 < nrows; r0 += kTile) {
-    const int r = r0 + threadIdx.x;
-    int q = -1;
-    if (r < nrows) {
-      const int e = *reinterpret_cast<const int*>(pbase + r * row_elems + dl);
-      if (e >= 0) {
-        if (e >= e_first && e < e_first + P) q = e - e_first;
-        else atomicCAS(status, 0, MOE_ERR_INVALID_ARG);  // an id this pool cannot hold
+    const int qpool = src * NPsrc + pool;
+    const long long prow0 = pool_row0(qpool, Cs, pool_off);
+    const int nrows = packed ? pool_fill[qpool] : Cs;
+    const uint16_t* pbase = pools + prow0 * row_elems;
+    for (int r0 = 0; r0 < nrows; r0 += kTile) {
+      const int r = r0 + threadIdx.x;
+      int q = -1;
+      if (r < nrows) {
+        const int e = *reinterpret_cast<const int*>(pbase + r * row_elems + dl);
+        if (e >= 0) {
+          if (e >= e_first && e < e_first + P) q = e - e_first;
+          else atomicCAS(status, 0, MOE_ERR_INVALID_ARG);  // an id this pool cannot hold
+        }
       }
+      // rank of this row among the tile's rows of the same local expert, in row order
+      int rank = 0;
+      for (int qq = 0; qq < P; ++qq) {
+        const unsigned m = __ballot_sync(0xffffffffu, q == qq);
+        if (q == qq) rank = __popc(m & ((1u << lane) - 1u));
+        if (lane == 0) s_warp_cnt[warp][qq] = __popc(m);
+      }
+      __syncthreads();
+      int slot = -1;
+      if (q >= 0) {
+        int before = s_run[q];
+        for (int w = 0; w < warp; ++w) before += s_warp_cnt[w][q];
+        slot = before + rank;
+      }
+      if (r < nrows)
+        row_map[prow0 + r] = packed ? slot : ((slot >= 0 && slot < Cr) ? (e_first + q) * Cr + slot : -1);
+      __syncthreads();
+      if (threadIdx.x < P) {
+        int tot = 0;
+        for (int w = 0; w < kTile / 32; ++w) tot += s_warp_cnt[w][threadIdx.x];
+        s_run[threadIdx.x] += tot;
+      }
+      __syncthreads();
     }
-    // rank of this row among the tile's rows of the same local expert, in row order
-    int rank = 0;
-    for (int qq = 0; qq < P; ++qq) {
-      const unsigned m = __ballot_sync(0xffffffffu, q == qq);
-      if (q == qq) rank = __popc(m & ((1u << lane) - 1u));
-      if (lane == 0) s_warp_cnt[warp][qq] = __popc(m);
-    }
-    __syncthreads();
-    int slot = -1;
-    if (q >= 0) {
-      int before = s_run[q];
-      for (int w = 0; w < warp; ++w) before += s_warp_cnt[w][q];
-      slot = before + rank;
-    }
-    if (r < nrows)
-      row_map[prow0 + r] = packed ? slot : ((slot >= 0 && slot < Cr) ? (e_first + q) * Cr + slot : -1);
-    __syncthreads();
-    if (threadIdx.x < P) {
-      int tot = 0;
-      for (int w = 0; w < kTile / 32; ++w) tot += s_warp_cnt[w][threadIdx.x];
-      s_run[threadIdx.x] += tot;
-    }
-    __syncthreads();
-  }
   }  // sources
   if (threadIdx.x < P) rows_out[e_first + threadIdx.x] = packed ? s_run[threadIdx.x] : min(s_run[threadIdx.x], Cr);
 }
