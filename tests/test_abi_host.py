@@ -132,3 +132,34 @@ def test_plan_with_sources(M):
         M.Plan(**base, n_sources=3)    # 512 / 3 is not whole
     with pytest.raises(M.MoEError):
         M.Plan(**base, n_sources=32)   # 16 tokens per source: not whole 32-token chunks
+
+
+def test_struct_layouts_match_the_header(M, tmp_path):
+    """Every struct the binding passes across the ABI has the size and field offsets the
+    header gives it, as compiled by the host C compiler."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    structs = [M.moe_config_t, M.moe_plan_info_t, M.moe_weights_t, M.moe_grads_t, M.moe_expert_weights_t,
+               M.moe_profile_record_t, M.moe_saved_view_t]
+    lines = ['#include <stdio.h>', '#include <stddef.h>', f'#include "{os.path.join(ROOT, "include", "moe.h")}"',
+             "int main(void) {"]
+    for st in structs:
+        n = st.__name__
+        lines.append(f'  printf("{n} size %zu\\n", sizeof({n}));')
+        for f, _ in st._fields_:
+            lines.append(f'  printf("{n} {f} %zu\\n", offsetof({n}, {f}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-std=c11", "-o", str(exe), str(src)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    got = {" ".join(l.split()[:2]): int(l.split()[2]) for l in out if l.strip()}
+    for st in structs:
+        n = st.__name__
+        assert got[f"{n} size"] == ctypes.sizeof(st), n
+        for f, _ in st._fields_:
+            assert got[f"{n} {f}"] == getattr(st, f).offset, (n, f)
