@@ -207,33 +207,37 @@ class ClockSampler:
 # ------------------------------------------------------------------ CPU oracle baseline
 
 
-def oracle_sample_shape(s):
-    """A bounded sample of the workload for the CPU oracle: 256 tokens at the full widths
+def oracle_sample_shape(s, T=256):
+    """A bounded sample of the workload for the CPU oracle: T tokens at the full widths
     (every token still runs top-k full-width experts, the shared experts and both latent
     projections), with 24 routed experts (4 destinations x 6) instead of 384 so the
     weights fit the host; per-token work is the same."""
-    return s.with_(T=256, n_experts=24, n_dest=4)
+    return s.with_(T=T, n_experts=24, n_dest=4)
 
 
-def run_oracle_sample(s, reps=1):
-    import numpy as np
+def oracle_inputs(s, T=256):
+    """The sample's synthetic inputs (drawn once; drawing is not part of a step)."""
     from capacity_limited_routed_b200 import synth
+    ss = oracle_sample_shape(s, T).with_(backward=True)
+    return ss, synth.make_inputs(ss, seed=123)
+
+
+def run_oracle_sample(s, ss, inp):
+    """One step of the oracle on the sample: forward, and for a training workload the
+    backward and the bias step.  Returns (tokens/s, threads used)."""
     from oracle import moe_oracle as O
-    ss = oracle_sample_shape(s).with_(backward=True)
-    inp = synth.make_inputs(ss, seed=123)
     t0 = time.perf_counter()
-    for _ in range(reps):
-        y, ctx = O.forward(inp["x"], inp["weights"], inp["bias"], ss, logit_offset=inp["logit_offset"])
-        if s.backward:
-            O.backward(inp["dy"], inp["weights"], ctx)
-            O.bias_update(ctx["hist"], inp["bias"], 1e-3, ss.T, ss.top_k)
+    y, ctx = O.forward(inp["x"], inp["weights"], inp["bias"], ss, logit_offset=inp["logit_offset"])
+    if s.backward:
+        O.backward(inp["dy"], inp["weights"], ctx)
+        O.bias_update(ctx["hist"], inp["bias"], 1e-3, ss.T, ss.top_k)
     dt = time.perf_counter() - t0
     try:
         from threadpoolctl import threadpool_info
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:
         cores = os.cpu_count()
-    return ss.T * reps / dt, cores, ss
+    return ss.T / dt, cores
 
 
 def reference_arm(args, s):
@@ -241,12 +245,15 @@ def reference_arm(args, s):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    steps, warm = max(1, min(args.steps, 3)), max(0, min(args.warmup, 1))
+    # every step is a bounded sample (64 tokens, a few seconds of host work), so that the
+    # whole run of exactly --warmup + --steps steps ends within a few minutes
+    steps, warm = max(1, args.steps), max(0, args.warmup)
+    ss, inp = oracle_inputs(s, T=64)
     for _ in range(warm):
-        run_oracle_sample(s)
+        run_oracle_sample(s, ss, inp)
     rates = []
     for _ in range(steps):
-        r, cores, ss = run_oracle_sample(s)
+        r, cores = run_oracle_sample(s, ss, inp)
         rates.append(r)
     v = statistics.median(rates)
     sample = (f"per step {ss.T} tokens at full widths ({ss.d_model}/{ss.d_latent}/{ss.hidden_routed}, "
@@ -264,6 +271,127 @@ def reference_arm(args, s):
 # ------------------------------------------------------------------ GPU arm
 
 
+def end_to_end(args, s, blk, x, dy, hist_plan, world, dev, barrier):
+    """The same steps through the public API with host buffers: every step copies its
+    inputs (x, and dy for training) in from pinned host memory and its results (y, and
+    dx for training) out to pinned host memory.  The copies run on two copy streams and
+    overlap the neighbouring steps' kernels (inputs one step ahead, outputs one step
+    behind, double-buffered on the device); the timed region ends when the last step's
+    results are on the host."""
+    import torch
+    from capacity_limited_routed_b200 import moe as M
+    from capacity_limited_routed_b200.parallel import global_histogram
+    cs = torch.cuda.current_stream(dev)
+    h2d = torch.cuda.Stream(dev)
+    d2h = torch.cuda.Stream(dev)
+    x_h = x.cpu().pin_memory()
+    dy_h = dy.cpu().pin_memory() if s.backward else None
+    y_h = torch.empty((s.T, s.d_model), dtype=torch.float32).pin_memory()
+    dx_h = torch.empty((s.T, s.d_model), dtype=torch.float32).pin_memory() if s.backward else None
+    xs = [torch.empty_like(x) for _ in range(2)]
+    dys = [torch.empty_like(dy) for _ in range(2)] if s.backward else None
+    ys = [torch.empty((s.T, s.d_model), dtype=torch.float32, device=dev) for _ in range(2)]
+    dxs = [torch.empty((s.T, s.d_model), dtype=torch.float32, device=dev) for _ in range(2)] if s.backward else None
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_ready = [ev(), ev()]      # inputs of buffer b are on the device
+    in_free = [ev(), ev()]       # the step that used buffer b no longer reads its inputs
+    out_ready = [ev(), ev()]     # results of buffer b are written
+    out_free = [ev(), ev()]      # results of buffer b are on the host
+    for b in range(2):
+        in_free[b].record(cs)
+        out_free[b].record(cs)
+
+    def load(i):
+        b = i % 2
+        with torch.cuda.stream(h2d):
+            h2d.wait_event(in_free[b])
+            xs[b].copy_(x_h, non_blocking=True)
+            if s.backward:
+                dys[b].copy_(dy_h, non_blocking=True)
+            in_ready[b].record(h2d)
+
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(cs)
+    h2d.wait_event(e0)
+    d2h.wait_event(e0)
+    load(0)
+    for i in range(args.steps):
+        b = i % 2
+        if i + 1 < args.steps:
+            load(i + 1)
+        cs.wait_event(in_ready[b])
+        cs.wait_event(out_free[b])
+        blk.forward(xs[b], y=ys[b])
+        if s.backward:
+            blk.backward(xs[b], dys[b], dx=dxs[b])
+            global_histogram(blk.hist())
+            M.moe_bias_update(hist_plan, blk.hist(), blk.bias, 1e-3)
+        in_free[b].record(cs)
+        out_ready[b].record(cs)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(out_ready[b])
+            y_h.copy_(ys[b], non_blocking=True)
+            if s.backward:
+                dx_h.copy_(dxs[b], non_blocking=True)
+            out_free[b].record(d2h)
+    cs.wait_stream(d2h)
+    e1.record(cs)
+    torch.cuda.synchronize()
+    barrier()
+    e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+    e_step = float(e_ms.item()) / args.steps
+    if not bool(torch.isfinite(y_h[:: max(1, s.T // 64)]).all()):
+        raise RuntimeError("end-to-end: non-finite y on the host")
+    h2d_b = x.numel() * 2 + (dy.numel() * 2 if s.backward else 0)
+    d2h_b = y_h.numel() * 4 + (dx_h.numel() * 4 if s.backward else 0)
+    return {"value": world * s.T / (e_step * 1e-3), "unit": "tokens/s", "ms_per_step": e_step,
+            "h2d_bytes_per_step": h2d_b, "d2h_bytes_per_step": d2h_b,
+            "copies": "x, dy in from pinned host; y, dx out to pinned host, every step "
+                      "(two copy streams, overlapping the neighbouring steps)"}
+
+
+def forward_pass(shape, weights, dev, steps, warmup):
+    """Forward-only throughput of a full-width workload on weights already on the device
+    (same widths): CUDA events around `steps` forward passes after `warmup` of them."""
+    import torch
+    from capacity_limited_routed_b200 import synth
+    from capacity_limited_routed_b200.block import MoEBlock
+    inp = synth.make_tokens_device(shape, device=dev)
+    inp["weights"] = weights
+    blk = MoEBlock(shape, device=dev, training=False)
+    blk.load(inp)
+    x = inp["x"]
+    y = torch.empty((shape.T, shape.d_model), dtype=torch.float32, device=dev)
+    for _ in range(warmup):
+        blk.forward(x, y=y)
+    st = torch.cuda.current_stream(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(st)
+    for _ in range(steps):
+        blk.forward(x, y=y)
+    e1.record(st)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    sd = blk.stats_dict()
+    if sd["status"] != 0:
+        raise RuntimeError(f"kernel status {sd['status']} in the {shape.name} forward pass")
+    A = shape.T * shape.top_k
+    out = {"tokens_per_s": shape.T / (ms * 1e-3), "ms_per_step": ms, "steps": steps, "warmup": warmup,
+           "workload": describe(shape), "kept": sd["kept"],
+           "drop_fraction": {"sender": sd["dropped_sender"] / A, "receiver": sd["dropped_receiver"] / A}}
+    del blk, inp, x, y
+    return out
+
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -273,6 +401,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-only", action="store_true", help="a few steps, no baseline, no e2e (for ncu)")
+    ap.add_argument("--no-forward-passes", action="store_true",
+                    help="skip the forward-only passes of the full and skewed workloads")
     args = ap.parse_args()
     s = workload_shape(args.workload)
     if args.impl == "reference":
@@ -396,41 +526,22 @@ def main():
     # ---------------- end to end through the public API, host buffers
     e2e = None
     if not args.profile_only:
-        x_h = x.cpu().pin_memory()
-        dy_h = dy.cpu().pin_memory() if dy is not None else None
-        out_h = torch.empty(8, dtype=torch.int32).pin_memory()
-        xs = torch.empty_like(x)
-        dys = torch.empty_like(dy) if dy is not None else None
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        barrier()
+        e2e = end_to_end(args, s, blk, x, dy, hist_plan, world, dev, barrier)
+
+    # ---------------- forward-only passes of the full-width layer and the skewed stress
+    fwd_extra = {}
+    if not args.profile_only and not args.no_forward_passes and world == 1 and \
+            (s.d_model, s.d_latent, s.n_experts, s.hidden_routed) == (6144, 3072, 384, 3072):
+        for name, shape in (("fwd_full", synth.FULL), ("fwd_skewed", synth.SKEWED)):
+            fwd_extra[name] = forward_pass(shape, blk.weights, dev, args.steps, max(args.warmup, 3))
         torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(args.steps):
-            xs.copy_(x_h, non_blocking=True)
-            if s.backward:
-                dys.copy_(dy_h, non_blocking=True)
-            blk.forward(xs)
-            if s.backward:
-                blk.backward(xs, dys)
-                global_histogram(blk.hist())
-                M.moe_bias_update(hist_plan, blk.hist(), blk.bias, 1e-3)
-            out_h.copy_(blk.stats[:8], non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-        e_step = float(e_ms.item()) / args.steps
-        e2e = {"value": world * s.T / (e_step * 1e-3), "unit": "tokens/s",
-               "h2d_bytes_per_step": x.numel() * 2 + (dy.numel() * 2 if dy is not None else 0),
-               "d2h_bytes_per_step": 32, "read_back": "stats head (kept / dropped counters)"}
 
     # ---------------- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile_only:
-        r, cores, ss = run_oracle_sample(s)
+        ss, oinp = oracle_inputs(s, T=256)
+        r, cores = run_oracle_sample(s, ss, oinp)
+        del oinp
         cpu = {"value": r, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"{ss.T} tokens of this workload at full widths with {ss.n_experts} routed experts "
                          f"instead of {s.n_experts} (same per-token work), one pass, float64 numpy"}
@@ -444,6 +555,8 @@ def main():
             "config": {"workload": describe(s), "parallelism": f"replicas x{world} (one source per GPU)",
                        "l2": "inputs larger than L2 (22 GB of expert weights streamed every step)"},
             "fwd_tokens_per_s": world * s.T / (fwd_ms * 1e-3) if fwd_ms > 0 else None,
+            "fwd_tokens_per_s_kind": "sum of the forward steps' CUDA-event times inside the timed training steps",
+            **fwd_extra,
             "drop_fraction": {"sender": st["dropped_sender"] / A, "receiver": st["dropped_receiver"] / A},
             "roofline": roof,
             "dispatch_hbm_frac": kernels.get("fwd.dispatch_pack", {}).get("frac"),

@@ -1124,12 +1124,9 @@ template <int BN, bool A_MN, bool B_MN, int EPI>
 moe_status_t launch_instance(const TmaMaps& maps, const KParams& kp, int grid, cudaStream_t st) {
   auto kern = gemm_kernel<BN, A_MN, B_MN, EPI>;
   const int smem = Cfg<BN, A_MN && B_MN, EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BWD>::kSmem;
-  static bool attr_set = false;  // per instantiation
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return cuda_check(e, "cudaFuncSetAttribute(gemm)");
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};  // per instantiation, one bit per device
+  const moe_status_t r = ensure_max_smem(reinterpret_cast<const void*>(kern), smem, attr_done, "gemm");
+  if (r != MOE_OK) return r;
   kern<<<grid, Roles<A_MN && B_MN>::kThreads, smem, st>>>(maps, kp);
   count_launch();
   return cuda_check(cudaGetLastError(), "gemm launch");
@@ -1137,14 +1134,38 @@ moe_status_t launch_instance(const TmaMaps& maps, const KParams& kp, int grid, c
 
 }  // namespace
 
-int device_sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+int current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return -1;
   }
+  return dev;
+}
+
+moe_status_t ensure_max_smem(const void* func, int bytes, std::atomic<uint64_t>& done_mask, const char* what) {
+  const int dev = current_device();
+  const uint64_t bit = (dev >= 0 && dev < kMaxDevices) ? (uint64_t(1) << dev) : 0;
+  if (bit != 0 && (done_mask.load(std::memory_order_acquire) & bit)) return MOE_OK;
+  const cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return cuda_check(e, (std::string("cudaFuncSetAttribute(") + what + ")").c_str());
+  if (bit != 0) done_mask.fetch_or(bit, std::memory_order_acq_rel);
+  return MOE_OK;
+}
+
+int device_sm_count() {
+  static std::atomic<int> cached[kMaxDevices];  // 0: not looked up yet
+  const int dev = current_device();
+  if (dev >= 0 && dev < kMaxDevices) {
+    const int c = cached[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int n = 0;
+  if (dev < 0 || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    (void)cudaGetLastError();
+    n = 148;
+  }
+  if (dev >= 0 && dev < kMaxDevices) cached[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
@@ -1263,11 +1284,17 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
   if (a.a_mn && a.b_mn && a.epi == EPI_F32 && a.nseg == 1 && a.ragged != 1 && a.bn == 256) {
     const long long pair_tiles =
         static_cast<long long>(a.groups) * ((a.M + 255) / 256) * ((a.N + 255) / 256);
-    static int max_pairs = 0;  // pairs that fit on the device at once
+    // pairs that fit on the device at once, per device (0: not measured yet)
+    static std::atomic<int> max_pairs_dev[kMaxDevices];
+    static std::atomic<uint64_t> attr_done{0};
+    const int dev = current_device();
+    int max_pairs = (dev >= 0 && dev < kMaxDevices) ? max_pairs_dev[dev].load(std::memory_order_relaxed) : 0;
+    {
+      const moe_status_t r = ensure_max_smem(reinterpret_cast<const void*>(gemm_pair_wgrad_kernel), PairCfg::kSmem,
+                                             attr_done, "pair gemm");
+      if (r != MOE_OK) return r;
+    }
     if (max_pairs == 0) {
-      cudaError_t e = cudaFuncSetAttribute(gemm_pair_wgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           PairCfg::kSmem);
-      if (e != cudaSuccess) return cuda_check(e, "cudaFuncSetAttribute(pair gemm)");
       cudaLaunchConfig_t cfg;
       memset(&cfg, 0, sizeof(cfg));
       cfg.gridDim = dim3(2 * (device_sm_count() / 2));
@@ -1279,6 +1306,7 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
         nc = device_sm_count() / 2;
       }
       max_pairs = std::min(nc, device_sm_count() / 2);
+      if (dev >= 0 && dev < kMaxDevices) max_pairs_dev[dev].store(max_pairs, std::memory_order_relaxed);
     }
     const int pairs = static_cast<int>(std::min<long long>(pair_tiles, max_pairs));
     if (pairs <= 0) return MOE_OK;

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <string>
 
 #include "../../include/moe.h"
@@ -15,6 +16,21 @@ namespace moe {
 void set_error(const std::string& msg);
 moe_status_t fail(moe_status_t code, const std::string& msg);
 moe_status_t cuda_check(cudaError_t e, const char* what);
+
+// ------------------------------------------------------------------ per-device set-up
+//
+// The CUDA runtime keeps function attributes (the dynamic shared-memory limit) and
+// occupancy answers per device, so every cache of them is keyed by the device index.
+// A set bit in a mask means "done on this device"; two threads racing on the same
+// device only repeat the (idempotent) set-up.
+
+constexpr int kMaxDevices = 64;
+
+// index of the calling thread's current device, or -1 when there is none
+int current_device();
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per device for `func`
+moe_status_t ensure_max_smem(const void* func, int bytes, std::atomic<uint64_t>& done_mask, const char* what);
 
 // ------------------------------------------------------------------ launch accounting
 

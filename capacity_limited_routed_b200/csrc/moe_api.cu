@@ -200,17 +200,17 @@ moe_status_t device_ok() {
     cudaGetLastError();
     return fail(MOE_ERR_UNSUPPORTED, std::string("no CUDA device: ") + cudaGetErrorString(e));
   }
-  static int checked[64] = {0};  // 0 unknown, 1 ok, 2 bad
-  if (dev >= 0 && dev < 64 && checked[dev] == 1) return MOE_OK;
+  static std::atomic<int> checked[kMaxDevices];  // per device: 0 unknown, 1 ok, 2 bad
+  if (dev >= 0 && dev < kMaxDevices && checked[dev].load(std::memory_order_relaxed) == 1) return MOE_OK;
   int major = 0, minor = 0;
   cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
   cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
   if (major != 10 || minor != 0) {
-    if (dev >= 0 && dev < 64) checked[dev] = 2;
+    if (dev >= 0 && dev < kMaxDevices) checked[dev].store(2, std::memory_order_relaxed);
     return fail(MOE_ERR_UNSUPPORTED, "libmoe needs an sm_100 (B200) device, found sm_" + std::to_string(major) +
                                          std::to_string(minor));
   }
-  if (dev >= 0 && dev < 64) checked[dev] = 1;
+  if (dev >= 0 && dev < kMaxDevices) checked[dev].store(1, std::memory_order_relaxed);
   return MOE_OK;
 }
 

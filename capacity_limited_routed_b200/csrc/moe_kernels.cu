@@ -987,14 +987,10 @@ moe_status_t launch_pack(const Geo& g, const uint16_t* z, const int32_t* idx, co
     // two row buffers per warp; rows too wide for that take the register path
     const size_t smem = static_cast<size_t>(kPackWarps) * 2 * g.dl * 2;
     if (g.k <= 32 && smem <= 200 * 1024) {
-      static bool attr_set = false;
-      if (!attr_set) {
-        const moe_status_t r = cuda_check(
-            cudaFuncSetAttribute(pack_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024),
-            "cudaFuncSetAttribute(pack)");
-        if (r != MOE_OK) return r;
-        attr_set = true;
-      }
+      static std::atomic<uint64_t> attr_done{0};  // one bit per device
+      const moe_status_t r =
+          ensure_max_smem(reinterpret_cast<const void*>(pack_bulk_kernel), 200 * 1024, attr_done, "pack");
+      if (r != MOE_OK) return r;
       const int per_sm = smem <= 100 * 1024 ? 2 : 1;
       const int grid = static_cast<int>(std::min<long long>((g.T + kPackWarps - 1) / kPackWarps,
                                                             static_cast<long long>(device_sm_count()) * per_sm));

@@ -25,14 +25,17 @@ static __device__ __align__(256) int32_t g_dispatch_scratch[kStaticScratchInts];
 
 // The device address of g_dispatch_scratch, per device.  In host code the array's
 // name only stands in for the symbol; a kernel given it would read the wrong memory.
+// The address is looked up once per device and kept for the life of the process: a
+// cudaDeviceReset reloads the module and may move the array, so the library must not
+// be used across a reset of a device it has already run on.
 std::mutex g_mu;
-int32_t* g_scratch_ptr[64] = {nullptr};
+int32_t* g_scratch_ptr[kMaxDevices] = {nullptr};
 
 moe_status_t scratch_for_current_device(int32_t** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_check(e, "cudaGetDevice");
-  if (dev < 0 || dev >= 64) return fail(MOE_ERR_UNSUPPORTED, "device index out of range for static scratch");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device index out of range for static scratch");
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;

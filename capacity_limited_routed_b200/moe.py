@@ -172,9 +172,11 @@ class Plan:
                    s.hidden_shared, s.n_waves, cap_send, cap_recv, getattr(s, "n_sources", 1))
 
     def __del__(self):
+        # at interpreter shutdown the module globals may already be gone
         h = getattr(self, "handle", None)
-        if h is not None and h.value:
-            _lib.moe_plan_destroy(h)
+        lib_ = globals().get("_lib")
+        if h is not None and h.value and lib_ is not None:
+            lib_.moe_plan_destroy(h)
             self.handle = None
 
 

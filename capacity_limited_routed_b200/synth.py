@@ -239,6 +239,19 @@ def make_inputs_device(shape: MoEShape, device="cuda", seed: int | None = None) 
             ("w3", (E, h, dl), dl), ("w2", (E, dl, h), h), ("w_lat_up", (dm, dl), dl),
             ("ws1", (S * hs, dm), dm), ("ws3", (S * hs, dm), dm), ("ws2", (dm, S * hs), hs)]
     weights = {n: _dev_normal(shp, 1.0 / math.sqrt(fan), base + i, device) for i, (n, shp, fan) in enumerate(spec)}
+    out = make_tokens_device(s, device=device, seed=seed)
+    out["weights"] = weights
+    return out
+
+
+def make_tokens_device(shape: MoEShape, device="cuda", seed: int | None = None) -> dict:
+    """The per-batch inputs of ``make_inputs_device`` alone (x, bias, logit_offset and,
+    for a backward workload, dy), drawn exactly as there: a workload of the same widths
+    can then run on weights that already sit on the device."""
+    import torch
+    s = shape
+    base = (shape.seed if seed is None else seed) * 1000003
+    dm, E = s.d_model, s.n_experts
     if s.window and s.rho > 0.0:
         n_win = (s.T + s.window - 1) // s.window
         gwin = _dev_normal((n_win, dm), 1.0, base + 20, device).float()
@@ -253,7 +266,6 @@ def make_inputs_device(shape: MoEShape, device="cuda", seed: int | None = None) 
     lo_ = make_logit_offset(s)
     out = {
         "x": x,
-        "weights": weights,
         "bias": torch.zeros(E, dtype=torch.float32, device=device),
         "logit_offset": None if lo_ is None else torch.from_numpy(lo_).to(device),
     }

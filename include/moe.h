@@ -173,7 +173,13 @@ typedef struct {
 
 /* Create a plan for one block shape (host only: checks sizes, computes C_s, C_r
  * and the buffer layouts).  Returns MOE_ERR_UNSUPPORTED for shapes outside the
- * supported set, MOE_ERR_INVALID_ARG for nonsense. */
+ * supported set, MOE_ERR_INVALID_ARG for nonsense.  The capacities are the expected
+ * rows times the factors, rounded up: C_s = ceil(1.10 * (T/S)*k / (D*W)) per
+ * (destination, wave) pool of a source, C_r = ceil(1.15 * T*k / E) per expert.
+ * ("Marin начинает открытое обучение MoE-модели с 535 млрд параметров", §2: six
+ * experts per GPU, three waves of identical shape, sender cap 1.10 per pool,
+ * receiver cap 1.15 per local expert; "Marin 535B-A23B：一场完全公开的前沿 MoE 训练直播",
+ * §2.1 spec table: 384 routed experts, top-8, 64-way expert parallelism.) */
 MOE_API moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out);
 MOE_API moe_status_t moe_plan_destroy(moe_plan_t plan);
 MOE_API moe_status_t moe_plan_info(moe_plan_t plan, moe_plan_info_t* out);
@@ -210,11 +216,13 @@ MOE_API moe_status_t moe_dispatch(moe_plan_t plan, const uint16_t* z, const int3
  * a static array inside the library (2^21 int32 words, 8 MiB, held on every GPU that
  * loads the library until the process exits).  Inputs and outputs are those of
  * moe_dispatch, with the same results.
- *   - Plans whose scan needs more than 2^21 words (T/32 * (D*W + E) + D*W) are
- *     rejected with MOE_ERR_UNSUPPORTED; use moe_dispatch for them.
+ *   - Plans whose scan needs more than 2^21 words (ceil(T/32) * (D*W + E) +
+ *     n_sources * D*W) are rejected with MOE_ERR_UNSUPPORTED; use moe_dispatch for
+ *     them.
  *   - The first call on a device looks up the array's device address (once per
  *     device, with that device current); make that first call before any stream
- *     capture.
+ *     capture.  The address is kept for the life of the process, so do not use the
+ *     library across a cudaDeviceReset of a device it has already run on.
  *   - Every call uses the same array.  Calls whose work overlaps on the GPU (other
  *     streams, other threads) race on it; order them on one stream.  Nothing in the
  *     array has to start at zero: each call writes every word it reads.
@@ -224,7 +232,11 @@ MOE_API moe_status_t moe_dispatch_noalloc(moe_plan_t plan, const uint16_t* z, co
                                           uint16_t* pools, int32_t* slot, void* stats, void* stream);
 
 /* Receiver side and the routed experts: unpack each pool by the packed expert ids
- * (first C_r rows per expert in pool order), then the grouped SwiGLU GEMMs.
+ * (first C_r rows per expert in pool order), then the grouped SwiGLU GEMMs
+ * Y_e = (silu(X_e w1_e^T) * (X_e w3_e^T)) w2_e^T.  ("Marin начинает открытое обучение
+ * MoE-модели с 535 млрд параметров", §2: the receiver learns each row's expert from
+ * the id in the payload, with no separate count or metadata exchange;
+ * "Marin 535B-A23B：一场完全公开的前沿 MoE 训练直播", §2.2: SwiGLU experts of width 3072.)
  *   pools as written by moe_dispatch; expert_out [E][C_r][d_latent] bf16 device
  *   (rows at and past the expert's row count are zero or unspecified);
  *   expert_rows [E] int32 device, rows each expert received (may be NULL). */
@@ -233,7 +245,11 @@ MOE_API moe_status_t moe_expert_ffn(moe_plan_t plan, const moe_expert_weights_t*
                             void* ws, size_t ws_bytes, void* stream);
 
 /* Combine: r_t = sum_j kept gate_tj * expert_out[e_tj][rslot_tj], in rank order,
- * float32 accumulation, bf16 result.  r [T][d_latent] bf16 device. */
+ * float32 accumulation, bf16 result.  r [T][d_latent] bf16 device.  Dropped
+ * assignments contribute nothing and the gates are not renormalised.
+ * ("Marin 535B-A23B：一场完全公开的前沿 MoE 训练直播", §2.2 diagram: the routed
+ * outputs are weighted and summed in the latent space, then projected back to
+ * d_model before they meet the shared path.) */
 MOE_API moe_status_t moe_combine(moe_plan_t plan, const uint16_t* expert_out, const float* topk_gate,
                          const int32_t* topk_idx, const int32_t* slot, uint16_t* r,
                          void* stream);
@@ -241,14 +257,26 @@ MOE_API moe_status_t moe_combine(moe_plan_t plan, const uint16_t* expert_out, co
 /* Whole forward pass: y [T][d_model] float32 device from x [T][d_model] bf16 device.
  * bias [E] float32 device; logit_offset [E] float32 device or NULL.  stats: stats
  * buffer (device), fully overwritten.  saved: forward context for moe_backward
- * (saved_bytes) or NULL for inference. */
+ * (saved_bytes) or NULL for inference.  Steps, in order: latent down-projection,
+ * router, top-k, slot assignment, pack, unpack, grouped SwiGLU experts, combine,
+ * shared experts, up-projection with the shared down-projection.
+ * ("Marin начинает открытое обучение MoE-модели с 535 млрд параметров", §2, and
+ * "Marin 535B-A23B：一场完全公开的前沿 MoE 训练直播", §2.2: the 6144 -> 3072 latent
+ * projection around the routed path, top-8 of 384 routed experts, two always-on
+ * shared SwiGLU experts on every token; "Treinamento aberto do Marin 535B",
+ * "A matemática do MoE": the shared experts at half width.) */
 MOE_API moe_status_t moe_forward(moe_plan_t plan, const moe_weights_t* w, const uint16_t* x,
                          const float* bias, const float* logit_offset, float* y,
                          void* stats, void* saved, void* ws, size_t ws_bytes, void* stream);
 
 /* Whole backward pass for the loss sum(y * dy): dy [T][d_model] bf16 device, dx
- * [T][d_model] float32 device and every weight gradient (overwritten, float32).  Dropped assignments get no gradient;
- * the bias gets none.  x must be the forward's input, saved its context. */
+ * [T][d_model] float32 device and every weight gradient (overwritten, float32).
+ * Dropped assignments get no gradient; the bias gets none, while the router weights
+ * get theirs through the gates.  x must be the forward's input, saved its context.
+ * ("Marin 535B-A23B：一场完全公开的前沿 MoE 训练直播", §2.2: the balancing bias stays
+ * outside backpropagation and does not change the router's gradients;
+ * "Marin начинает открытое обучение MoE-модели с 535 млрд параметров", §2: dropped
+ * rows are counted and contribute nothing.) */
 MOE_API moe_status_t moe_backward(moe_plan_t plan, const moe_weights_t* w, const void* saved,
                           const uint16_t* x, const uint16_t* dy, float* dx,
                           const moe_grads_t* grads, void* ws, size_t ws_bytes, void* stream);

@@ -570,46 +570,102 @@ def forward_tokens(weights, rb: dict, tokens):
         r = st(r)
         a_s, b_s, H_s = swiglu_hidden(x[t:t + 1], ws1, ws3, st)
         out.append(r @ W_up.T + H_s[0] @ ws2.T)
-        per.append({"r": r, "rows": rows, "a_s": a_s[0], "b_s": b_s[0]})
+        per.append({"r": r, "rows": rows, "a_s": a_s[0], "b_s": b_s[0], "H_s": H_s[0]})
     return np.array(out), per
+
+
+def _backward_token(dy, weights, rb: dict, t, p, dense):
+    """The backward pass of one token t of a batch routed by ``route_batch``, for the
+    loss y_t . dy: every intermediate of the token and its kept rows."""
+    st = _storage(rb["storage"])
+    idx, gate = rb["idx"], rb["gate"]
+    dy = np.asarray(dy, np.float64)
+    dr = st(dy @ dense["w_lat_up"])
+    dH_s = dy @ dense["ws2"]
+    da_s = st(dH_s * p["b_s"] * silu_grad(p["a_s"]))
+    db_s = st(dH_s * silu(p["a_s"]))
+    k = idx.shape[1]
+    dg = np.zeros(k)
+    dXsum = np.zeros(dr.shape[0])
+    rows = []
+    for (j, a, b, H, Y, (W1, W3, W2)) in p["rows"]:
+        dg[j] = float(dr @ Y)
+        dY = st(gate[t, j] * dr)
+        dH = dY @ W2
+        dA = st(dH * b * silu_grad(a))
+        dB = st(dH * silu(a))
+        dXsum = dXsum + st(dA @ W1 + dB @ W3)
+        rows.append((j, dY, dA, dB, H))
+    dl_chosen = gate[t] * (dg - (gate[t] * dg).sum())
+    dlog = np.zeros(dense["w_router"].shape[0])
+    dlog[idx[t].astype(np.int64)] = dl_chosen
+    dlog = st(dlog)
+    dz = st(dlog @ dense["w_router"] + dXsum)
+    dx = dz @ dense["w_lat_down"] + da_s @ dense["ws1"] + db_s @ dense["ws3"]
+    return {"dx": dx, "dr": dr, "da_s": da_s, "db_s": db_s, "dlogits": dlog, "dz": dz, "rows": rows}
+
+
+def _dense_weights(weights):
+    return {n: np.asarray(weights[n], np.float64)
+            for n in ("w_lat_up", "w_router", "w_lat_down", "ws1", "ws3", "ws2")}
 
 
 def backward_tokens(dy_rows, weights, rb: dict, tokens, per):
     """dx for the given tokens (rows of dy given for those tokens, in order)."""
-    st = _storage(rb["storage"])
-    idx, gate = rb["idx"], rb["gate"]
-    W_up = np.asarray(weights["w_lat_up"], np.float64)
-    W_r = np.asarray(weights["w_router"], np.float64)
-    W_dn = np.asarray(weights["w_lat_down"], np.float64)
-    ws1 = np.asarray(weights["ws1"], np.float64)
-    ws3 = np.asarray(weights["ws3"], np.float64)
-    ws2 = np.asarray(weights["ws2"], np.float64)
-    E = W_r.shape[0]
-    out = []
+    dense = _dense_weights(weights)
+    return np.array([_backward_token(dy_rows[n], weights, rb, t, per[n], dense)["dx"]
+                     for n, t in enumerate(tokens)])
+
+
+def sampled_weight_grads(dy_rows, weights, rb: dict, tokens, per):
+    """Every weight gradient of the loss sum over the given tokens of y_t . dy_t (the
+    upstream gradient is zero on every other token): each gradient is the sum over
+    those tokens of its per-token outer products, formed as one matrix product of the
+    stacked per-token factors.  Returns the dense gradients as arrays and the routed
+    ones as {expert: {"w1", "w3", "w2"}} for the experts those tokens' kept rows reach
+    (every other expert's gradient is zero)."""
+    dense = _dense_weights(weights)
+    x, z, idx = rb["x"], rb["z"], rb["idx"]
+    cols = {n: [] for n in ("dy", "r", "H_s", "dlogits", "z", "dz", "x", "da_s", "db_s")}
+    rows_of = {}
     for n, t in enumerate(tokens):
         dy = np.asarray(dy_rows[n], np.float64)
         p = per[n]
-        dr = st(dy @ W_up)
-        dH_s = dy @ ws2
-        da_s = st(dH_s * p["b_s"] * silu_grad(p["a_s"]))
-        db_s = st(dH_s * silu(p["a_s"]))
-        k = idx.shape[1]
-        dg = np.zeros(k)
-        dXsum = np.zeros(dr.shape[0])
-        for (j, a, b, H, Y, (W1, W3, W2)) in p["rows"]:
-            dg[j] = float(dr @ Y)
-            dY = st(gate[t, j] * dr)
-            dH = dY @ W2
-            dA = st(dH * b * silu_grad(a))
-            dB = st(dH * silu(a))
-            dXsum = dXsum + st(dA @ W1 + dB @ W3)
-        dl_chosen = gate[t] * (dg - (gate[t] * dg).sum())
-        dlog = np.zeros(E)
-        dlog[idx[t].astype(np.int64)] = dl_chosen
-        dlog = st(dlog)
-        dz = st(dlog @ W_r + dXsum)
-        out.append(dz @ W_dn + da_s @ ws1 + db_s @ ws3)
-    return np.array(out)
+        b = _backward_token(dy, weights, rb, t, p, dense)
+        for key, val in (("dy", dy), ("r", p["r"]), ("H_s", p["H_s"]), ("dlogits", b["dlogits"]), ("z", z[t]),
+                         ("dz", b["dz"]), ("x", x[t]), ("da_s", b["da_s"]), ("db_s", b["db_s"])):
+            cols[key].append(val)
+        for (j, dY, dA, dB, H) in b["rows"]:
+            rows_of.setdefault(int(idx[t, j]), []).append((dA, dB, dY, z[t], H))
+    m = {key: np.array(v) for key, v in cols.items()}
+    g = {"w_lat_up": m["dy"].T @ m["r"], "ws2": m["dy"].T @ m["H_s"], "w_router": m["dlogits"].T @ m["z"],
+         "w_lat_down": m["dz"].T @ m["x"], "ws1": m["da_s"].T @ m["x"], "ws3": m["db_s"].T @ m["x"]}
+    routed = {}
+    for e, rows in rows_of.items():
+        dA, dB, dY, X, H = (np.array(c) for c in zip(*rows))
+        routed[e] = {"w1": dA.T @ X, "w3": dB.T @ X, "w2": dY.T @ H}
+    return g, routed
+
+
+def shared_weight_grad_rows(x, dy, weights, units, storage="bf16"):
+    """Gradients of the shared experts' weights for the hidden units ``units`` (rows of
+    ws1 and ws3, columns of ws2) over every token, for the loss sum(y * dy).  The shared
+    path does not depend on routing, so this is the whole-batch gradient restricted to
+    those units: a_u = x ws1[u]^T, b_u = x ws3[u]^T, H_u = silu(a_u) b_u, dH_u = dy ws2[:, u],
+    dws1[u] = (dH_u b_u silu'(a_u))^T x, dws3[u] = (dH_u silu(a_u))^T x, dws2[:, u] = dy^T H_u.
+    Returns (dws1 rows [n][d_model], dws3 rows [n][d_model], dws2 columns [d_model][n])."""
+    st = _storage(storage)
+    x = np.asarray(x, np.float64)
+    dy = np.asarray(dy, np.float64)
+    units = np.asarray(units, np.int64)
+    ws1 = np.asarray(weights["ws1"][units], np.float64)
+    ws3 = np.asarray(weights["ws3"][units], np.float64)
+    ws2 = np.asarray(weights["ws2"][:, units], np.float64)
+    a, b, H = swiglu_hidden(x, ws1, ws3, st)
+    dH = dy @ ws2
+    da = st(dH * b * silu_grad(a))
+    db = st(dH * silu(a))
+    return da.T @ x, db.T @ x, dy.T @ H
 
 
 def expert_weight_grads(dy, weights, rb: dict, e: int):

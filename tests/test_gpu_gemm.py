@@ -102,3 +102,29 @@ def test_gemm_weight_gradient_short_contractions(M, k):
         torch.cuda.synchronize()
         err = (D.double().cpu() - ref).abs().max().item()
         assert err <= 1e-4 * rms(ref.numpy()) * max(1.0, np.sqrt(k / 64)), err
+
+
+def test_gemm_weight_gradient_full_token_contraction(M):
+    """The dense weight-gradient form at the block's full size: both operands MN-major,
+    K = 16,384 tokens, a [6144][3072] float32 result (the latent-projection and shared
+    weight gradients of the training step), checked on sampled output rows against a
+    float64 contraction of the same bf16 operands."""
+    m, n, k = 6144, 3072, 16384
+    gen = torch.Generator(device=dev()).manual_seed(77)
+    A = torch.randn((k, m), generator=gen, device=dev()).to(torch.bfloat16)   # [K][M]
+    B = torch.randn((k, n), generator=gen, device=dev()).to(torch.bfloat16)   # [K][N]
+    D = torch.full((m, n), float("nan"), dtype=torch.float32, device=dev())
+    status = torch.zeros(1, dtype=torch.int32, device=dev())
+    M.moe_gemm_bf16(m, n, k, A, 1, B, 1, D, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert bool(torch.isfinite(D).all().item())
+    rows = np.sort(np.random.default_rng(3).choice(m, size=24, replace=False))
+    rows = np.unique(np.concatenate([rows, [0, 255, 256, m - 1]]))
+    a_h = A[:, torch.from_numpy(rows).to(dev())].double().cpu().numpy()        # [K][rows]
+    b_h = B.double().cpu().numpy()                                            # [K][N]
+    ref = a_h.T @ b_h
+    got = D[torch.from_numpy(rows).to(dev())].double().cpu().numpy()
+    err = np.abs(got - ref).max()
+    # float32 accumulation of 16,384 products of unit-variance terms
+    assert err <= 1e-4 * rms(ref) * np.sqrt(k / 64), err

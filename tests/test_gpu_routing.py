@@ -148,23 +148,18 @@ def test_expert_ffn_and_combine(M, shape, skew):
     Y = host64(out)
     W1, W3, W2 = (w[n].astype(np.float64) for n in ("w1", "w3", "w2"))
     want_all, got_all = [], []
+    Yo = np.zeros((s.n_experts, g.C_r, s.d_latent), dtype=np.float32)
     for e in range(s.n_experts):
         n = counts_o[e]
         if n == 0:
             continue
-        X = rows_o[e].astype(np.float64)
-        a, b = X @ W1[e].T, X @ W3[e].T
-        H = O.round_bf16(O.silu(a) * b)
-        want_all.append(H @ W2[e].T)
+        # the oracle's SwiGLU of the rows the receiver kept, bf16 hidden and output
+        _, _, H = O.swiglu_hidden(rows_o[e].astype(np.float64), W1[e], W3[e], O.round_bf16)
+        Yo[e, :n] = O.round_bf16(H @ W2[e].T)
+        want_all.append(Yo[e, :n])
         got_all.append(Y[e, :n])
     assert_close_rms(np.concatenate(got_all), np.concatenate(want_all), what="expert_out")
     # combine, fed the oracle's own expert outputs (uploaded as bf16)
-    Yo = np.zeros((s.n_experts, g.C_r, s.d_latent), dtype=np.float32)
-    for e in range(s.n_experts):
-        n = counts_o[e]
-        if n:
-            X = rows_o[e].astype(np.float64)
-            Yo[e, :n] = O.round_bf16(O.round_bf16(O.silu(X @ W1[e].T) * (X @ W3[e].T)) @ W2[e].T)
     slot = np.stack([slots["sslot"], slots["rslot"]], axis=-1).astype(np.int32)
     r = torch.empty((s.T, s.d_latent), dtype=torch.bfloat16, device=dev())
     M.moe_combine(plan, bf16_dev(Yo), f32_dev(gate_o), i32_dev(idx_o), i32_dev(slot), r)
