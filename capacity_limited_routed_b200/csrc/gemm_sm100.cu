@@ -17,6 +17,12 @@
 // Two accumulators in TMEM let the epilogue of one tile overlap the main loop of
 // the next.  Tiles of all groups (experts) form one list that CTAs stride over;
 // ragged groups take their row (or K) counts from device memory.
+//
+// PAIR instances run the same roles on a pair of CTAs (a cluster of two,
+// cta_group::2): 256-row tiles, each CTA loading its 128 rows of A and half of B's
+// columns, the leader issuing M=256 MMAs that read both CTAs' shared memory, each CTA
+// draining its own 128 accumulator rows.  Per output element the pair reads a third
+// fewer operand bytes into shared memory than one CTA with a 128-row tile.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -88,12 +94,12 @@ constexpr int kMaxGroups = 1024;
 // 256 float32 = 128 KB) weighs as much as its operands: it gets a ring of two staging
 // buffers per epilogue warp so stores stream without waiting.  It never runs with
 // ragged rows, so it needs no tile-prefix array.
-template <int BN, bool WRITE_BOUND = false, bool SWIGLU = false>
+template <int BN, bool WRITE_BOUND = false, bool SWIGLU = false, bool PAIR = false>
 struct Cfg {
   static constexpr int kABytes = kBM * kBK * 2;  // 16 KB
-  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * kBK * 2;  // a pair CTA holds half of B
   static constexpr int kStage = kABytes + kBBytes;
-  static constexpr int kStages = WRITE_BOUND ? MOE_WB_STAGES : ((BN == 256) ? 4 : 6);
+  static constexpr int kStages = WRITE_BOUND ? MOE_WB_STAGES : ((BN == 256 && !PAIR) ? 4 : 6);
   static constexpr int kTmemCols = 2 * BN;
   static constexpr int kBufs = WRITE_BOUND ? MOE_WB_BUFS : 1;  // staging buffers per epilogue warp
   static constexpr int kEpiWarps = Roles<WRITE_BOUND>::kEpiWarps;
@@ -118,7 +124,7 @@ struct Tile {
 };
 
 // Tile bookkeeping shared by the three roles; all of them walk the same list.
-template <int BN, int EPI>
+template <int BN, int EPI, int TM = kBM>
 struct Sched {
   const KParams& p;
   const int* prefix;  // ragged == 1: tiles before group g (shared memory)
@@ -127,7 +133,7 @@ struct Sched {
   __device__ Sched(const KParams& pp, const int* pre) : p(pp), prefix(pre) {
     const int out_cols = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
     nt = (p.N + out_cols - 1) / out_cols;
-    mt_fixed = (p.M + kBM - 1) / kBM;
+    mt_fixed = (p.M + TM - 1) / TM;
     tiles_per_group = mt_fixed * nt;
     total = (p.ragged == 1) ? prefix[p.groups] : p.groups * tiles_per_group;
   }
@@ -182,10 +188,14 @@ struct Sched {
   }
 };
 
-template <int BN, bool A_MN, bool B_MN, int EPI>
+template <int BN, bool A_MN, bool B_MN, int EPI, bool PAIR>
 __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
     gemm_kernel(const __grid_constant__ TmaMaps maps, const KParams p) {
-  using C = Cfg<BN, A_MN && B_MN, EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BWD>;
+  using C = Cfg<BN, A_MN && B_MN, EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BWD, PAIR>;
+  constexpr int TM = PAIR ? 2 * kBM : kBM;  // rows of A per tile (per pair of CTAs for PAIR)
+  // PAIR: this CTA's rank in its cluster of two; rank 0 (the leader) issues the MMAs
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + C::kStages * C::kStage;
@@ -209,7 +219,7 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 32 * C::kEpiWarps);
+      mbar_init(&tempty[a], 32 * C::kEpiWarps * (PAIR ? 2 : 1));  // PAIR: both CTAs' epilogues
     }
     mbar_init(drain, 1);
     for (int w = 0; w < 12; ++w) mbar_init(&ebar[w], 1);
@@ -223,8 +233,13 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(tmem_slot, C::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::kTmemCols);
+      tmem_relinquish();
+    }
   }
   // tiles per group and their prefix (ragged rows only)
   if (C::kPrefixInts > 0 && p.ragged == 1) {
@@ -238,7 +253,7 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
       if (g < p.groups) {
         int r = p.group_rows[g];
         r = r < 0 ? 0 : (r > p.M ? p.M : r);
-        local += ((r + kBM - 1) / kBM) * nt;
+        local += ((r + TM - 1) / TM) * nt;
       }
     }
     // block exclusive scan of `local` over 192 threads
@@ -260,18 +275,19 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
         prefix[g] = run;
         int r = p.group_rows[g];
         r = r < 0 ? 0 : (r > p.M ? p.M : r);
-        run += ((r + kBM - 1) / kBM) * nt;
+        run += ((r + TM - 1) / TM) * nt;
       }
     }
     if (threadIdx.x == kThreads - 1) prefix[p.groups] = before + incl;
   }
   tc_fence_before();
   __syncthreads();
+  if (PAIR) cluster_sync_all();  // both CTAs' barriers exist before either touches the other's
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const volatile int* abort_v = abort_flag;
 
-  Sched<BN, EPI> sc(p, prefix);
+  Sched<BN, EPI, TM> sc(p, prefix);
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -305,25 +321,38 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
           const int k0 = kl * kBK;
           uint8_t* sa = smem + stage * C::kStage;
           uint8_t* sb = sa + C::kABytes;
-          mbar_arrive_expect_tx(&full[stage], C::kStage);
+          // PAIR: the leader's barrier counts both CTAs' bytes
+          if (!PAIR) mbar_arrive_expect_tx(&full[stage], C::kStage);
+          else if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kStage);
           armed_phase[stage] = static_cast<int>(phase);
-          const int m0 = mt * kBM;
+          const uint32_t lbar = leader_addr(smem_u32(&full[stage]));
+          auto ld = [&](const CUtensorMap* map, void* dst, int c0, int c1, int c2) {
+            if (PAIR) tma_load_3d_pair(map, dst, lbar, c0, c1, c2);
+            else tma_load_3d(map, dst, &full[stage], c0, c1, c2);
+          };
+          const int m0 = mt * TM + (PAIR ? kBM * static_cast<int>(rank) : 0);
           if (!A_MN) {
-            tma_load_3d(&maps.a[s], sa, &full[stage], k0, gro + m0, gz);
+            ld(&maps.a[s], sa, k0, gro + m0, gz);
           } else {
-            tma_load_3d(&maps.a[s], sa, &full[stage], m0, k0, g);
-            tma_load_3d(&maps.a[s], sa + 8192, &full[stage], m0 + 64, k0, g);
+            ld(&maps.a[s], sa, m0, k0, g);
+            ld(&maps.a[s], sa + 8192, m0 + 64, k0, g);
           }
           if (EPI == EPI_SWIGLU) {
+            // B = [gate rows | value rows]; PAIR: the leader holds the gate half, its partner the value half
             const int n0 = ntile * (BN / 2);
-            tma_load_3d(&maps.b[0], sb, &full[stage], k0, n0, g);
-            tma_load_3d(&maps.bv, sb + (BN / 2) * 128, &full[stage], k0, n0, g);
+            if (PAIR) {
+              ld(rank == 0 ? &maps.b[0] : &maps.bv, sb, k0, n0, g);
+            } else {
+              ld(&maps.b[0], sb, k0, n0, g);
+              ld(&maps.bv, sb + (BN / 2) * 128, k0, n0, g);
+            }
           } else if (!B_MN) {
-            tma_load_3d(&maps.b[s], sb, &full[stage], k0, ntile * BN, g);
+            ld(&maps.b[s], sb, k0, ntile * BN + (PAIR ? (BN / 2) * static_cast<int>(rank) : 0), g);
           } else {
+            constexpr int nb = (PAIR ? BN / 2 : BN) / 64;
+            const int nc0 = ntile * BN + (PAIR ? (BN / 2) * static_cast<int>(rank) : 0);
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j)
-              tma_load_3d(&maps.b[s], sb + j * 8192, &full[stage], ntile * BN + 64 * j, k0, g);
+            for (int j = 0; j < nb; ++j) ld(&maps.b[s], sb + j * 8192, nc0 + 64 * j, k0, g);
           }
           if (++stage == C::kStages) {
             stage = 0;
@@ -334,15 +363,17 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
       if (!ok) {
         *abort_flag = 1;
         record_status(p.status, MOE_ERR_TIMEOUT);
-        // let every load already issued land before the CTA goes away
-        for (int s = 0; s < C::kStages; ++s)
-          if (armed_phase[s] >= 0) mbar_wait(&full[s], static_cast<uint32_t>(armed_phase[s]), nullptr, 50000000ull);
+        // let every load already issued land before the CTA goes away (PAIR: the leader's
+        // barriers count both CTAs' loads, and neither CTA leaves before the other)
+        if (leader)
+          for (int s = 0; s < C::kStages; ++s)
+            if (armed_phase[s] >= 0) mbar_wait(&full[s], static_cast<uint32_t>(armed_phase[s]), nullptr, 50000000ull);
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, A_MN, B_MN);
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = idesc_bf16_f32(TM, BN, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -375,17 +406,20 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
                                      : smem_desc_sw128(a_addr + k * 32, 16, 1024);
             const uint64_t bd = B_MN ? smem_desc_sw128(b_addr + k * 2048, 8192, 1024)
                                      : smem_desc_sw128(b_addr + k * 32, 16, 1024);
-            mma_bf16_ss(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            if (PAIR) mma_bf16_ss_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            else mma_bf16_ss(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
           }
           issued = true;
-          mma_commit(&empty[stage]);
+          if (PAIR) mma_commit_pair(&empty[stage]);
+          else mma_commit(&empty[stage]);
           if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        mma_commit(&tfull[acc]);
+        if (PAIR) mma_commit_pair(&tfull[acc]);
+        else mma_commit(&tfull[acc]);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
@@ -393,7 +427,8 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
         *abort_flag = 1;
         record_status(p.status, MOE_ERR_TIMEOUT);
         if (issued) {
-          mma_commit(drain);
+          if (PAIR) mma_commit_pair(drain);
+          else mma_commit(drain);
           mbar_wait(drain, 0, nullptr, 50000000ull);
         }
       }
@@ -407,6 +442,14 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
     const int col_lo = (C::kEpiWarps == 8) ? (ew >> 2) * (BN / 2) : 0;
     const int col_hi = (C::kEpiWarps == 8) ? col_lo + BN / 2 : BN;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    // hand an accumulator back to the MMA warp (PAIR: to the leader's barrier)
+    uint32_t tempty_leader = 0;
+    if (PAIR)
+      asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(tempty_leader) : "r"(smem_u32(&tempty[0])), "r"(0));
+    auto release = [&](int a) {
+      if (PAIR) mbar_arrive_cluster(tempty_leader + static_cast<uint32_t>(a * 8));
+      else mbar_arrive(&tempty[a]);
+    };
     int acc = 0;
     uint32_t acc_phase = 0;
     int ring = 0;        // next staging buffer of this warp
@@ -421,7 +464,8 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
         const int gz = p.group_off != nullptr ? 0 : g, gro = cur.off;
         (void)gz;
         (void)gro;
-      const int row = mt * kBM + row_in_tile;
+      const int mbase = mt * TM + (PAIR ? kBM * static_cast<int>(rank) : 0);  // this CTA's first row
+      const int row = mbase + row_in_tile;
       const bool row_ok = row < p.M;
       if (kb_total == 0) {
         // an empty contraction (group with no rows): the product is zero
@@ -444,7 +488,7 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
       // SwiGLU backward: a and b come in by TMA one 16-column chunk ahead of their use,
       // into a ring of three slots per warp; the first chunk's load starts before the
       // accumulator is ready
-      const int srow0 = mt * kBM + q * 32;
+      const int srow0 = mbase + q * 32;
       int s_live = 0;  // live 16-column chunks of this warp in this tile
       if constexpr (EPI == EPI_SWIGLU_BWD) {
         if (srow0 < p.M) {
@@ -481,7 +525,7 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
         // per chunk of 32 output columns: H, a, b as three 32 x 64-byte tiles (64-byte
         // swizzle: 16-byte piece j of row r at j ^ ((r >> 1) & 3)), three TMA stores
         const int n_out0 = ntile * (BN / 2);
-        const int row0 = mt * kBM + q * 32;
+        const int row0 = mbase + q * 32;
         uint8_t* buf = staging + ew * C::kBufBytes;
         const uint32_t rbase = smem_u32(buf) + lane * 64;
         const int sw = (lane >> 1) & 3;
@@ -498,7 +542,7 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
           tmem_wait_ld();
           if (c2 + 64 >= BN / 2) {
             tc_fence_before();
-            mbar_arrive(&tempty[acc]);
+            release(acc);
             released = true;
           }
 #pragma unroll
@@ -545,7 +589,7 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
         // instruction writes four whole 128-byte lines.
         constexpr int kChunk = (EPI == EPI_F32) ? 32 : 64;
         constexpr int kEsz = (EPI == EPI_F32) ? 4 : 2;
-        const int row0 = mt * kBM + q * 32;
+        const int row0 = mbase + q * 32;
         uint8_t* buf = staging + ew * C::kBufs * C::kBufBytes;
         const uint32_t sbase = smem_u32(buf);
         const int piece = lane & 7;    // 16-byte piece of a row this lane reads back
@@ -598,7 +642,7 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
         // Rows past M and columns past N are clipped by the tensor map.  The accumulator
         // is released as soon as the whole tile is in registers.
         constexpr int kChunk = (EPI == EPI_F32) ? 32 : 64;  // columns per 128-byte row
-        const int row0 = mt * kBM + q * 32;
+        const int row0 = mbase + q * 32;
 #pragma unroll 1
         for (int half = 0; half < BN; half += 128) {
           uint32_t r[4][32];
@@ -608,7 +652,7 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
           tmem_wait_ld();
           if (half + 128 >= BN) {
             tc_fence_before();
-            mbar_arrive(&tempty[acc]);
+            release(acc);
             released = true;
           }
 #pragma unroll
@@ -749,7 +793,7 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
       __syncwarp();
       if (!released) {
         tc_fence_before();
-        mbar_arrive(&tempty[acc]);
+        release(acc);
       }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
@@ -760,10 +804,12 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (PAIR) cluster_sync_all();  // neither CTA leaves while the other may still touch its memory
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::kTmemCols);
+    if (PAIR) tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    else tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
@@ -1120,16 +1166,54 @@ moe_status_t make_map(CUtensorMap* m, const Mat& t, uint32_t box_inner, uint32_t
   return MOE_OK;
 }
 
-template <int BN, bool A_MN, bool B_MN, int EPI>
-moe_status_t launch_instance(const TmaMaps& maps, const KParams& kp, int grid, cudaStream_t st) {
-  auto kern = gemm_kernel<BN, A_MN, B_MN, EPI>;
-  const int smem = Cfg<BN, A_MN && B_MN, EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BWD>::kSmem;
+// tiles: output tiles of the launch (pair tiles for PAIR); the grid is one CTA (or pair)
+// per tile up to what fits on the device at once
+template <int BN, bool A_MN, bool B_MN, int EPI, bool PAIR>
+moe_status_t launch_instance(const TmaMaps& maps, const KParams& kp, long long tiles, cudaStream_t st) {
+  auto kern = gemm_kernel<BN, A_MN, B_MN, EPI, PAIR>;
+  const int smem = Cfg<BN, A_MN && B_MN, EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BWD, PAIR>::kSmem;
+  constexpr int threads = Roles<A_MN && B_MN>::kThreads;
   static std::atomic<uint64_t> attr_done{0};  // per instantiation, one bit per device
   const moe_status_t r = ensure_max_smem(reinterpret_cast<const void*>(kern), smem, attr_done, "gemm");
   if (r != MOE_OK) return r;
-  kern<<<grid, Roles<A_MN && B_MN>::kThreads, smem, st>>>(maps, kp);
+  if (!PAIR) {
+    const int grid = static_cast<int>(std::min<long long>(tiles, device_sm_count()));
+    kern<<<grid, threads, smem, st>>>(maps, kp);
+    count_launch();
+    return cuda_check(cudaGetLastError(), "gemm launch");
+  }
+  // pairs that fit on the device at once, per device (0: not asked yet)
+  static std::atomic<int> max_pairs_dev[kMaxDevices];
+  const int dev = current_device();
+  int max_pairs = (dev >= 0 && dev < kMaxDevices) ? max_pairs_dev[dev].load(std::memory_order_relaxed) : 0;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (max_pairs == 0) {
+    cfg.gridDim = dim3(2 * (device_sm_count() / 2));
+    int nc = 0;
+    if (cudaOccupancyMaxActiveClusters(&nc, kern, &cfg) != cudaSuccess || nc <= 0) {
+      (void)cudaGetLastError();
+      nc = device_sm_count() / 2;
+    }
+    max_pairs = std::min(nc, device_sm_count() / 2);
+    if (dev >= 0 && dev < kMaxDevices) max_pairs_dev[dev].store(max_pairs, std::memory_order_relaxed);
+  }
+  const int pairs = static_cast<int>(std::min<long long>(tiles, max_pairs));
+  cfg.gridDim = dim3(2 * pairs);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, maps, kp);
   count_launch();
-  return cuda_check(cudaGetLastError(), "gemm launch");
+  if (e != cudaSuccess) return cuda_check(e, "pair gemm launch");
+  return cuda_check(cudaGetLastError(), "pair gemm launch");
 }
 
 }  // namespace
@@ -1204,7 +1288,8 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
     moe_status_t r;
     r = make_map(&maps.a[s], a.A[s], 64, a.a_mn ? 64 : 128, "A");
     if (r != MOE_OK) return r;
-    const uint32_t b_rows = a.b_mn ? 64 : (a.epi == EPI_SWIGLU ? a.bn / 2 : a.bn);
+    // a pair CTA loads half of B's rows (SwiGLU: the gate or the value half)
+    const uint32_t b_rows = a.b_mn ? 64 : ((a.epi == EPI_SWIGLU || a.pair) ? a.bn / 2 : a.bn);
     r = make_map(&maps.b[s], a.B[s], 64, b_rows, "B");
     if (r != MOE_OK) return r;
     kp.seg_kb[s] = a.ragged == 2 ? 0 : static_cast<int>((a.K[s] + kBK - 1) / kBK);
@@ -1315,13 +1400,14 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
     return cuda_check(cudaGetLastError(), "pair gemm launch");
   }
   const int out_cols = a.epi == EPI_SWIGLU ? a.bn / 2 : a.bn;
-  const long long tiles = static_cast<long long>(a.groups) * ((a.M + kBM - 1) / kBM) * ((a.N + out_cols - 1) / out_cols);
-  const int grid = static_cast<int>(std::min<long long>(tiles, device_sm_count()));
-  if (grid <= 0) return MOE_OK;
+  const int tm = a.pair ? 2 * kBM : kBM;
+  const long long tiles = static_cast<long long>(a.groups) * ((a.M + tm - 1) / tm) * ((a.N + out_cols - 1) / out_cols);
+  if (tiles <= 0) return MOE_OK;
 
 #define MOE_GEMM_CASE(BN_, AMN_, BMN_, EPI_)                                               \
   if (a.bn == BN_ && a.a_mn == AMN_ && a.b_mn == BMN_ && a.epi == EPI_)                   \
-    return launch_instance<BN_, AMN_, BMN_, EPI_>(maps, kp, grid, st);
+    return a.pair ? launch_instance<BN_, AMN_, BMN_, EPI_, true>(maps, kp, tiles, st)     \
+                  : launch_instance<BN_, AMN_, BMN_, EPI_, false>(maps, kp, tiles, st);
   // forward: projections / experts (bf16 out), SwiGLU, router logits, block output (f32)
   MOE_GEMM_CASE(256, false, false, EPI_BF16)
   MOE_GEMM_CASE(256, false, false, EPI_SWIGLU)
@@ -1332,12 +1418,17 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
   MOE_GEMM_CASE(256, false, true, EPI_SWIGLU_BWD)
   MOE_GEMM_CASE(256, false, true, EPI_BF16_ADD_F32)
   MOE_GEMM_CASE(256, false, true, EPI_F32)
-  MOE_GEMM_CASE(256, true, true, EPI_F32)
+  // A stored [K][M] (MN-major): one CTA per tile only
+#define MOE_GEMM_CASE1(BN_, AMN_, BMN_, EPI_)                                              \
+  if (a.bn == BN_ && a.a_mn == AMN_ && a.b_mn == BMN_ && a.epi == EPI_ && !a.pair)        \
+    return launch_instance<BN_, AMN_, BMN_, EPI_, false>(maps, kp, tiles, st);
+  MOE_GEMM_CASE1(256, true, true, EPI_F32)
   // the remaining layouts of the test entry point
-  MOE_GEMM_CASE(256, true, false, EPI_F32)
-  MOE_GEMM_CASE(256, true, true, EPI_BF16)
-  MOE_GEMM_CASE(256, true, false, EPI_BF16)
+  MOE_GEMM_CASE1(256, true, false, EPI_F32)
+  MOE_GEMM_CASE1(256, true, true, EPI_BF16)
+  MOE_GEMM_CASE1(256, true, false, EPI_BF16)
 #undef MOE_GEMM_CASE
+#undef MOE_GEMM_CASE1
   return fail(MOE_ERR_UNSUPPORTED, "no gemm instance for this layout / epilogue");
 }
 

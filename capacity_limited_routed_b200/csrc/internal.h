@@ -78,6 +78,7 @@ struct Mat {
 // operand's K extent zero-fills the rest).
 struct GemmArgs {
   int bn = 256;
+  bool pair = false;  // 256-row tiles on a pair of CTAs (cta_group::2); not with both operands MN-major
   bool a_mn = false, b_mn = false;
   int epi = EPI_BF16;
   int M = 0, N = 0;  // per group; N counts output columns

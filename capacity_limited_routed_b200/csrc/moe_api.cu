@@ -276,7 +276,16 @@ Mat expert_mat(const Geo& g, const void* ptr, int64_t width) {
   return g.dropless ? mat(ptr, width, g.exp_rows, 1) : mat(ptr, width, g.Cr, g.E);
 }
 
+// Routed (ragged-row) GEMMs on CTA pairs.  An expert's ~341 rows fill three 128-row
+// tiles (11% padding) but two 256-row pair tiles (33% padding).  Only the capped
+// layout may take pair tiles: a dropless expert region is padded to 128 rows, and a
+// 256-row tile would reach into the next expert's rows.
+#ifndef MOE_ROUTED_PAIR
+#define MOE_ROUTED_PAIR 0
+#endif
+
 void pack_groups(const Geo& g, GemmArgs& a, const int32_t* exp_off) {
+  if (a.ragged == 1) a.pair = MOE_ROUTED_PAIR && !g.dropless;
   if (!g.dropless) return;
   a.group_off = exp_off;
   a.rows_total = g.exp_rows;
@@ -575,6 +584,7 @@ moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const uint16_t* x
   {
     ProfScope ps("fwd.lat_down", st);
     GemmArgs a;
+    a.pair = true;  // dense rows: 256-row tiles on CTA pairs
     a.M = g.T;
     a.N = p->dl;
     a.A[0] = mat(x, p->dm, g.T);
@@ -589,6 +599,7 @@ moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const uint16_t* x
   {
     ProfScope ps("fwd.router", st);
     GemmArgs a;
+    a.pair = true;  // dense rows: 256-row tiles on CTA pairs
     a.bn = 128;
     a.epi = EPI_F32;
     a.M = g.T;
@@ -629,6 +640,7 @@ moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const uint16_t* x
   {
     ProfScope ps("fwd.shared_gate_up", st);
     GemmArgs a;
+    a.pair = true;  // dense rows: 256-row tiles on CTA pairs
     a.epi = EPI_SWIGLU;
     a.M = g.T;
     a.N = static_cast<int>(SH);
@@ -647,6 +659,7 @@ moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const uint16_t* x
   {
     ProfScope ps("fwd.lat_up_shared_down", st);
     GemmArgs a;
+    a.pair = true;  // dense rows: 256-row tiles on CTA pairs
     a.epi = EPI_F32;
     a.M = g.T;
     a.N = p->dm;
@@ -710,6 +723,7 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
   {
     ProfScope ps("bwd.dr", st);
     GemmArgs a;
+    a.pair = true;  // dense rows: 256-row tiles on CTA pairs
     a.b_mn = true;
     a.M = g.T;
     a.N = p->dl;
@@ -723,6 +737,7 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
   {
     ProfScope ps("bwd.shared_dgrad_swiglu", st);
     GemmArgs a;
+    a.pair = true;  // dense rows: 256-row tiles on CTA pairs
     a.b_mn = true;
     a.epi = EPI_SWIGLU_BWD;
     a.M = g.T;
@@ -863,6 +878,7 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
   {
     ProfScope ps("bwd.router_dgrad", st);
     GemmArgs a;
+    a.pair = true;  // dense rows: 256-row tiles on CTA pairs
     a.b_mn = true;
     a.epi = EPI_BF16_ADD_F32;
     a.M = g.T;
@@ -894,6 +910,7 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
   {
     ProfScope ps("bwd.dx", st);
     GemmArgs a;
+    a.pair = true;  // dense rows: 256-row tiles on CTA pairs
     a.epi = EPI_F32;
     a.b_mn = true;
     a.M = g.T;
@@ -956,6 +973,7 @@ moe_status_t moe_gemm_bf16(int32_t M, int32_t N, int32_t K, const uint16_t* A, i
   GemmArgs a;
   a.a_mn = a_mn_major != 0;
   a.b_mn = b_mn_major != 0;
+  a.pair = !a.a_mn && M > 128;  // as the block's dense GEMMs run (A stored [M][K])
   a.epi = d_f32 ? EPI_F32 : EPI_BF16;
   a.M = M;
   a.N = N;

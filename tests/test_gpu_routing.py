@@ -153,10 +153,11 @@ def test_expert_ffn_and_combine(M, shape, skew):
         n = counts_o[e]
         if n == 0:
             continue
-        # the oracle's SwiGLU of the rows the receiver kept, bf16 hidden and output
+        # the oracle's SwiGLU of the rows the receiver kept (bf16 hidden); the device's
+        # bf16 output is held against the unrounded product, its bf16 value feeds combine
         _, _, H = O.swiglu_hidden(rows_o[e].astype(np.float64), W1[e], W3[e], O.round_bf16)
-        Yo[e, :n] = O.round_bf16(H @ W2[e].T)
-        want_all.append(Yo[e, :n])
+        want_all.append(H @ W2[e].T)
+        Yo[e, :n] = O.round_bf16(want_all[-1])
         got_all.append(Y[e, :n])
     assert_close_rms(np.concatenate(got_all), np.concatenate(want_all), what="expert_out")
     # combine, fed the oracle's own expert outputs (uploaded as bf16)
