@@ -109,7 +109,8 @@ def step_work(s, kept):
         "fwd.lat_up_shared_down": 2 * T * dm * (dl + SH),
         "bwd.dr": 2 * T * dm * dl,
         "bwd.shared_dgrad_swiglu": 2 * T * dm * SH,
-        "bwd.wgrad_lat_up_shared_down": 2 * T * dm * (dl + SH),
+        "bwd.wgrad_lat_up": 2 * T * dm * dl,
+        "bwd.wgrad_shared": 2 * T * dm * 3 * SH,
         "bwd.experts_dgrad_down": 2 * kept * dl * h,
         "bwd.experts_wgrad_down": 2 * kept * dl * h,
         "bwd.experts_dgrad_gate_up": 2 * kept * 2 * h * dl,
@@ -117,7 +118,7 @@ def step_work(s, kept):
         "bwd.router_dgrad": 2 * T * E * dl,
         "bwd.router_wgrad": 2 * T * E * dl,
         "bwd.dx": 2 * T * dm * (dl + 2 * SH),
-        "bwd.wgrad_lat_down_shared": 2 * T * dm * (dl + 2 * SH),
+        "bwd.wgrad_lat_down": 2 * T * dm * dl,
     }
     A = T * k
     w_routed = E * h * dl * 2           # one routed weight tensor, bf16
@@ -131,7 +132,8 @@ def step_work(s, kept):
         "fwd.lat_up_shared_down": T * (dl + SH) * 2 + dm * (dl + SH) * 2 + T * dm * 4,
         "bwd.dr": T * dm * 2 + dm * dl * 2 + T * dl * 2,
         "bwd.shared_dgrad_swiglu": T * dm * 2 + dm * SH * 2 + 4 * T * SH * 2,
-        "bwd.wgrad_lat_up_shared_down": T * dm * 2 + T * (dl + SH) * 2 + dm * (dl + SH) * 4,
+        "bwd.wgrad_lat_up": T * dm * 2 + T * dl * 2 + dm * dl * 4,
+        "bwd.wgrad_shared": T * dm * 2 + T * SH * 2 + dm * SH * 4 + 2 * T * SH * 2 + T * dm * 2 + 2 * SH * dm * 4,
         "bwd.experts_dgrad_down": kept * dl * 2 + w_routed + 4 * kept * h * 2,
         "bwd.experts_wgrad_down": kept * dl * 2 + kept * h * 2 + E * dl * h * 4,
         "bwd.experts_dgrad_gate_up": 2 * kept * h * 2 + 2 * w_routed + kept * dl * 2,
@@ -139,7 +141,7 @@ def step_work(s, kept):
         "bwd.router_dgrad": T * E * 2 + E * dl * 2 + T * dl * 4 + T * dl * 2,
         "bwd.router_wgrad": T * E * 2 + T * dl * 2 + E * dl * 4,
         "bwd.dx": T * (dl + 2 * SH) * 2 + dm * (dl + 2 * SH) * 2 + T * dm * 4,
-        "bwd.wgrad_lat_down_shared": T * (dl + 2 * SH) * 2 + T * dm * 2 + dm * (dl + 2 * SH) * 4,
+        "bwd.wgrad_lat_down": T * dl * 2 + T * dm * 2 + dm * dl * 4,
         # logits read, idx + gate written
         "fwd.route_topk": T * E * 4 + A * 8 + E * 4,
         # z read once, every sender-kept row written with its 16-byte header
@@ -356,6 +358,57 @@ def end_to_end(args, s, blk, x, dy, hist_plan, world, dev, barrier):
                       "(two copy streams, overlapping the neighbouring steps)"}
 
 
+def drop_sweep(weights, dev):
+    """Drop fraction against context length and capacity factor, on the device: router
+    path only (latent projection, router, top-k, slot assignment, pack) for one source of
+    T = 65,536 tokens at full width, uniform router, bias 0.  The tokens of one sequence of
+    L tokens share a component (x_t = sqrt(0.6) g_seq + sqrt(0.4) eps_t): L = 512 is the
+    skewed workload's windows, L = T one sequence per source; "independent" has none.
+    Capacity factors 1.10/1.15 (the pages'), 1.25/1.30, and dropless (no cap: its largest
+    expert load is reported instead)."""
+    import torch
+    from capacity_limited_routed_b200 import moe as M
+    from capacity_limited_routed_b200 import synth
+    T, s0 = 65536, synth.FULL
+    out = {"tokens_per_source": T, "rho": 0.6, "rows": []}
+    dl, E, k = s0.d_latent, s0.n_experts, s0.top_k
+    z = torch.empty((T, dl), dtype=torch.bfloat16, device=dev)
+    logits = torch.empty((T, E), dtype=torch.float32, device=dev)
+    bias = torch.zeros(E, dtype=torch.float32, device=dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    gate = torch.empty((T, k), dtype=torch.float32, device=dev)
+    hist = torch.empty(E, dtype=torch.int32, device=dev)
+    for L in (0, 512, 4096, 16384, 65536):
+        shape = s0.with_(T=T, window=L, rho=0.6 if L else 0.0, seed=31)
+        x = synth.make_tokens_device(shape, device=dev)["x"]
+        M.moe_gemm_bf16(T, dl, s0.d_model, x, 0, weights["w_lat_down"], 0, z)
+        M.moe_gemm_bf16(T, E, dl, z, 0, weights["w_router"], 0, logits)
+        del x
+        row = {"sequence_tokens": L or "independent"}
+        for name, cs, cr in (("caps_1.10_1.15", (110, 100), (115, 100)), ("caps_1.25_1.30", (125, 100), (130, 100))):
+            plan = M.Plan(T, s0.d_model, dl, E, k, s0.n_dest, s0.hidden_routed, s0.n_shared, s0.hidden_shared,
+                          cap_send=cs, cap_recv=cr)
+            info = plan.info
+            M.moe_route(plan, logits, bias, idx, gate, hist)
+            pools = torch.empty(info.pools_bytes // 2, dtype=torch.int16, device=dev)
+            slot = torch.empty((T, k, 2), dtype=torch.int32, device=dev)
+            stats = torch.zeros(info.stats_bytes // 4, dtype=torch.int32, device=dev)
+            ws = torch.empty(info.workspace_bytes, dtype=torch.uint8, device=dev)
+            M.moe_dispatch(plan, z, idx, pools, slot, stats, ws)
+            st = stats[:4].cpu().tolist()
+            if st[3] != 0:
+                raise RuntimeError(f"kernel status {st[3]} in the drop sweep")
+            row[name] = {"sender": st[1] / (T * k), "receiver": st[2] / (T * k)}
+            del pools, slot, stats, ws
+        h = hist.cpu().numpy()
+        row["dropless_largest_expert_load"] = int(h.max())
+        row["mean_expert_load"] = T * k / E
+        out["rows"].append(row)
+    out["note"] = ("synthetic latent correlations with an untrained router; the pages' 7% (4K) -> 40% (65K) "
+                   "comes from a trained router on real text and is not reproduced, only the direction")
+    return out
+
+
 def forward_pass(shape, weights, dev, steps, warmup):
     """Forward-only throughput of a full-width workload on weights already on the device
     (same widths): CUDA events around `steps` forward passes after `warmup` of them."""
@@ -401,6 +454,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-only", action="store_true", help="a few steps, no baseline, no e2e (for ncu)")
+    ap.add_argument("--parallelism", default="auto", choices=["auto", "ep", "replicas"],
+                    help="N > 1: expert parallelism (each rank one source and the receiver of D/N destinations, "
+                         "blocks exchanged over NCCL) or data-parallel replicas; auto = ep when D divides by N")
     ap.add_argument("--no-forward-passes", action="store_true",
                     help="skip the forward-only passes of the full and skewed workloads")
     args = ap.parse_args()
@@ -427,11 +483,27 @@ def main():
     from capacity_limited_routed_b200.parallel import global_histogram, global_tokens
 
     peaks = load_peaks()
-    inp = synth.make_inputs_device(s, device=dev, seed=s.seed + 7919 * rank)
-    blk = MoEBlock(s, device=dev, training=s.backward)
-    blk.load(inp)
+    mode = args.parallelism
+    if mode == "auto":
+        mode = "ep" if world > 1 and s.n_dest % world == 0 and not s.dropless else "replicas"
+    if mode == "ep" and world < 2:
+        mode = "replicas"
+    if mode == "ep":
+        # the same weights on every rank (one seed), each rank its own tokens
+        from capacity_limited_routed_b200.parallel import EPBlock
+        inp = synth.make_inputs_device(s, device=dev, seed=s.seed)
+        tok = synth.make_tokens_device(s, device=dev, seed=s.seed + 7919 * rank)
+        inp.update({k_: v_ for k_, v_ in tok.items() if k_ in ("x", "dy")})
+        blk = EPBlock(s, world, rank, device=dev)
+        blk.load(inp["weights"], inp["bias"], inp["logit_offset"], training=s.backward)
+        del inp["weights"]
+    else:
+        inp = synth.make_inputs_device(s, device=dev, seed=s.seed + 7919 * rank)
+        blk = MoEBlock(s, device=dev, training=s.backward)
+        blk.load(inp)
     x, dy = inp["x"], inp.get("dy")
     hist_plan = M.Plan.from_shape(s.with_(T=global_tokens(s.T))) if world > 1 else blk.plan
+    torch.cuda.synchronize()
     stream = torch.cuda.current_stream(dev)
 
     def step():
@@ -487,6 +559,13 @@ def main():
         d[0] += t
         d[1] += 1
         d[2] += n
+    if mode == "ep":
+        # rows kept by this rank's experts, and the step's drops summed over ranks
+        agg = torch.tensor([st["kept_here"], st["dropped_sender"]], dtype=torch.int64, device=dev)
+        dist.all_reduce(agg)
+        kept_all, ds_all = int(agg[0].item()), int(agg[1].item())
+        st = dict(st, kept=kept_all // world, dropped_sender=ds_all / world,
+                  dropped_receiver=(world * s.T * s.top_k - kept_all - ds_all) / world)
     kept = st["kept"]
     flops, bytes_ = step_work(s, kept)
     tc_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
@@ -495,7 +574,7 @@ def main():
     hbm = peaks["hbm_gbs"]
     kernels = {}
     for name, (tot, cnt, nl) in per.items():
-        avg = tot / cnt
+        avg = tot / args.steps  # per step (a step may launch a name more than once, e.g. per wave)
         e = {"ms": round(avg, 4), "share": round(tot / sum(v[0] for v in per.values()), 4)}
         t_tc = flops[name] / (tc_peak * 1e12) if name in flops else 0.0
         t_mem = bytes_[name] / (hbm * 1e9) if name in bytes_ else 0.0
@@ -508,17 +587,19 @@ def main():
             e["frac"] = round(max(t_tc, t_mem) / (avg * 1e-3), 3)
         kernels[name] = e
     top = max(per.items(), key=lambda kv: kv[1][0])[0]
-    avg_top = per[top][0] / per[top][1]
     kt = kernels[top]
+    per_step = per[top][1] / args.steps  # records of the top step per training step (waves: 3)
+    traffic = measured_traffic(top, s)
     if kt.get("bound") == "tensor":
         roof = {"kernel": top, "bound": "tensor", "achieved": kt["tflops"], "peak": tc_peak,
-                "unit": "TFLOP/s", "frac": round(kt["tflops"] / tc_peak, 3), "traffic": measured_traffic(top, s),
+                "unit": "TFLOP/s", "frac": round(kt["tflops"] / tc_peak, 3), "traffic": traffic,
                 "peak_kind": f"bf16_tflops_sustained ({peaks['_source']}): kernel timed inside a long step",
-                "flops_per_launch": flops[top]}
+                "flops_per_launch": flops[top] / per_step, "launches_per_step": per_step}
     else:
         roof = {"kernel": top, "bound": "hbm", "achieved": kt.get("gbs"), "peak": hbm,
-                "unit": "GB/s", "frac": round((kt.get("gbs") or 0) / hbm, 3), "traffic": measured_traffic(top, s),
-                "peak_kind": f"hbm_gbs ({peaks['_source']})", "bytes_per_launch": bytes_.get(top)}
+                "unit": "GB/s", "frac": round((kt.get("gbs") or 0) / hbm, 3), "traffic": traffic,
+                "peak_kind": f"hbm_gbs ({peaks['_source']})", "bytes_per_launch": bytes_.get(top, 0) / per_step,
+                "launches_per_step": per_step}
     fwd_ms = sum(v[0] for k_, v in per.items() if k_.startswith("fwd.") or k_.startswith("experts.")) / args.steps
     step_ms = ms_max / args.steps
     value = world * s.T / (step_ms * 1e-3)
@@ -534,6 +615,7 @@ def main():
             (s.d_model, s.d_latent, s.n_experts, s.hidden_routed) == (6144, 3072, 384, 3072):
         for name, shape in (("fwd_full", synth.FULL), ("fwd_skewed", synth.SKEWED)):
             fwd_extra[name] = forward_pass(shape, blk.weights, dev, args.steps, max(args.warmup, 3))
+        fwd_extra["drop_sweep"] = drop_sweep(blk.weights, dev)
         torch.cuda.synchronize()
 
     # ---------------- CPU oracle baseline (rank 0, N = 1 only)
@@ -552,7 +634,11 @@ def main():
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": describe(s), "parallelism": f"replicas x{world} (one source per GPU)",
+            "config": {"workload": describe(s),
+                       "parallelism": (f"expert parallelism x{world} (each GPU one source of T tokens and the "
+                                       f"receiver of {s.n_dest // world} destinations; fixed-shape blocks per wave "
+                                       f"over NCCL)" if mode == "ep" else
+                                       f"replicas x{world} (one source per GPU)"),
                        "l2": "inputs larger than L2 (22 GB of expert weights streamed every step)"},
             "fwd_tokens_per_s": world * s.T / (fwd_ms * 1e-3) if fwd_ms > 0 else None,
             "fwd_tokens_per_s_kind": "sum of the forward steps' CUDA-event times inside the timed training steps",

@@ -64,7 +64,28 @@ struct KParams {
   const float* addend;
   long long add_ld;
   int32_t* status;
+  // rows gathered by index (receiver-side rows read straight from the pools): row r of
+  // group g is row gather_rows[base_g + r] of the 2-D source tensor, base_g = group_off[g]
+  // (packed) or g * gather_ld; rows at or past the group's row count read gather_zero,
+  // an all-zero row of the source
+  const int32_t* gather_rows;
+  long long gather_ld;
+  int gather_zero;
+  // group g of the launch is expert (g / map_p) * map_l + map_off + g % map_p (map_p = 0:
+  // expert g); one wave's experts are one launch of D * P groups
+  int map_p, map_l, map_off;
 };
+
+__device__ __forceinline__ int expert_of(const KParams& p, int g) {
+  return p.map_p > 0 ? (g / p.map_p) * p.map_l + p.map_off + g % p.map_p : g;
+}
+
+// source row of row r of group g for a gathered operand (the zero row past the group's rows)
+__device__ __forceinline__ int gather_src_row(const KParams& p, int g, long long base, int nrows, int r) {
+  if (r >= nrows) return p.gather_zero;
+  const int v = p.gather_rows[base + r];
+  return (v >= 0 && v <= p.gather_zero) ? v : p.gather_zero;
+}
 
 // Tuning of the weight-gradient (write-bound) instance: pipeline stages and staging
 // buffers per epilogue warp.
@@ -173,6 +194,7 @@ struct Sched {
       return r;
     }
     decode(t, r.g, r.m, r.n);
+    r.g = expert_of(p, r.g);  // from here on the group is the expert
     r.kb = k_blocks(r.g);
     r.off = p.group_off != nullptr ? p.group_off[r.g] : 0;
     return r;
@@ -251,7 +273,7 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
     for (int i = 0; i < per; ++i) {
       const int g = g0 + i;
       if (g < p.groups) {
-        int r = p.group_rows[g];
+        int r = p.group_rows[expert_of(p, g)];
         r = r < 0 ? 0 : (r > p.M ? p.M : r);
         local += ((r + TM - 1) / TM) * nt;
       }
@@ -273,7 +295,7 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
       const int g = g0 + i;
       if (g < p.groups) {
         prefix[g] = run;
-        int r = p.group_rows[g];
+        int r = p.group_rows[expert_of(p, g)];
         r = r < 0 ? 0 : (r > p.M ? p.M : r);
         run += ((r + TM - 1) / TM) * nt;
       }
@@ -288,8 +310,74 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
   const volatile int* abort_v = abort_flag;
 
   Sched<BN, EPI, TM> sc(p, prefix);
+  // both CTAs of a pair walk the same tiles: tile slots are per CTA, or per pair for PAIR
+  const int slot0 = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int nslots = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
-  if (warp == 0) {
+  bool gathered = false;  // A rows gathered by index (K-major A, one CTA per tile)
+  if constexpr (!A_MN && !PAIR) gathered = p.gather_rows != nullptr;
+  if (warp == 0 && gathered) {
+    // ---------------------------------------------------------------- TMA producer, gathered A
+    // The whole warp loads: lane l gathers rows 4l..4l+3 of the tile's 128 A rows with one
+    // tile::gather4 per k-block (the same rows for every k-block of the tile); lane 0 waits
+    // for the stage, arms its barrier and loads B as a tile.
+    int stage = 0;
+    uint32_t phase = 0;
+    int armed_phase[C::kStages];
+    for (int s = 0; s < C::kStages; ++s) armed_phase[s] = -1;
+    bool ok = true;
+    Tile nxt = sc.tile(slot0);
+    for (int t = slot0; ok && t < sc.total; t += nslots) {
+      const Tile cur = nxt;
+      nxt = sc.tile(t + nslots);
+      const int g = cur.g, mt = cur.m, ntile = cur.n, kb_total = cur.kb;
+      int nrows = p.group_rows != nullptr ? p.group_rows[g] : p.M;
+      nrows = nrows < 0 ? 0 : (nrows > p.M ? p.M : nrows);
+      const long long base = p.group_off != nullptr ? static_cast<long long>(p.group_off[g])
+                                                    : static_cast<long long>(g) * p.gather_ld;
+      int src[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) src[j] = gather_src_row(p, g, base, nrows, mt * kBM + 4 * lane + j);
+      for (int kb = 0; kb < kb_total; ++kb) {
+        bool w = true;
+        if (lane == 0) w = mbar_wait(&empty[stage], phase ^ 1u, abort_v);
+        if (!__shfl_sync(0xffffffffu, w, 0)) {
+          ok = false;
+          break;
+        }
+        const int k0 = kb * kBK;  // one K segment
+        uint8_t* sa = smem + stage * C::kStage;
+        uint8_t* sb = sa + C::kABytes;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[stage], C::kStage);
+          armed_phase[stage] = static_cast<int>(phase);
+          if (EPI == EPI_SWIGLU) {
+            const int n0 = ntile * (BN / 2);
+            tma_load_3d(&maps.b[0], sb, &full[stage], k0, n0, g);
+            tma_load_3d(&maps.bv, sb + (BN / 2) * 128, &full[stage], k0, n0, g);
+          } else if (!B_MN) {
+            tma_load_3d(&maps.b[0], sb, &full[stage], k0, ntile * BN, g);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_3d(&maps.b[0], sb + j * 8192, &full[stage], ntile * BN + 64 * j, k0, g);
+          }
+        }
+        __syncwarp();
+        tma_gather4(&maps.a[0], sa + lane * 512, &full[stage], k0, src[0], src[1], src[2], src[3]);
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      record_status(p.status, MOE_ERR_TIMEOUT);
+      for (int s = 0; s < C::kStages; ++s)
+        if (armed_phase[s] >= 0) mbar_wait(&full[s], static_cast<uint32_t>(armed_phase[s]), nullptr, 50000000ull);
+    }
+  } else if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       int stage = 0;
@@ -297,10 +385,10 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
       int armed_phase[C::kStages];
       for (int s = 0; s < C::kStages; ++s) armed_phase[s] = -1;
       bool ok = true;
-      Tile nxt = sc.tile(blockIdx.x);
-      for (int t = blockIdx.x; ok && t < sc.total; t += gridDim.x) {
+      Tile nxt = sc.tile(slot0);
+      for (int t = slot0; ok && t < sc.total; t += nslots) {
         const Tile cur = nxt;
-        nxt = sc.tile(t + gridDim.x);  // issued a tile ahead: its count load overlaps this tile
+        nxt = sc.tile(t + nslots);  // issued a tile ahead: its count load overlaps this tile
         const int g = cur.g, mt = cur.m, ntile = cur.n, kb_total = cur.kb;
         // packed activations: 2-D tensors, rows offset by the group's first row
         const int gz = p.group_off != nullptr ? 0 : g, gro = cur.off;
@@ -380,10 +468,10 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       bool issued = false;
-      Tile nxt = sc.tile(blockIdx.x);
-      for (int t = blockIdx.x; ok && t < sc.total; t += gridDim.x) {
+      Tile nxt = sc.tile(slot0);
+      for (int t = slot0; ok && t < sc.total; t += nslots) {
         const Tile cur = nxt;
-        nxt = sc.tile(t + gridDim.x);
+        nxt = sc.tile(t + nslots);
         const int kb_total = cur.kb;
         if (kb_total == 0) continue;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_v)) {
@@ -455,10 +543,10 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
     int ring = 0;        // next staging buffer of this warp
     uint32_t eph = 0;    // SwiGLU backward: parity of each of this warp's three load barriers
     int eslot = 0;       // SwiGLU backward: slot of the next live chunk
-    Tile nxt = sc.tile(blockIdx.x);
-    for (int t = blockIdx.x; t < sc.total; t += gridDim.x) {
+    Tile nxt = sc.tile(slot0);
+    for (int t = slot0; t < sc.total; t += nslots) {
       const Tile cur = nxt;
-      nxt = sc.tile(t + gridDim.x);
+      nxt = sc.tile(t + nslots);
       const int g = cur.g, mt = cur.m, ntile = cur.n, kb_total = cur.kb;
         // packed activations: 2-D tensors, rows offset by the group's first row
         const int gz = p.group_off != nullptr ? 0 : g, gro = cur.off;
@@ -863,6 +951,48 @@ __device__ __forceinline__ void pair_drain(const TmaMaps& maps, const KParams& p
   }
 }
 
+#ifndef MOE_WB_DIRECT
+#define MOE_WB_DIRECT 0
+#endif
+
+// The same share drained straight to global memory: per 16-row half and 64 columns, one
+// 16x256b TMEM load (a thread holds two rows, two adjacent columns of each 8-column group)
+// and st.global.v2 stores, each instruction writing eight whole 32-byte sectors; the next
+// load is in flight while the current registers are stored.  No shared-memory staging.
+__device__ __forceinline__ void pair_drain_direct(const KParams& p, uint32_t tbase, int col_lo, int ntile, int row0,
+                                                  int g, int lane) {
+  float* obase = static_cast<float*>(p.out) + static_cast<long long>(g) * p.out_gs;
+  const int rq = lane >> 2, cq = 2 * (lane & 3);
+  uint32_t r[2][32];
+  auto issue = [&](int it, uint32_t (&dst)[32]) {
+    const int h = it >> 1, c = col_lo + 64 * (it & 1);
+    tmem_ld_16x256b_x8_async(tbase + (static_cast<uint32_t>(16 * h) << 16) + static_cast<uint32_t>(c), dst);
+  };
+  issue(0, r[0]);
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    tmem_wait_ld();
+    if (it + 1 < 4) issue(it + 1, r[(it + 1) & 1]);
+    const int h = it >> 1, c = col_lo + 64 * (it & 1);
+    const int ra = row0 + 16 * h + rq, rb = ra + 8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int col = ntile * 256 + c + 8 * i + cq;
+      if (col < p.N) {
+        const uint32_t* v = &r[it & 1][4 * i];
+        if (ra < p.M)
+          asm volatile("st.global.v2.b32 [%0], {%1, %2};" ::"l"(obase + static_cast<long long>(ra) * p.ldo + col),
+                       "r"(v[0]), "r"(v[1])
+                       : "memory");
+        if (rb < p.M)
+          asm volatile("st.global.v2.b32 [%0], {%1, %2};" ::"l"(obase + static_cast<long long>(rb) * p.ldo + col),
+                       "r"(v[2]), "r"(v[3])
+                       : "memory");
+      }
+    }
+  }
+}
+
 // the same share of a tile whose contraction is empty: zeros
 __device__ __forceinline__ void pair_zero(const KParams& p, int col_lo, int ntile, int row0, int g, int lane) {
   float* obase = static_cast<float*>(p.out) + static_cast<long long>(g) * p.out_gs;
@@ -949,13 +1079,73 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       const int l = t - r.g * per_group;
       r.n = l % nt_n;
       r.m = l / nt_n;
+      r.g = expert_of(p, r.g);
       r.kb = k_blocks(r.g);
       r.off = p.group_off != nullptr ? p.group_off[r.g] : 0;
     }
     return r;
   };
 
-  if (warp == 0) {
+  if (warp == 0 && p.gather_rows != nullptr) {
+    // ------------------------------------------------------------ TMA producer, gathered B (both CTAs)
+    // B's K rows are the group's rows gathered by index: per k-block this CTA's 128 columns
+    // of B are two 64-column boxes of 64 K rows; lane l gathers K rows 4(l%16)..+3 of box
+    // l/16 with one tile::gather4.  Lane 0 waits for the stage and loads A as tiles.
+    int stage = 0;
+    uint32_t phase = 0;
+    int armed_phase[C::kStages];
+    for (int s = 0; s < C::kStages; ++s) armed_phase[s] = -1;
+    bool ok = true;
+    PairTile nxt = fetch(pair);
+    const int box = lane >> 4, kr = 4 * (lane & 15);
+    for (int t = pair; ok && t < total; t += npairs) {
+      const PairTile cur = nxt;
+      nxt = fetch(t + npairs);
+      const int g = cur.g, mt = cur.m, ntile = cur.n, kb_total = cur.kb;
+      const int gz = p.group_off != nullptr ? 0 : g, gro = cur.off;
+      int nrows = p.ragged == 2 ? p.group_rows[g] : kb_total * kBK;
+      nrows = nrows < 0 ? 0 : nrows;
+      const long long base = p.group_off != nullptr ? static_cast<long long>(p.group_off[g])
+                                                    : static_cast<long long>(g) * p.gather_ld;
+      const int m0 = mt * 256 + 128 * static_cast<int>(rank);
+      const int n0 = ntile * 256 + 128 * static_cast<int>(rank);
+      for (int kb = 0; kb < kb_total; ++kb) {
+        bool w = true;
+        if (lane == 0) w = mbar_wait(&empty[stage], phase ^ 1u, abort_v);
+        if (!__shfl_sync(0xffffffffu, w, 0)) {
+          ok = false;
+          break;
+        }
+        const uint32_t bar = leader_addr(smem_u32(&full[stage]));
+        uint8_t* sa = smem + stage * C::kStage;
+        uint8_t* sb = sa + C::kABytes;
+        const int k0 = kb * kBK;
+        if (lane == 0) {
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kStage);
+          armed_phase[stage] = static_cast<int>(phase);
+          tma_load_3d_pair(&maps.a[0], sa, bar, m0, gro + k0, gz);
+          tma_load_3d_pair(&maps.a[0], sa + 8192, bar, m0 + 64, gro + k0, gz);
+        }
+        __syncwarp();
+        int src[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) src[j] = gather_src_row(p, g, base, nrows, k0 + kr + j);
+        tma_gather4_pair(&maps.b[0], sb + box * 8192 + (lane & 15) * 512, bar, n0 + 64 * box, src[0], src[1], src[2],
+                         src[3]);
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      record_status(p.status, MOE_ERR_TIMEOUT);
+      if (leader)
+        for (int s = 0; s < C::kStages; ++s)
+          if (armed_phase[s] >= 0) mbar_wait(&full[s], static_cast<uint32_t>(armed_phase[s]), nullptr, 50000000ull);
+    }
+  } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
       int stage = 0;
@@ -1100,8 +1290,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         break;
       }
       tc_fence_after();
-      pair_drain(maps, p, tmem_base + lane_off + static_cast<uint32_t>(acc * 256), col_lo, ntile, row0, g, buf,
-                 row_addr, lane);
+      if (MOE_WB_DIRECT)
+        pair_drain_direct(p, tmem_base + lane_off + static_cast<uint32_t>(acc * 256), col_lo, ntile, row0, g, lane);
+      else
+        pair_drain(maps, p, tmem_base + lane_off + static_cast<uint32_t>(acc * 256), col_lo, ntile, row0, g, buf,
+                   row_addr, lane);
       __syncwarp();
       tc_fence_before();
       // hand the accumulator back to the leader's MMA warp
@@ -1168,6 +1361,27 @@ moe_status_t make_map(CUtensorMap* m, const Mat& t, uint32_t box_inner, uint32_t
 
 // tiles: output tiles of the launch (pair tiles for PAIR); the grid is one CTA (or pair)
 // per tile up to what fits on the device at once
+// 2-D map of a gather source: boxes one row high and 64 bf16 columns wide (tile::gather4)
+moe_status_t make_gather_map(CUtensorMap* m, const Mat& t) {
+  if (t.ptr == nullptr) return fail(MOE_ERR_INVALID_ARG, "gather source is null");
+  if ((reinterpret_cast<uintptr_t>(t.ptr) & 15) != 0 || t.inner <= 0 || t.rows <= 1 || t.ld < t.inner ||
+      (t.ld * 2) % 16 != 0 || t.inner % 64 != 0)
+    return fail(MOE_ERR_INVALID_ARG, "gather source has a bad shape, stride or alignment");
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(t.inner), static_cast<cuuint64_t>(t.rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(t.ld * 2)};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(t.ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the gather source (" +
+                                  std::to_string(static_cast<int>(r)) + ")");
+  return MOE_OK;
+}
+
 template <int BN, bool A_MN, bool B_MN, int EPI, bool PAIR>
 moe_status_t launch_instance(const TmaMaps& maps, const KParams& kp, long long tiles, cudaStream_t st) {
   auto kern = gemm_kernel<BN, A_MN, B_MN, EPI, PAIR>;
@@ -1272,7 +1486,18 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
   if (a.a_mn && a.b_mn && a.ragged == 1)
     return fail(MOE_ERR_UNSUPPORTED, "gemm with both operands MN-major takes no ragged rows");
   if (a.out == nullptr) return fail(MOE_ERR_INVALID_ARG, "gemm output is null");
+  const bool gather = a.gather_rows != nullptr;
+  // gathered A: one-CTA tiles, A stored [M][K], one K segment, ragged rows; gathered B:
+  // the CTA-pair weight gradient (both operands [K][.], float32 out)
+  const bool gather_a = gather && !a.a_mn;
+  const bool gather_b = gather && a.a_mn;
+  if (gather_a && (a.pair || a.nseg != 1 || a.ragged != 1))
+    return fail(MOE_ERR_UNSUPPORTED, "a gathered A takes one-CTA tiles, one K segment and ragged rows");
+  if (gather_b && !(a.b_mn && a.epi == EPI_F32 && a.nseg == 1 && a.ragged == 2 && a.bn == 256))
+    return fail(MOE_ERR_UNSUPPORTED, "a gathered B takes the ragged-K weight-gradient form");
 
+  // groups of the output and element-wise tensors (a launch may cover some of them)
+  const int tgroups = a.tensor_groups > 0 ? a.tensor_groups : a.groups;
   TmaMaps maps;
   memset(&maps, 0, sizeof(maps));
   KParams kp;
@@ -1286,11 +1511,11 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
   kp.nseg = a.nseg;
   for (int s = 0; s < a.nseg; ++s) {
     moe_status_t r;
-    r = make_map(&maps.a[s], a.A[s], 64, a.a_mn ? 64 : 128, "A");
+    r = gather_a ? make_gather_map(&maps.a[s], a.gather_src) : make_map(&maps.a[s], a.A[s], 64, a.a_mn ? 64 : 128, "A");
     if (r != MOE_OK) return r;
     // a pair CTA loads half of B's rows (SwiGLU: the gate or the value half)
     const uint32_t b_rows = a.b_mn ? 64 : ((a.epi == EPI_SWIGLU || a.pair) ? a.bn / 2 : a.bn);
-    r = make_map(&maps.b[s], a.B[s], 64, b_rows, "B");
+    r = gather_b ? make_gather_map(&maps.b[s], a.gather_src) : make_map(&maps.b[s], a.B[s], 64, b_rows, "B");
     if (r != MOE_OK) return r;
     kp.seg_kb[s] = a.ragged == 2 ? 0 : static_cast<int>((a.K[s] + kBK - 1) / kBK);
   }
@@ -1305,9 +1530,9 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
       o.ptr = ptr;
       o.inner = a.N;
       o.rows = packed ? a.rows_total : a.M;
-      o.groups = packed ? 1 : a.groups;
+      o.groups = packed ? 1 : tgroups;
       o.ld = ld;
-      o.gs = (a.groups > 1 && !packed) ? gs : ld * o.rows;
+      o.gs = (tgroups > 1 && !packed) ? gs : ld * o.rows;
       return make_map(m, o, 32, 32, what, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, CU_TENSOR_MAP_SWIZZLE_64B);
     };
     moe_status_t r = tile(&maps.out, a.out, a.ldo, a.out_gs, "output");
@@ -1324,9 +1549,9 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
         o.ptr = ptr;
         o.inner = a.N;
         o.rows = packed ? a.rows_total : a.M;
-        o.groups = packed ? 1 : a.groups;
+        o.groups = packed ? 1 : tgroups;
         o.ld = ld;
-        o.gs = (a.groups > 1 && !packed) ? gs : ld * o.rows;
+        o.gs = (tgroups > 1 && !packed) ? gs : ld * o.rows;
         return make_map(m, o, 16, 32, what, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, CU_TENSOR_MAP_SWIZZLE_NONE);
       };
       if ((r = tile16(&maps.out, a.out, a.ldo, a.out_gs, "dA")) != MOE_OK) return r;
@@ -1342,9 +1567,9 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
     // a packed ragged-row output is 2-D; a weight gradient's output stays one per group
     const bool packed_out = packed && a.ragged == 1;
     o.rows = packed_out ? a.rows_total : a.M;
-    o.groups = packed_out ? 1 : a.groups;
+    o.groups = packed_out ? 1 : tgroups;
     o.ld = a.ldo;
-    o.gs = (a.groups > 1 && !packed_out) ? a.out_gs : a.ldo * o.rows;
+    o.gs = (tgroups > 1 && !packed_out) ? a.out_gs : a.ldo * o.rows;
     moe_status_t r = a.epi == EPI_F32
                          ? make_map(&maps.out, o, 32, 32, "output", CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4)
                          : make_map(&maps.out, o, 64, 32, "output");
@@ -1365,6 +1590,12 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
   kp.addend = a.addend;
   kp.add_ld = a.add_ld;
   kp.status = a.status;
+  kp.gather_rows = a.gather_rows;
+  kp.gather_ld = a.gather_ld;
+  kp.gather_zero = gather ? static_cast<int>(a.gather_src.rows - 1) : 0;
+  kp.map_p = a.map_p;
+  kp.map_l = a.map_l;
+  kp.map_off = a.map_off;
 
   if (a.a_mn && a.b_mn && a.epi == EPI_F32 && a.nseg == 1 && a.ragged != 1 && a.bn == 256) {
     const long long pair_tiles =

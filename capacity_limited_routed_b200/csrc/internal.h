@@ -107,6 +107,19 @@ struct GemmArgs {
   const float* addend = nullptr;
   int64_t add_ld = 0;
   int32_t* status = nullptr;
+  // A gathered operand: rows chosen by index from a 2-D source tensor whose last row is
+  // all zeros.  One-CTA GEMMs with A stored [M][K] gather A's rows (gather_src inner =
+  // K); CTA-pair weight gradients gather B's K rows (gather_src inner = N).  Row r of
+  // group g is source row gather_rows[group_off[g] + r] (packed) or
+  // gather_rows[g * gather_ld + r]; rows at or past the group's count read the zero row.
+  const int32_t* gather_rows = nullptr;
+  int64_t gather_ld = 0;
+  Mat gather_src;
+  // launch group g is expert (g / map_p) * map_l + map_off + g % map_p (map_p = 0: g):
+  // one wave's D * P experts as one launch; tensors stay indexed by expert and hold
+  // tensor_groups groups (0: groups)
+  int map_p = 0, map_l = 0, map_off = 0;
+  int tensor_groups = 0;
 };
 
 moe_status_t gemm_run(const GemmArgs& a, cudaStream_t stream);
@@ -142,23 +155,33 @@ moe_status_t launch_pack(const Geo& g, const uint16_t* z, const int32_t* idx, co
 moe_status_t launch_offsets(const int32_t* counts, int n, int align, int32_t* off, cudaStream_t st);
 // scratch ints needed by the receiver's row map
 size_t unpack_scratch_ints(const Geo& g);
+// Receiver side: ranks the rows of every pool by their packed ids and writes, for each
+// expert row, the pool row it came from (src, indexed like the expert buffers).
 // capacity layout: pool_off = exp_off = nullptr.  Dropless: pool_off / pool_fill give
 // each pool's packed row range; exp_off (E+1 ints) is computed here from the counts.
-moe_status_t launch_unpack(const Geo& g, const uint16_t* pools, uint16_t* xe, int32_t* rows, int32_t* row_map,
+// id_base: the packed (global) expert id of this receiver's expert 0 (expert parallelism)
+moe_status_t launch_unpack(const Geo& g, const uint16_t* pools, int32_t* src, int32_t* rows, int32_t* row_map,
                            int32_t* status, cudaStream_t st, const int32_t* pool_off = nullptr,
-                           const int32_t* pool_fill = nullptr, int32_t* exp_off = nullptr);
+                           const int32_t* pool_fill = nullptr, int32_t* exp_off = nullptr, int id_base = 0);
+// rows between a receiver's pool positions and its expert rows by the row map (see map_rows_kernel)
+moe_status_t launch_map_rows(const uint16_t* in, uint16_t* out, const int32_t* map, const uint16_t* hdr_pools,
+                             int hdr_ld, int hdr_col, long long n_rows, int width, long long ld_pool, bool to_pools,
+                             cudaStream_t st);
 moe_status_t launch_zero_tail_rows(const Geo& g, uint16_t* buf, int64_t width, const int32_t* rows,
                                    cudaStream_t st, const int32_t* exp_off = nullptr);
 // exp_off: row of each expert's first row in the expert buffers (dropless); nullptr:
-// expert e's rows start at e * C_r
+// expert e's rows start at e * C_r.  by_pool: the expert rows are the ones receivers sent
+// back under expert parallelism, laid out like the pools (row pool(e) * C_s + sender slot,
+// receiver-dropped rows zero), and an assignment counts as kept when its sender kept it.
 moe_status_t launch_combine(const Geo& g, const uint16_t* ye, const float* gate, const int32_t* idx,
-                            const int32_t* slot, uint16_t* r, cudaStream_t st, const int32_t* exp_off = nullptr);
+                            const int32_t* slot, uint16_t* r, cudaStream_t st, const int32_t* exp_off = nullptr,
+                            bool by_pool = false);
 moe_status_t launch_combine_bwd(const Geo& g, const uint16_t* dr, const uint16_t* ye, const float* gate,
                                 const int32_t* idx, const int32_t* slot, uint16_t* dye, float* dg,
-                                cudaStream_t st, const int32_t* exp_off = nullptr);
+                                cudaStream_t st, const int32_t* exp_off = nullptr, bool by_pool = false);
 moe_status_t launch_undispatch(const Geo& g, const uint16_t* dxe, const float* gate, const float* dg,
                                const int32_t* idx, const int32_t* slot, float* dz_routed, uint16_t* dlogits,
-                               cudaStream_t st, const int32_t* exp_off = nullptr);
+                               cudaStream_t st, const int32_t* exp_off = nullptr, bool by_pool = false);
 moe_status_t launch_bias_update(const Geo& g, const int32_t* hist, float* bias, float step, cudaStream_t st);
 
 // plan geometry and the device check, for entry points defined in other files

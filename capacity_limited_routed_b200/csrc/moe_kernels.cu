@@ -12,7 +12,9 @@
 //   pack            sender: z rows into the fixed pools with the expert id in a 16-byte row
 //                   header (same page, §2: one pool per receiving GPU, ids in the payload)
 //   unpack          receiver: reads only the pools; ranks rows of each local expert by the
-//                   packed id, keeps the first C_r, gathers them per expert
+//                   packed id, keeps the first C_r, and records for each expert row the
+//                   pool row it came from (the expert GEMMs gather their rows from the
+//                   pools by these indices)
 //   combine         r_t = sum_j kept g_tj Y[e_tj][rslot_tj], fixed j order, fp32 accumulation
 //   combine_bwd     dY = g dr on kept rows, dg = <dr, Y>
 //   undispatch      dz_routed = sum_j kept dX, and the softmax backward to the logits
@@ -497,7 +499,7 @@ __global__ void pack_empty_headers(const int32_t* __restrict__ pool_fill, int NP
 __global__ void unpack_rank_kernel(const uint16_t* __restrict__ pools, int Cs, int Cr, int dl, int L, int P, int W,
                                    int32_t* __restrict__ row_map, int32_t* __restrict__ rows_out,
                                    int32_t* __restrict__ status, const int32_t* __restrict__ pool_off,
-                                   const int32_t* __restrict__ pool_fill, int S) {
+                                   const int32_t* __restrict__ pool_fill, int S, int id_base) {
   constexpr int kTile = 256;
   __shared__ int s_warp_cnt[kTile / 32][32];
   __shared__ int s_run[32];
@@ -521,8 +523,10 @@ __global__ void unpack_rank_kernel(const uint16_t* __restrict__ pools, int Cs, i
       const int r = r0 + threadIdx.x;
       int q = -1;
       if (r < nrows) {
-        const int e = *reinterpret_cast<const int*>(pbase + r * row_elems + dl);
-        if (e >= 0) {
+        // packed ids are global; a receiver of experts [id_base, ...) numbers them from 0
+        const int eg = *reinterpret_cast<const int*>(pbase + r * row_elems + dl);
+        const int e = eg >= 0 ? eg - id_base : -1;
+        if (eg >= 0) {
           if (e >= e_first && e < e_first + P) q = e - e_first;
           else atomicCAS(status, 0, MOE_ERR_INVALID_ARG);  // an id this pool cannot hold
         }
@@ -555,16 +559,15 @@ __global__ void unpack_rank_kernel(const uint16_t* __restrict__ pools, int Cs, i
   if (threadIdx.x < P) rows_out[e_first + threadIdx.x] = packed ? s_run[threadIdx.x] : min(s_run[threadIdx.x], Cr);
 }
 
-// receiver, pass 2: one warp per pool row, up to 8 vectors per lane in flight
-__global__ void unpack_copy_kernel(const uint16_t* __restrict__ pools, const int32_t* __restrict__ row_map,
-                                   long long n_rows, int dl, uint16_t* __restrict__ xe,
-                                   const int32_t* __restrict__ exp_off, int E) {
-  const int lane = threadIdx.x & 31;
-  const int warps = blockDim.x >> 5;
+// receiver, pass 2: one thread per pool row.  A kept row's receive-buffer row d (e * C_r +
+// slot, or exp_off[e] + slot for packed buffers) records the pool row it came from:
+// src[d] = pool row.  The expert GEMMs gather their input rows through src.
+__global__ void unpack_index_kernel(const uint16_t* __restrict__ pools, const int32_t* __restrict__ row_map,
+                                    long long n_rows, int dl, int32_t* __restrict__ src,
+                                    const int32_t* __restrict__ exp_off, int E) {
   const long long row_elems = dl + 8;
-  const int nvec = dl / 8;
-  for (long long r = static_cast<long long>(blockIdx.x) * warps + (threadIdx.x >> 5); r < n_rows;
-       r += static_cast<long long>(gridDim.x) * warps) {
+  for (long long r = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; r < n_rows;
+       r += static_cast<long long>(gridDim.x) * blockDim.x) {
     long long d = row_map[r];
     if (d < 0) continue;
     if (exp_off != nullptr) {  // packed buffers: the row map holds the slot within the expert
@@ -572,16 +575,37 @@ __global__ void unpack_copy_kernel(const uint16_t* __restrict__ pools, const int
       if (e < 0 || e >= E) continue;
       d += exp_off[e];
     }
-    const uint4* src = reinterpret_cast<const uint4*>(pools + r * row_elems);
-    uint4* dst = reinterpret_cast<uint4*>(xe + d * dl);
-    for (int v0 = lane; v0 < nvec; v0 += 32 * 8) {
-      uint4 val[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (v0 + 32 * u < nvec) val[u] = src[v0 + 32 * u];
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = val[u];
+    src[d] = static_cast<int32_t>(r);
+  }
+}
+
+// Rows between pool positions and expert rows under expert parallelism, one warp per pool
+// row r of a receiver (its G sources' pools, in order), map[r] = expert row or -1:
+//   to_pools: out[r] = in[map[r]] (expert row sent back to its pool position), zeros for a
+//             receiver-dropped row; rows whose pool header says empty are not written
+//             (their source never reads them)
+//   else:     out[map[r]] = in[r] (a received row placed in its expert's buffer)
+// Rows are `width` bf16 wide; pool-side rows have stride ld_pool, expert rows `width`.
+__global__ void map_rows_kernel(const uint16_t* __restrict__ in, uint16_t* __restrict__ out,
+                                const int32_t* __restrict__ map, const uint16_t* __restrict__ hdr_pools,
+                                int hdr_ld, int hdr_col, long long n_rows, int width, long long ld_pool,
+                                int to_pools) {
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  const int nvec = width / 8;
+  for (long long r = static_cast<long long>(blockIdx.x) * warps + (threadIdx.x >> 5); r < n_rows;
+       r += static_cast<long long>(gridDim.x) * warps) {
+    const long long d = map[r];
+    if (to_pools) {
+      if (*reinterpret_cast<const int*>(hdr_pools + r * hdr_ld + hdr_col) < 0) continue;  // empty pool row
+      uint4* dst = reinterpret_cast<uint4*>(out + r * ld_pool);
+      const uint4* src = reinterpret_cast<const uint4*>(in + (d >= 0 ? d : 0) * width);
+      for (int v = lane; v < nvec; v += 32) dst[v] = d >= 0 ? src[v] : make_uint4(0, 0, 0, 0);
+    } else {
+      if (d < 0) continue;
+      const uint4* src = reinterpret_cast<const uint4*>(in + r * ld_pool);
+      uint4* dst = reinterpret_cast<uint4*>(out + d * width);
+      for (int v = lane; v < nvec; v += 32) dst[v] = src[v];
     }
   }
 }
@@ -603,6 +627,26 @@ __global__ void zero_tail_rows_kernel(uint16_t* __restrict__ buf, long long widt
 }
 
 // ---------------------------------------------------------------------- combine and its backward
+
+// Where the expert row of an assignment lives.  Receiver side (one GPU): expert e's rows
+// start at e * C_r (or exp_off[e], packed) and the row is the receiver slot.  Source side
+// under expert parallelism: the rows the receivers sent back sit in pool order, row
+// pool(e) * C_s + sender slot, and a receiver-dropped row comes back as zeros.
+struct RowAddr {
+  int Cr;
+  const int32_t* exp_off;
+  int by_pool;
+  int Cs, L, P, W;
+};
+
+__device__ __forceinline__ long long row_of(const RowAddr& ra, int e, const int32_t* slot_pair) {
+  if (ra.by_pool) {
+    const int s = slot_pair[0];
+    return (s >= 0 && s < ra.Cs) ? static_cast<long long>(pool_of(e, ra.L, ra.P, ra.W)) * ra.Cs + s : -1;
+  }
+  const int rs = slot_pair[1];
+  return (rs >= 0 && rs < ra.Cr) ? exp_row0(e, ra.Cr, ra.exp_off) + rs : -1;
+}
 
 __device__ __forceinline__ void acc8(float (&acc)[8], const uint4& v, float g) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -632,7 +676,7 @@ constexpr int kCombRows = 8;
 
 __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ ye, const float* __restrict__ gate,
                                const int32_t* __restrict__ idx, const int32_t* __restrict__ slot, int T, int k,
-                               int dl, int Cr, int E, uint16_t* __restrict__ r, const int32_t* __restrict__ exp_off) {
+                               int dl, int E, uint16_t* __restrict__ r, const RowAddr ra) {
   __shared__ long long s_row[8][32];
   __shared__ float s_g[8][32];
   const int lane = threadIdx.x & 31;
@@ -642,11 +686,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
   for (int t = blockIdx.x * warps + wib; t < T; t += gridDim.x * warps) {
     if (lane < k) {
       const long long a = static_cast<long long>(t) * k + lane;
-      const int rs = slot[2 * a + 1];
       const int e = idx[a];
-      const bool ok = rs >= 0 && rs < Cr && e >= 0 && e < E;
-      s_row[wib][lane] = ok ? exp_row0(e, Cr, exp_off) + rs : -1;
-      s_g[wib][lane] = ok ? gate[a] : 0.0f;
+      const long long row = (e >= 0 && e < E) ? row_of(ra, e, slot + 2 * a) : -1;
+      s_row[wib][lane] = row;
+      s_g[wib][lane] = row >= 0 ? gate[a] : 0.0f;
     }
     __syncwarp();
     for (int v0 = lane; v0 < nvec; v0 += 32 * kCombVpl) {
@@ -691,9 +734,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
 // the eight partial dot products stay in registers until the row is done.
 __global__ void __launch_bounds__(256) combine_bwd_kernel(const uint16_t* __restrict__ dr, const uint16_t* __restrict__ ye,
                                    const float* __restrict__ gate, const int32_t* __restrict__ idx,
-                                   const int32_t* __restrict__ slot, int T, int k, int dl, int Cr, int E,
-                                   uint16_t* __restrict__ dye, float* __restrict__ dg,
-                                   const int32_t* __restrict__ exp_off) {
+                                   const int32_t* __restrict__ slot, int T, int k, int dl, int E,
+                                   uint16_t* __restrict__ dye, float* __restrict__ dg, const RowAddr ra) {
   __shared__ long long s_row[8][32];
   __shared__ float s_g[8][32];
   const int lane = threadIdx.x & 31;
@@ -703,11 +745,10 @@ __global__ void __launch_bounds__(256) combine_bwd_kernel(const uint16_t* __rest
   for (int t = blockIdx.x * warps + wib; t < T; t += gridDim.x * warps) {
     if (lane < k) {
       const long long a = static_cast<long long>(t) * k + lane;
-      const int rs = slot[2 * a + 1];
       const int e = idx[a];
-      const bool ok = rs >= 0 && rs < Cr && e >= 0 && e < E;
-      s_row[wib][lane] = ok ? exp_row0(e, Cr, exp_off) + rs : -1;
-      s_g[wib][lane] = ok ? gate[a] : 0.0f;
+      const long long row = (e >= 0 && e < E) ? row_of(ra, e, slot + 2 * a) : -1;
+      s_row[wib][lane] = row;
+      s_g[wib][lane] = row >= 0 ? gate[a] : 0.0f;
     }
     __syncwarp();
     const uint4* drow = reinterpret_cast<const uint4*>(dr + static_cast<long long>(t) * dl);
@@ -781,9 +822,8 @@ __global__ void __launch_bounds__(256) combine_bwd_kernel(const uint16_t* __rest
 // chosen experts, zero elsewhere
 __global__ void undispatch_kernel(const uint16_t* __restrict__ dxe, const float* __restrict__ gate,
                                   const float* __restrict__ dg, const int32_t* __restrict__ idx,
-                                  const int32_t* __restrict__ slot, int T, int k, int dl, int Cr, int E,
-                                  float* __restrict__ dz, uint16_t* __restrict__ dlogits,
-                                  const int32_t* __restrict__ exp_off) {
+                                  const int32_t* __restrict__ slot, int T, int k, int dl, int E,
+                                  float* __restrict__ dz, uint16_t* __restrict__ dlogits, const RowAddr ra) {
   __shared__ long long s_row[8][32];
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
@@ -794,12 +834,11 @@ __global__ void undispatch_kernel(const uint16_t* __restrict__ dxe, const float*
     int e_j = -1;
     if (lane < k) {
       const long long a = static_cast<long long>(t) * k + lane;
-      const int rs = slot[2 * a + 1];
       e_j = idx[a];
       g_j = gate[a];
       dg_j = dg[a];
       if (e_j < 0 || e_j >= E) e_j = -1;
-      s_row[wib][lane] = (rs >= 0 && rs < Cr && e_j >= 0) ? exp_row0(e_j, Cr, exp_off) + rs : -1;
+      s_row[wib][lane] = e_j >= 0 ? row_of(ra, e_j, slot + 2 * a) : -1;
     }
     __syncwarp();
     for (int v = lane; v < nvec; v += 64) {
@@ -983,6 +1022,11 @@ moe_status_t launch_slot_scan(const Geo& g, const int32_t* idx, int32_t* slot, i
 
 moe_status_t launch_pack(const Geo& g, const uint16_t* z, const int32_t* idx, const int32_t* slot,
                          int32_t* stats, uint16_t* pools, cudaStream_t st, const int32_t* pool_off) {
+  // the trailing all-zero row after the pools (the receiver's padding rows read it)
+  {
+    const cudaError_t e = cudaMemsetAsync(pools + g.pool_rows * (g.dl + 8), 0, sizeof(uint16_t) * (g.dl + 8), st);
+    if (e != cudaSuccess) return cuda_check(e, "pools zero row");
+  }
   if (g.T > 0) {
     // two row buffers per warp; rows too wide for that take the register path
     const size_t smem = static_cast<size_t>(kPackWarps) * 2 * g.dl * 2;
@@ -1024,23 +1068,34 @@ moe_status_t launch_offsets(const int32_t* counts, int n, int align, int32_t* of
   return cuda_check(cudaGetLastError(), "offsets");
 }
 
-moe_status_t launch_unpack(const Geo& g, const uint16_t* pools, uint16_t* xe, int32_t* rows, int32_t* row_map,
+moe_status_t launch_unpack(const Geo& g, const uint16_t* pools, int32_t* src, int32_t* rows, int32_t* row_map,
                            int32_t* status, cudaStream_t st, const int32_t* pool_off, const int32_t* pool_fill,
-                           int32_t* exp_off) {
+                           int32_t* exp_off, int id_base) {
   if (g.P > 32) return fail(MOE_ERR_UNSUPPORTED, "more than 32 experts per wave");
   const bool packed = pool_off != nullptr;
   if (packed && (pool_fill == nullptr || exp_off == nullptr))
     return fail(MOE_ERR_INVALID_ARG, "packed pools need their fills and the expert offsets");
   unpack_rank_kernel<<<g.NP, 256, 0, st>>>(pools, g.Cs, g.Cr, g.dl, g.L, g.P, g.W, row_map, rows, status, pool_off,
-                                           pool_fill, g.S);
+                                           pool_fill, g.S, id_base);
   count_launch();
   if (packed) MOE_TRY_K(launch_offsets(rows, g.E, 128, exp_off, st));
   const long long n_rows = g.pool_rows;
-  const int warps = 8;
-  unpack_copy_kernel<<<blocks_for(n_rows, warps), 32 * warps, 0, st>>>(pools, row_map, n_rows, g.dl, xe,
-                                                                       packed ? exp_off : nullptr, g.E);
+  unpack_index_kernel<<<blocks_for(n_rows, 256), 256, 0, st>>>(pools, row_map, n_rows, g.dl, src,
+                                                               packed ? exp_off : nullptr, g.E);
   count_launch();
   return cuda_check(cudaGetLastError(), "unpack");
+}
+
+moe_status_t launch_map_rows(const uint16_t* in, uint16_t* out, const int32_t* map, const uint16_t* hdr_pools,
+                             int hdr_ld, int hdr_col, long long n_rows, int width, long long ld_pool, bool to_pools,
+                             cudaStream_t st) {
+  if (n_rows <= 0) return MOE_OK;
+  if (width % 8 != 0 || ld_pool % 8 != 0) return fail(MOE_ERR_INVALID_ARG, "row mover needs 16-byte rows");
+  const int warps = 8;
+  map_rows_kernel<<<blocks_for(n_rows, warps), 32 * warps, 0, st>>>(in, out, map, hdr_pools, hdr_ld, hdr_col, n_rows,
+                                                                    width, ld_pool, to_pools ? 1 : 0);
+  count_launch();
+  return cuda_check(cudaGetLastError(), "map rows");
 }
 
 moe_status_t launch_zero_tail_rows(const Geo& g, uint16_t* buf, int64_t width, const int32_t* rows,
@@ -1051,34 +1106,50 @@ moe_status_t launch_zero_tail_rows(const Geo& g, uint16_t* buf, int64_t width, c
   return cuda_check(cudaGetLastError(), "zero tail rows");
 }
 
+namespace {
+RowAddr row_addr(const Geo& g, const int32_t* exp_off, bool by_pool) {
+  RowAddr ra;
+  ra.Cr = g.Cr;
+  ra.exp_off = exp_off;
+  ra.by_pool = by_pool ? 1 : 0;
+  ra.Cs = g.Cs;
+  ra.L = g.L;
+  ra.P = g.P;
+  ra.W = g.W;
+  return ra;
+}
+}  // namespace
+
 moe_status_t launch_combine(const Geo& g, const uint16_t* ye, const float* gate, const int32_t* idx,
-                            const int32_t* slot, uint16_t* r, cudaStream_t st, const int32_t* exp_off) {
+                            const int32_t* slot, uint16_t* r, cudaStream_t st, const int32_t* exp_off,
+                            bool by_pool) {
   if (g.T == 0) return MOE_OK;
   const int warps = 8;
-  combine_kernel<<<blocks_for(g.T, warps), 32 * warps, 0, st>>>(ye, gate, idx, slot, g.T, g.k, g.dl, g.Cr, g.E, r,
-                                                                exp_off);
+  combine_kernel<<<blocks_for(g.T, warps), 32 * warps, 0, st>>>(ye, gate, idx, slot, g.T, g.k, g.dl, g.E, r,
+                                                                row_addr(g, exp_off, by_pool));
   count_launch();
   return cuda_check(cudaGetLastError(), "combine");
 }
 
 moe_status_t launch_combine_bwd(const Geo& g, const uint16_t* dr, const uint16_t* ye, const float* gate,
                                 const int32_t* idx, const int32_t* slot, uint16_t* dye, float* dg,
-                                cudaStream_t st, const int32_t* exp_off) {
+                                cudaStream_t st, const int32_t* exp_off, bool by_pool) {
   if (g.T == 0) return MOE_OK;
   const int warps = 8;
   combine_bwd_kernel<<<blocks_for(g.T, warps), 32 * warps, 0, st>>>(dr, ye, gate, idx, slot, g.T, g.k, g.dl,
-                                                                    g.Cr, g.E, dye, dg, exp_off);
+                                                                    g.E, dye, dg, row_addr(g, exp_off, by_pool));
   count_launch();
   return cuda_check(cudaGetLastError(), "combine_bwd");
 }
 
 moe_status_t launch_undispatch(const Geo& g, const uint16_t* dxe, const float* gate, const float* dg,
                                const int32_t* idx, const int32_t* slot, float* dz_routed, uint16_t* dlogits,
-                               cudaStream_t st, const int32_t* exp_off) {
+                               cudaStream_t st, const int32_t* exp_off, bool by_pool) {
   if (g.T == 0) return MOE_OK;
   const int warps = 8;
-  undispatch_kernel<<<blocks_for(g.T, warps), 32 * warps, 0, st>>>(dxe, gate, dg, idx, slot, g.T, g.k, g.dl, g.Cr,
-                                                                   g.E, dz_routed, dlogits, exp_off);
+  undispatch_kernel<<<blocks_for(g.T, warps), 32 * warps, 0, st>>>(dxe, gate, dg, idx, slot, g.T, g.k, g.dl,
+                                                                   g.E, dz_routed, dlogits,
+                                                                   row_addr(g, exp_off, by_pool));
   count_launch();
   return cuda_check(cudaGetLastError(), "undispatch");
 }

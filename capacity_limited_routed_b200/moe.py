@@ -18,7 +18,8 @@ EXPORTS = (
     "moe_plan_create", "moe_plan_destroy", "moe_plan_info", "moe_route", "moe_dispatch", "moe_dispatch_noalloc",
     "moe_expert_ffn", "moe_combine", "moe_forward", "moe_backward", "moe_bias_update",
     "moe_saved_view", "moe_gemm_bf16", "moe_profile_start", "moe_profile_stop", "moe_kernel_launches",
-    "moe_last_error",
+    "moe_last_error", "moe_ep_view", "moe_ep_forward_send", "moe_ep_forward_experts", "moe_ep_forward_combine",
+    "moe_ep_backward_send", "moe_ep_backward_experts", "moe_ep_backward_finish",
 )
 
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
@@ -35,7 +36,7 @@ class moe_config_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "T", "d_model", "d_latent", "n_experts", "top_k", "n_dest", "n_waves", "hidden_routed",
         "n_shared", "hidden_shared", "cap_send_num", "cap_send_den", "cap_recv_num", "cap_recv_den",
-        "n_sources")]
+        "n_sources", "ep_ranks", "ep_rank")]
 
 
 class moe_plan_info_t(ctypes.Structure):
@@ -68,7 +69,15 @@ class moe_profile_record_t(ctypes.Structure):
 
 class moe_saved_view_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
-        "z", "logits", "topk_idx", "topk_gate", "slot", "expert_rows", "expert_in", "expert_out", "r")]
+        "z", "logits", "topk_idx", "topk_gate", "slot", "expert_rows", "pools", "expert_src", "expert_out",
+        "r")]
+
+
+class moe_ep_view_t(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("ranks", "rank", "dest_per_rank", "n_waves", "cap_send",
+                                                "pool_row_elems", "row_elems")] + \
+               [(n, ctypes.c_void_p) for n in ("send_pools", "recv_pools", "y_send", "y_recv", "dy_send", "dy_recv",
+                                                "dx_send", "dx_recv", "expert_rows", "topk_idx", "slot")]
 
 
 def _load():
@@ -93,6 +102,14 @@ def _load():
         "moe_gemm_bf16": [I, I, I, P, I, P, I, P, I, P, P],
         "moe_profile_start": [],
         "moe_profile_stop": [ctypes.POINTER(moe_profile_record_t), I, ctypes.POINTER(I)],
+        "moe_ep_view": [P, P, P, ctypes.POINTER(moe_ep_view_t)],
+        "moe_ep_forward_send": [P, ctypes.POINTER(moe_weights_t), P, P, P, P, P, P, S, P],
+        "moe_ep_forward_experts": [P, ctypes.POINTER(moe_expert_weights_t), P, P, P, S, P],
+        "moe_ep_forward_combine": [P, ctypes.POINTER(moe_weights_t), P, P, P, S, P],
+        "moe_ep_backward_send": [P, ctypes.POINTER(moe_weights_t), P, P, P, ctypes.POINTER(moe_grads_t), P, S, P],
+        "moe_ep_backward_experts": [P, ctypes.POINTER(moe_expert_weights_t), P, ctypes.POINTER(moe_grads_t), P, S,
+                                    P],
+        "moe_ep_backward_finish": [P, ctypes.POINTER(moe_weights_t), P, P, P, ctypes.POINTER(moe_grads_t), P, S, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -153,10 +170,10 @@ class Plan:
     """Owns a moe_plan_t for one block shape."""
 
     def __init__(self, T, d_model, d_latent, n_experts, top_k, n_dest, hidden_routed, n_shared, hidden_shared,
-                 n_waves=3, cap_send=(110, 100), cap_recv=(115, 100), n_sources=1):
+                 n_waves=3, cap_send=(110, 100), cap_recv=(115, 100), n_sources=1, ep_ranks=0, ep_rank=0):
         self.cfg = moe_config_t(T, d_model, d_latent, n_experts, top_k, n_dest, n_waves, hidden_routed,
                                 n_shared, hidden_shared, cap_send[0], cap_send[1], cap_recv[0], cap_recv[1],
-                                n_sources)
+                                n_sources, ep_ranks, ep_rank)
         h = ctypes.c_void_p()
         _check(_lib.moe_plan_create(ctypes.byref(self.cfg), ctypes.byref(h)), "moe_plan_create")
         self.handle = h
@@ -165,11 +182,11 @@ class Plan:
         self.info = PlanInfo(**{f: getattr(info, f) for f, _ in moe_plan_info_t._fields_})
 
     @classmethod
-    def from_shape(cls, s):
+    def from_shape(cls, s, ep_ranks=0, ep_rank=0):
         # both capacity numerators 0 select the dropless variant
         cap_send, cap_recv = ((0, 1), (0, 1)) if getattr(s, "dropless", False) else (s.cap_send, s.cap_recv)
         return cls(s.T, s.d_model, s.d_latent, s.n_experts, s.top_k, s.n_dest, s.hidden_routed, s.n_shared,
-                   s.hidden_shared, s.n_waves, cap_send, cap_recv, getattr(s, "n_sources", 1))
+                   s.hidden_shared, s.n_waves, cap_send, cap_recv, getattr(s, "n_sources", 1), ep_ranks, ep_rank)
 
     def __del__(self):
         # at interpreter shutdown the module globals may already be gone
@@ -269,3 +286,61 @@ def moe_kernel_launches() -> int:
 
 def moe_last_error() -> str:
     return _lib.moe_last_error().decode(errors="replace")
+
+
+# ------------------------------------------------------------------ expert parallelism
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
+def _grads_or_null(g: dict) -> moe_grads_t:
+    return moe_grads_t(*[_ptr(g.get(n)) for n in _W])
+
+
+def moe_ep_view(plan: Plan, saved, ws) -> moe_ep_view_t:
+    v = moe_ep_view_t()
+    _check(_lib.moe_ep_view(plan.handle, _ptr(saved), _ptr(ws), ctypes.byref(v)), "moe_ep_view")
+    return v
+
+
+def moe_ep_forward_send(plan: Plan, weights: dict, x, bias, logit_offset, stats, saved, ws, stream=None):
+    w_ = weights_struct(weights)
+    _check(_lib.moe_ep_forward_send(plan.handle, ctypes.byref(w_), _ptr(x), _ptr(bias), _ptr(logit_offset),
+                                    _ptr(stats), _ptr(saved), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "moe_ep_forward_send")
+
+
+def moe_ep_forward_experts(plan: Plan, w1, w3, w2, stats, saved, ws, stream=None):
+    ew = moe_expert_weights_t(_ptr(w1), _ptr(w3), _ptr(w2))
+    _check(_lib.moe_ep_forward_experts(plan.handle, ctypes.byref(ew), _ptr(stats), _ptr(saved), _ptr(ws),
+                                       _nbytes(ws), _stream(stream)), "moe_ep_forward_experts")
+
+
+def moe_ep_forward_combine(plan: Plan, weights: dict, y, saved, ws, stream=None):
+    w_ = weights_struct(weights)
+    _check(_lib.moe_ep_forward_combine(plan.handle, ctypes.byref(w_), _ptr(y), _ptr(saved), _ptr(ws), _nbytes(ws),
+                                       _stream(stream)), "moe_ep_forward_combine")
+
+
+def moe_ep_backward_send(plan: Plan, weights: dict, saved, x, dy, grads: dict, ws, stream=None):
+    w_ = weights_struct(weights)
+    g_ = _grads_or_null(grads)
+    _check(_lib.moe_ep_backward_send(plan.handle, ctypes.byref(w_), _ptr(saved), _ptr(x), _ptr(dy), ctypes.byref(g_),
+                                     _ptr(ws), _nbytes(ws), _stream(stream)), "moe_ep_backward_send")
+
+
+def moe_ep_backward_experts(plan: Plan, w1, w3, w2, saved, grads: dict, ws, stream=None):
+    ew = moe_expert_weights_t(_ptr(w1), _ptr(w3), _ptr(w2))
+    g_ = _grads_or_null(grads)
+    _check(_lib.moe_ep_backward_experts(plan.handle, ctypes.byref(ew), _ptr(saved), ctypes.byref(g_), _ptr(ws),
+                                        _nbytes(ws), _stream(stream)), "moe_ep_backward_experts")
+
+
+def moe_ep_backward_finish(plan: Plan, weights: dict, saved, x, dx, grads: dict, ws, stream=None):
+    w_ = weights_struct(weights)
+    g_ = _grads_or_null(grads)
+    _check(_lib.moe_ep_backward_finish(plan.handle, ctypes.byref(w_), _ptr(saved), _ptr(x), _ptr(dx),
+                                       ctypes.byref(g_), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "moe_ep_backward_finish")

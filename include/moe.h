@@ -97,6 +97,15 @@ typedef struct {
                            * ranhao.site, §3.1 topology; lamjinlab.com §2 caps per pool).
                            * Pools are source-major; a destination's receiver reads its
                            * pools source by source.  T/S must be a multiple of 32. */
+  /* Expert parallelism over ep_ranks GPUs (0 or 1: none), this GPU being rank ep_rank:
+   * every rank is one source of T tokens and the receiver of destinations
+   * [ep_rank * D/G, (ep_rank + 1) * D/G), i.e. of experts [ep_rank * E/G, ...), with
+   * G = ep_ranks ("Marin 535B-A23B：一场完全公开的前沿 MoE 训练直播", §3.1 topology and
+   * §3.2: 64-way expert parallelism, six experts per GPU, one fixed-shape exchange per
+   * wave).  Sender caps use this rank's T; receiver caps all ranks' tokens,
+   * C_r = ceil(1.15 * G*T*k / E).  EP plans run through the moe_ep_* calls only. */
+  int32_t ep_ranks;
+  int32_t ep_rank;
 } moe_config_t;
 
 typedef struct moe_plan* moe_plan_t;
@@ -109,7 +118,8 @@ typedef struct {
   int32_t cap_send;          /* C_s, rows of one pool (0: dropless) */
   int32_t cap_recv;          /* C_r, rows of one expert (0: dropless) */
   int32_t pool_row_elems;    /* bf16 elements per pool row: d_latent payload + 8 header */
-  uint64_t pools_bytes;      /* [D*W][C_s][pool_row_elems] bf16 (dropless: [T*k][...]) */
+  uint64_t pools_bytes;      /* [D*W][C_s][pool_row_elems] bf16 (dropless: [T*k][...]) and one
+                              * trailing all-zero row, written by moe_dispatch */
   uint64_t expert_out_bytes; /* [E][C_r][d_latent] bf16 (dropless: [T*k + 127*E][...]) */
   uint64_t slot_bytes;       /* [T][k][2] int32 */
   uint64_t stats_bytes;      /* moe_stats_t + per-expert and per-pool counters */
@@ -166,7 +176,10 @@ typedef struct {
   const float* topk_gate;     /* [T][k] */
   const int32_t* slot;        /* [T][k][2]: sender slot, receiver slot (-1 = dropped) */
   const int32_t* expert_rows; /* [E] rows each expert received (<= C_r) */
-  const uint16_t* expert_in;  /* [E][C_r][d_latent] bf16, receiver-side rows */
+  const uint16_t* pools;      /* [n_pools * C_s + 1][d_latent + 8] bf16, as dispatched (the last
+                               * row all zeros); the experts read their input rows from here */
+  const int32_t* expert_src;  /* [E][C_r] int32: pool row of each expert row (rows below the
+                               * expert's count; the rest unspecified) */
   const uint16_t* expert_out; /* [E][C_r][d_latent] bf16 */
   const uint16_t* r;          /* [T][d_latent] bf16, combined routed output */
 } moe_saved_view_t;
@@ -198,7 +211,8 @@ MOE_API moe_status_t moe_route(moe_plan_t plan, const float* logits, const float
  * order, then packing of z rows into the fixed pools.
  *   z [T][d_latent] bf16 device; topk_idx [T][k] int32 device;
  *   pools [D*W][C_s][d_latent + 8] bf16 device: row = payload, then a 16-byte header
- *     whose first int32 is the global expert id (-1 for an empty row);
+ *     whose first int32 is the global expert id (-1 for an empty row); one more row
+ *     after the last pool is written all zeros (pools_bytes counts it);
  *   slot [T][k][2] int32 device: (sender slot | -1, receiver slot | -1);
  *   stats: stats buffer (device), counters overwritten (hist left as is);
  *   ws: scratch of ws_bytes >= workspace_bytes.
@@ -237,7 +251,9 @@ MOE_API moe_status_t moe_dispatch_noalloc(moe_plan_t plan, const uint16_t* z, co
  * MoE-модели с 535 млрд параметров", §2: the receiver learns each row's expert from
  * the id in the payload, with no separate count or metadata exchange;
  * "Marin 535B-A23B：一场完全公开的前沿 MoE 训练直播", §2.2: SwiGLU experts of width 3072.)
- *   pools as written by moe_dispatch; expert_out [E][C_r][d_latent] bf16 device
+ *   pools as written by moe_dispatch (with its trailing all-zero row: the expert GEMMs
+ *   read their input rows straight from the pools by row index, and padding rows read
+ *   the zero row); expert_out [E][C_r][d_latent] bf16 device
  *   (rows at and past the expert's row count are zero or unspecified);
  *   expert_rows [E] int32 device, rows each expert received (may be NULL). */
 MOE_API moe_status_t moe_expert_ffn(moe_plan_t plan, const moe_expert_weights_t* w,
@@ -288,6 +304,74 @@ MOE_API moe_status_t moe_backward(moe_plan_t plan, const moe_weights_t* w, const
  * outside backpropagation.) */
 MOE_API moe_status_t moe_bias_update(moe_plan_t plan, const int32_t* hist, float* bias, float step,
                              void* stream);
+
+/* ---------------------------------------------------------------- expert parallelism
+ *
+ * A plan with ep_ranks = G >= 2 makes this GPU rank ep_rank of G: one source of T tokens
+ * and the receiver of destinations [rank * D/G, (rank + 1) * D/G), i.e. of experts
+ * [rank * E/G, (rank + 1) * E/G).  ("Marin начинает открытое обучение MoE-модели с 535 млрд
+ * параметров", §2: one fixed pool per receiving GPU, three waves of identical shape, ids
+ * in the payload, no count or metadata exchange; "Marin 535B-A23B：一场完全公开的前沿 MoE
+ * 训练直播", §3.1 topology and §3.2 three-wave buffers.)  A training step is six calls
+ * with an exchange of fixed-shape blocks between consecutive ones, which the caller makes
+ * (capacity_limited_routed_b200/parallel.py uses NCCL send/recv):
+ *
+ *   moe_ep_forward_send      x -> send pools (router, top-k, sender slots, pack)
+ *     exchange 1: pools      send_pools -> every rank's recv_pools
+ *   moe_ep_forward_experts   recv pools -> this rank's experts -> y rows to send back
+ *     exchange 2: y rows     y_send -> every source's y_recv
+ *   moe_ep_forward_combine   y rows -> y (combine, up-projection, shared experts)
+ *   moe_ep_backward_send     dy -> dY rows to send, dW_up, shared gradients
+ *     exchange 3: dY rows    dy_send -> every rank's dy_recv
+ *   moe_ep_backward_experts  dY rows -> this rank's expert gradients -> dX rows to send back
+ *     exchange 4: dX rows    dx_send -> every source's dx_recv
+ *   moe_ep_backward_finish   dX rows -> dx, dW_router, dW_lat_down
+ *
+ * Blocks.  Every exchange buffer holds D*W blocks of C_s rows (pools: d_latent + 8
+ * elements per row, the others d_latent), block b = (a * D/G + d) * W + w for peer a,
+ * local destination d < D/G and wave w.  In every exchange a rank sends block b of its
+ * send buffer to peer a and receives block b of its receive buffer from peer a; wave w
+ * may travel as soon as it is ready.  The receiving side sees its blocks source-major,
+ * so its receiver walks sources in rank order (the virtual-sources layout, n_sources).
+ * Receiver-dropped rows travel back as zeros.  A forward on G ranks gives the results of
+ * a one-GPU forward with n_sources = G over all ranks' tokens in rank order.
+ *
+ * Buffers: saved and ws have the sizes moe_plan_info reports for the EP plan; the same
+ * saved and ws go to all six calls of a step (the backward keeps state in ws from its
+ * first call to its last).  Expert weights and gradients are this rank's E/G experts. */
+typedef struct {
+  int32_t ranks, rank, dest_per_rank, n_waves, cap_send;
+  int32_t pool_row_elems;     /* d_latent + 8 */
+  int32_t row_elems;          /* d_latent */
+  uint16_t* send_pools;       /* [D*W*C_s][d_latent + 8] bf16 (ws), then one zero row */
+  uint16_t* recv_pools;       /* [D*W*C_s][d_latent + 8] bf16 (saved): blocks from every source */
+  uint16_t* y_send;           /* [D*W*C_s][d_latent] (ws): expert outputs back to their sources */
+  uint16_t* y_recv;           /* [D*W*C_s][d_latent] (saved): this source's rows back */
+  uint16_t* dy_send;          /* [D*W*C_s][d_latent] (ws) */
+  uint16_t* dy_recv;          /* [D*W*C_s][d_latent] (ws) */
+  uint16_t* dx_send;          /* [D*W*C_s][d_latent] (ws) */
+  uint16_t* dx_recv;          /* [D*W*C_s][d_latent] (ws) */
+  int32_t* expert_rows;       /* [E/G] (saved): rows this rank's experts kept */
+  int32_t* topk_idx;          /* [T][k] (saved): this source's choices */
+  int32_t* slot;              /* [T][k][2] (saved): sender slot (receiver slots live at the receivers) */
+} moe_ep_view_t;
+
+MOE_API moe_status_t moe_ep_view(moe_plan_t plan, void* saved, void* ws, moe_ep_view_t* out);
+MOE_API moe_status_t moe_ep_forward_send(moe_plan_t plan, const moe_weights_t* w, const uint16_t* x,
+                                         const float* bias, const float* logit_offset, void* stats, void* saved,
+                                         void* ws, size_t ws_bytes, void* stream);
+MOE_API moe_status_t moe_ep_forward_experts(moe_plan_t plan, const moe_expert_weights_t* w, void* stats, void* saved,
+                                            void* ws, size_t ws_bytes, void* stream);
+MOE_API moe_status_t moe_ep_forward_combine(moe_plan_t plan, const moe_weights_t* w, float* y, void* saved, void* ws,
+                                            size_t ws_bytes, void* stream);
+MOE_API moe_status_t moe_ep_backward_send(moe_plan_t plan, const moe_weights_t* w, const void* saved,
+                                          const uint16_t* x, const uint16_t* dy, const moe_grads_t* grads, void* ws,
+                                          size_t ws_bytes, void* stream);
+MOE_API moe_status_t moe_ep_backward_experts(moe_plan_t plan, const moe_expert_weights_t* w, const void* saved,
+                                             const moe_grads_t* grads, void* ws, size_t ws_bytes, void* stream);
+MOE_API moe_status_t moe_ep_backward_finish(moe_plan_t plan, const moe_weights_t* w, const void* saved,
+                                            const uint16_t* x, float* dx, const moe_grads_t* grads, void* ws,
+                                            size_t ws_bytes, void* stream);
 
 /* Pointers into a forward context written by moe_forward (no device access). */
 MOE_API moe_status_t moe_saved_view(moe_plan_t plan, const void* saved, moe_saved_view_t* out);
