@@ -118,9 +118,7 @@ class MoEBlock:
             "topk_gate": view(v["topk_gate"], (T, k), torch.float32),
             "slot": view(v["slot"], (T, k, 2), torch.int32),
             "expert_rows": view(v["expert_rows"], (E,), torch.int32),
-            "pools": view(v["pools"], (self.plan.info.pools_bytes // (2 * (s.d_latent + 8)), s.d_latent + 8),
-                          torch.bfloat16),
-            "expert_src": view(v["expert_src"], (E, Cr), torch.int32),
+            "expert_in": view(v["expert_in"], (E, Cr, s.d_latent), torch.bfloat16),
             "expert_out": view(v["expert_out"], (E, Cr, s.d_latent), torch.bfloat16),
             "r": view(v["r"], (T, s.d_latent), torch.bfloat16),
         }

@@ -64,13 +64,6 @@ struct KParams {
   const float* addend;
   long long add_ld;
   int32_t* status;
-  // rows gathered by index (receiver-side rows read straight from the pools): row r of
-  // group g is row gather_rows[base_g + r] of the 2-D source tensor, base_g = group_off[g]
-  // (packed) or g * gather_ld; rows at or past the group's row count read gather_zero,
-  // an all-zero row of the source
-  const int32_t* gather_rows;
-  long long gather_ld;
-  int gather_zero;
   // group g of the launch is expert (g / map_p) * map_l + map_off + g % map_p (map_p = 0:
   // expert g); one wave's experts are one launch of D * P groups
   int map_p, map_l, map_off;
@@ -78,13 +71,6 @@ struct KParams {
 
 __device__ __forceinline__ int expert_of(const KParams& p, int g) {
   return p.map_p > 0 ? (g / p.map_p) * p.map_l + p.map_off + g % p.map_p : g;
-}
-
-// source row of row r of group g for a gathered operand (the zero row past the group's rows)
-__device__ __forceinline__ int gather_src_row(const KParams& p, int g, long long base, int nrows, int r) {
-  if (r >= nrows) return p.gather_zero;
-  const int v = p.gather_rows[base + r];
-  return (v >= 0 && v <= p.gather_zero) ? v : p.gather_zero;
 }
 
 // Tuning of the weight-gradient (write-bound) instance: pipeline stages and staging
@@ -314,70 +300,7 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
   const int slot0 = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   const int nslots = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
-  bool gathered = false;  // A rows gathered by index (K-major A, one CTA per tile)
-  if constexpr (!A_MN && !PAIR) gathered = p.gather_rows != nullptr;
-  if (warp == 0 && gathered) {
-    // ---------------------------------------------------------------- TMA producer, gathered A
-    // The whole warp loads: lane l gathers rows 4l..4l+3 of the tile's 128 A rows with one
-    // tile::gather4 per k-block (the same rows for every k-block of the tile); lane 0 waits
-    // for the stage, arms its barrier and loads B as a tile.
-    int stage = 0;
-    uint32_t phase = 0;
-    int armed_phase[C::kStages];
-    for (int s = 0; s < C::kStages; ++s) armed_phase[s] = -1;
-    bool ok = true;
-    Tile nxt = sc.tile(slot0);
-    for (int t = slot0; ok && t < sc.total; t += nslots) {
-      const Tile cur = nxt;
-      nxt = sc.tile(t + nslots);
-      const int g = cur.g, mt = cur.m, ntile = cur.n, kb_total = cur.kb;
-      int nrows = p.group_rows != nullptr ? p.group_rows[g] : p.M;
-      nrows = nrows < 0 ? 0 : (nrows > p.M ? p.M : nrows);
-      const long long base = p.group_off != nullptr ? static_cast<long long>(p.group_off[g])
-                                                    : static_cast<long long>(g) * p.gather_ld;
-      int src[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) src[j] = gather_src_row(p, g, base, nrows, mt * kBM + 4 * lane + j);
-      for (int kb = 0; kb < kb_total; ++kb) {
-        bool w = true;
-        if (lane == 0) w = mbar_wait(&empty[stage], phase ^ 1u, abort_v);
-        if (!__shfl_sync(0xffffffffu, w, 0)) {
-          ok = false;
-          break;
-        }
-        const int k0 = kb * kBK;  // one K segment
-        uint8_t* sa = smem + stage * C::kStage;
-        uint8_t* sb = sa + C::kABytes;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&full[stage], C::kStage);
-          armed_phase[stage] = static_cast<int>(phase);
-          if (EPI == EPI_SWIGLU) {
-            const int n0 = ntile * (BN / 2);
-            tma_load_3d(&maps.b[0], sb, &full[stage], k0, n0, g);
-            tma_load_3d(&maps.bv, sb + (BN / 2) * 128, &full[stage], k0, n0, g);
-          } else if (!B_MN) {
-            tma_load_3d(&maps.b[0], sb, &full[stage], k0, ntile * BN, g);
-          } else {
-#pragma unroll
-            for (int j = 0; j < BN / 64; ++j)
-              tma_load_3d(&maps.b[0], sb + j * 8192, &full[stage], ntile * BN + 64 * j, k0, g);
-          }
-        }
-        __syncwarp();
-        tma_gather4(&maps.a[0], sa + lane * 512, &full[stage], k0, src[0], src[1], src[2], src[3]);
-        if (++stage == C::kStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
-      }
-    }
-    if (!ok && lane == 0) {
-      *abort_flag = 1;
-      record_status(p.status, MOE_ERR_TIMEOUT);
-      for (int s = 0; s < C::kStages; ++s)
-        if (armed_phase[s] >= 0) mbar_wait(&full[s], static_cast<uint32_t>(armed_phase[s]), nullptr, 50000000ull);
-    }
-  } else if (warp == 0) {
+  if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       int stage = 0;
@@ -1086,66 +1009,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     return r;
   };
 
-  if (warp == 0 && p.gather_rows != nullptr) {
-    // ------------------------------------------------------------ TMA producer, gathered B (both CTAs)
-    // B's K rows are the group's rows gathered by index: per k-block this CTA's 128 columns
-    // of B are two 64-column boxes of 64 K rows; lane l gathers K rows 4(l%16)..+3 of box
-    // l/16 with one tile::gather4.  Lane 0 waits for the stage and loads A as tiles.
-    int stage = 0;
-    uint32_t phase = 0;
-    int armed_phase[C::kStages];
-    for (int s = 0; s < C::kStages; ++s) armed_phase[s] = -1;
-    bool ok = true;
-    PairTile nxt = fetch(pair);
-    const int box = lane >> 4, kr = 4 * (lane & 15);
-    for (int t = pair; ok && t < total; t += npairs) {
-      const PairTile cur = nxt;
-      nxt = fetch(t + npairs);
-      const int g = cur.g, mt = cur.m, ntile = cur.n, kb_total = cur.kb;
-      const int gz = p.group_off != nullptr ? 0 : g, gro = cur.off;
-      int nrows = p.ragged == 2 ? p.group_rows[g] : kb_total * kBK;
-      nrows = nrows < 0 ? 0 : nrows;
-      const long long base = p.group_off != nullptr ? static_cast<long long>(p.group_off[g])
-                                                    : static_cast<long long>(g) * p.gather_ld;
-      const int m0 = mt * 256 + 128 * static_cast<int>(rank);
-      const int n0 = ntile * 256 + 128 * static_cast<int>(rank);
-      for (int kb = 0; kb < kb_total; ++kb) {
-        bool w = true;
-        if (lane == 0) w = mbar_wait(&empty[stage], phase ^ 1u, abort_v);
-        if (!__shfl_sync(0xffffffffu, w, 0)) {
-          ok = false;
-          break;
-        }
-        const uint32_t bar = leader_addr(smem_u32(&full[stage]));
-        uint8_t* sa = smem + stage * C::kStage;
-        uint8_t* sb = sa + C::kABytes;
-        const int k0 = kb * kBK;
-        if (lane == 0) {
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kStage);
-          armed_phase[stage] = static_cast<int>(phase);
-          tma_load_3d_pair(&maps.a[0], sa, bar, m0, gro + k0, gz);
-          tma_load_3d_pair(&maps.a[0], sa + 8192, bar, m0 + 64, gro + k0, gz);
-        }
-        __syncwarp();
-        int src[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) src[j] = gather_src_row(p, g, base, nrows, k0 + kr + j);
-        tma_gather4_pair(&maps.b[0], sb + box * 8192 + (lane & 15) * 512, bar, n0 + 64 * box, src[0], src[1], src[2],
-                         src[3]);
-        if (++stage == C::kStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
-      }
-    }
-    if (!ok && lane == 0) {
-      *abort_flag = 1;
-      record_status(p.status, MOE_ERR_TIMEOUT);
-      if (leader)
-        for (int s = 0; s < C::kStages; ++s)
-          if (armed_phase[s] >= 0) mbar_wait(&full[s], static_cast<uint32_t>(armed_phase[s]), nullptr, 50000000ull);
-    }
-  } else if (warp == 0) {
+  if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
       int stage = 0;
@@ -1361,27 +1225,6 @@ moe_status_t make_map(CUtensorMap* m, const Mat& t, uint32_t box_inner, uint32_t
 
 // tiles: output tiles of the launch (pair tiles for PAIR); the grid is one CTA (or pair)
 // per tile up to what fits on the device at once
-// 2-D map of a gather source: boxes one row high and 64 bf16 columns wide (tile::gather4)
-moe_status_t make_gather_map(CUtensorMap* m, const Mat& t) {
-  if (t.ptr == nullptr) return fail(MOE_ERR_INVALID_ARG, "gather source is null");
-  if ((reinterpret_cast<uintptr_t>(t.ptr) & 15) != 0 || t.inner <= 0 || t.rows <= 1 || t.ld < t.inner ||
-      (t.ld * 2) % 16 != 0 || t.inner % 64 != 0)
-    return fail(MOE_ERR_INVALID_ARG, "gather source has a bad shape, stride or alignment");
-  auto fn = encode_fn();
-  if (fn == nullptr) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(t.inner), static_cast<cuuint64_t>(t.rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(t.ld * 2)};
-  cuuint32_t box[2] = {64, 1};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(t.ptr), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS)
-    return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the gather source (" +
-                                  std::to_string(static_cast<int>(r)) + ")");
-  return MOE_OK;
-}
-
 template <int BN, bool A_MN, bool B_MN, int EPI, bool PAIR>
 moe_status_t launch_instance(const TmaMaps& maps, const KParams& kp, long long tiles, cudaStream_t st) {
   auto kern = gemm_kernel<BN, A_MN, B_MN, EPI, PAIR>;
@@ -1486,15 +1329,6 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
   if (a.a_mn && a.b_mn && a.ragged == 1)
     return fail(MOE_ERR_UNSUPPORTED, "gemm with both operands MN-major takes no ragged rows");
   if (a.out == nullptr) return fail(MOE_ERR_INVALID_ARG, "gemm output is null");
-  const bool gather = a.gather_rows != nullptr;
-  // gathered A: one-CTA tiles, A stored [M][K], one K segment, ragged rows; gathered B:
-  // the CTA-pair weight gradient (both operands [K][.], float32 out)
-  const bool gather_a = gather && !a.a_mn;
-  const bool gather_b = gather && a.a_mn;
-  if (gather_a && (a.pair || a.nseg != 1 || a.ragged != 1))
-    return fail(MOE_ERR_UNSUPPORTED, "a gathered A takes one-CTA tiles, one K segment and ragged rows");
-  if (gather_b && !(a.b_mn && a.epi == EPI_F32 && a.nseg == 1 && a.ragged == 2 && a.bn == 256))
-    return fail(MOE_ERR_UNSUPPORTED, "a gathered B takes the ragged-K weight-gradient form");
 
   // groups of the output and element-wise tensors (a launch may cover some of them)
   const int tgroups = a.tensor_groups > 0 ? a.tensor_groups : a.groups;
@@ -1511,11 +1345,11 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
   kp.nseg = a.nseg;
   for (int s = 0; s < a.nseg; ++s) {
     moe_status_t r;
-    r = gather_a ? make_gather_map(&maps.a[s], a.gather_src) : make_map(&maps.a[s], a.A[s], 64, a.a_mn ? 64 : 128, "A");
+    r = make_map(&maps.a[s], a.A[s], 64, a.a_mn ? 64 : 128, "A");
     if (r != MOE_OK) return r;
     // a pair CTA loads half of B's rows (SwiGLU: the gate or the value half)
     const uint32_t b_rows = a.b_mn ? 64 : ((a.epi == EPI_SWIGLU || a.pair) ? a.bn / 2 : a.bn);
-    r = gather_b ? make_gather_map(&maps.b[s], a.gather_src) : make_map(&maps.b[s], a.B[s], 64, b_rows, "B");
+    r = make_map(&maps.b[s], a.B[s], 64, b_rows, "B");
     if (r != MOE_OK) return r;
     kp.seg_kb[s] = a.ragged == 2 ? 0 : static_cast<int>((a.K[s] + kBK - 1) / kBK);
   }
@@ -1590,9 +1424,6 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
   kp.addend = a.addend;
   kp.add_ld = a.add_ld;
   kp.status = a.status;
-  kp.gather_rows = a.gather_rows;
-  kp.gather_ld = a.gather_ld;
-  kp.gather_zero = gather ? static_cast<int>(a.gather_src.rows - 1) : 0;
   kp.map_p = a.map_p;
   kp.map_l = a.map_l;
   kp.map_off = a.map_off;

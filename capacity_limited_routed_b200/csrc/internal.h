@@ -107,14 +107,6 @@ struct GemmArgs {
   const float* addend = nullptr;
   int64_t add_ld = 0;
   int32_t* status = nullptr;
-  // A gathered operand: rows chosen by index from a 2-D source tensor whose last row is
-  // all zeros.  One-CTA GEMMs with A stored [M][K] gather A's rows (gather_src inner =
-  // K); CTA-pair weight gradients gather B's K rows (gather_src inner = N).  Row r of
-  // group g is source row gather_rows[group_off[g] + r] (packed) or
-  // gather_rows[g * gather_ld + r]; rows at or past the group's count read the zero row.
-  const int32_t* gather_rows = nullptr;
-  int64_t gather_ld = 0;
-  Mat gather_src;
   // launch group g is expert (g / map_p) * map_l + map_off + g % map_p (map_p = 0: g):
   // one wave's D * P experts as one launch; tensors stay indexed by expert and hold
   // tensor_groups groups (0: groups)
@@ -155,12 +147,12 @@ moe_status_t launch_pack(const Geo& g, const uint16_t* z, const int32_t* idx, co
 moe_status_t launch_offsets(const int32_t* counts, int n, int align, int32_t* off, cudaStream_t st);
 // scratch ints needed by the receiver's row map
 size_t unpack_scratch_ints(const Geo& g);
-// Receiver side: ranks the rows of every pool by their packed ids and writes, for each
-// expert row, the pool row it came from (src, indexed like the expert buffers).
+// Receiver side: ranks the rows of every pool by their packed ids and copies the kept
+// rows into the expert buffers xe.
 // capacity layout: pool_off = exp_off = nullptr.  Dropless: pool_off / pool_fill give
 // each pool's packed row range; exp_off (E+1 ints) is computed here from the counts.
 // id_base: the packed (global) expert id of this receiver's expert 0 (expert parallelism)
-moe_status_t launch_unpack(const Geo& g, const uint16_t* pools, int32_t* src, int32_t* rows, int32_t* row_map,
+moe_status_t launch_unpack(const Geo& g, const uint16_t* pools, uint16_t* xe, int32_t* rows, int32_t* row_map,
                            int32_t* status, cudaStream_t st, const int32_t* pool_off = nullptr,
                            const int32_t* pool_fill = nullptr, int32_t* exp_off = nullptr, int id_base = 0);
 // rows between a receiver's pool positions and its expert rows by the row map (see map_rows_kernel)

@@ -23,11 +23,11 @@ struct moe_plan {
   int dm, dl, E, k, h, S, hs;
   // forward context layout (byte offsets); training adds the SwiGLU pre-activations
   struct Ctx {
-    size_t z, logits, idx, gate, slot, rows, src, pools, ae, be, he, ye, r, as, bs, hsh, exp_off, pool_off, bytes;
+    size_t z, logits, idx, gate, slot, rows, xe, ae, be, he, ye, r, as, bs, hsh, exp_off, pool_off, bytes;
   } saved, infer;
   // scratch layouts
   size_t ws_scan, ws_pools, ws_rowmap, ws_ctx, ws_fwd_bytes;             // forward
-  size_t ws_ffn_src, ws_ffn_he, ws_ffn_rows, ws_ffn_rowmap, ws_ffn_bytes;  // moe_expert_ffn alone
+  size_t ws_ffn_xe, ws_ffn_he, ws_ffn_rows, ws_ffn_rowmap, ws_ffn_bytes;  // moe_expert_ffn alone
   size_t b_dr, b_das, b_dbs, b_dye, b_dg, b_dae, b_dbe, b_dxe, b_dlog, b_dzr, b_dz, ws_bwd_bytes;
   size_t pools_bytes, expert_out_bytes, slot_bytes, stats_bytes, ws_bytes;
   // expert parallelism (G > 1): this rank is one source of T tokens (geometry g) and the
@@ -38,7 +38,7 @@ struct moe_plan {
   struct Ep {
     // forward context: the source's, then the receiver's
     size_t z, logits, idx, gate, slot, r, as, bs, hsh, y_in;
-    size_t recv_pools, src, rows, row_map, ae, be, he, ye;
+    size_t recv_pools, xe, rows, row_map, ae, be, he, ye;
     size_t saved_bytes;
     // scratch: the exchange buffers, and what the backward keeps from its first call to its last
     size_t scan, send_pools, y_out, dy_out, dy_in, dx_out, dx_in;
@@ -149,9 +149,7 @@ void layout_ctx(const moe_plan& p, bool training, moe_plan::Ctx& c) {
   c.gate = take(off, T * k * 4);
   c.slot = take(off, T * k * 8);
   c.rows = take(off, E * 4);
-  c.src = take(off, R * 4);  // pool row of each expert row: the experts gather their rows from the pools
-  // training keeps the pools for the weight gradients (inference packs them into scratch)
-  c.pools = training ? take(off, p.pools_bytes) : 0;
+  c.xe = take(off, R * dl * 2);
   c.ae = training ? take(off, R * h * 2) : 0;
   c.be = training ? take(off, R * h * 2) : 0;
   c.he = take(off, R * h * 2);
@@ -168,8 +166,7 @@ void layout_ctx(const moe_plan& p, bool training, moe_plan::Ctx& c) {
 void layout(moe_plan& p) {
   const size_t T = p.g.T, E = p.E, k = p.k, dl = p.dl, h = p.h, SH = size_t(p.S) * p.hs;
   const size_t R = size_t(p.g.exp_rows);
-  // the pools and one trailing all-zero row (the receiver's padding rows read it)
-  p.pools_bytes = (size_t(p.g.pool_rows) + 1) * (dl + 8) * 2;
+  p.pools_bytes = size_t(p.g.pool_rows) * (dl + 8) * 2;
   layout_ctx(p, true, p.saved);
   layout_ctx(p, false, p.infer);
   p.expert_out_bytes = R * dl * 2;
@@ -182,7 +179,7 @@ void layout(moe_plan& p) {
   p.ws_ctx = take(off, p.infer.bytes);  // used only when the forward keeps no context
   p.ws_fwd_bytes = off;
   off = 0;
-  p.ws_ffn_src = take(off, R * 4);
+  p.ws_ffn_xe = take(off, R * dl * 2);
   p.ws_ffn_he = take(off, R * h * 2);
   p.ws_ffn_rows = take(off, E * 4);
   p.ws_ffn_rowmap = take(off, unpack_scratch_ints(p.g) * 4);
@@ -225,7 +222,7 @@ void layout_ep(moe_plan& p) {
   e.hsh = take(off, T * SH * 2);
   e.y_in = take(off, e.rows_bytes);
   e.recv_pools = take(off, p.pools_bytes);
-  e.src = take(off, Rr * 4);
+  e.xe = take(off, Rr * dl * 2);
   e.rows = take(off, size_t(p.E_loc) * 4);
   e.row_map = take(off, prow * 4);
   e.ae = take(off, Rr * h * 2);
@@ -348,8 +345,7 @@ const T* at(const void* base, size_t off) {
 }
 
 struct CtxPtrs {
-  uint16_t *z, *pools, *ae, *be, *he, *ye, *r, *as, *bs, *hsh;
-  int32_t* src;
+  uint16_t *z, *xe, *ae, *be, *he, *ye, *r, *as, *bs, *hsh;
   float *logits, *gate;
   int32_t *idx, *slot, *rows;
   int32_t *exp_off, *pool_off;  // used by the dropless variant
@@ -364,8 +360,7 @@ CtxPtrs ctx_ptrs(const moe_plan& p, void* base, bool training) {
   q.gate = at<float>(base, c.gate);
   q.slot = at<int32_t>(base, c.slot);
   q.rows = at<int32_t>(base, c.rows);
-  q.src = at<int32_t>(base, c.src);
-  q.pools = training ? at<uint16_t>(base, c.pools) : nullptr;
+  q.xe = at<uint16_t>(base, c.xe);
   q.ae = training ? at<uint16_t>(base, c.ae) : nullptr;
   q.be = training ? at<uint16_t>(base, c.be) : nullptr;
   q.he = at<uint16_t>(base, c.he);
@@ -401,26 +396,12 @@ void pack_groups(const Geo& g, GemmArgs& a, const int32_t* exp_off) {
   if (a.ragged == 1) a.M = static_cast<int>(g.exp_rows);  // local rows never reach it
 }
 
-// The pools as a gather source: [pool rows + 1][d_latent] payload columns of the
-// (d_latent + 8)-wide pool rows; the last row is all zeros.
-Mat pools_src(const Geo& g, const uint16_t* pools) {
-  Mat m;
-  m.ptr = pools;
-  m.inner = g.dl;
-  m.rows = g.pool_rows + 1;
-  m.groups = 1;
-  m.ld = g.dl + 8;
-  m.gs = m.ld * m.rows;
-  return m;
-}
-
-// receiver unpack + grouped SwiGLU experts (shared by moe_expert_ffn and moe_forward).
-// The receiver records each expert row's pool row (src); the gate/up GEMM gathers its
-// input rows from the pools through src, so no expert-input buffer is written.
+// receiver unpack + grouped SwiGLU experts (shared by moe_expert_ffn, moe_forward and the
+// expert-parallel receiver): the receiver copies its kept rows into the expert buffers xe.
 // g: the receiver's geometry; E its experts (weights [E][..]), dl, h the widths; id_base the
 // packed (global) id of its expert 0.
 moe_status_t run_experts_geo(const Geo& g, int E, int dl, int h, int id_base, const uint16_t* w1,
-                             const uint16_t* w3, const uint16_t* w2, const uint16_t* pools, int32_t* src,
+                             const uint16_t* w3, const uint16_t* w2, const uint16_t* pools, uint16_t* xe,
                              int32_t* rows, int32_t* row_map, uint16_t* ae, uint16_t* be, uint16_t* he,
                              uint16_t* ye, int32_t* status, cudaStream_t st, const int32_t* pool_off = nullptr,
                              const int32_t* pool_fill = nullptr, int32_t* exp_off = nullptr) {
@@ -429,7 +410,8 @@ moe_status_t run_experts_geo(const Geo& g, int E, int dl, int h, int id_base, co
   } p{E, dl, h};
   {
     ProfScope ps("experts.unpack", st);
-    MOE_TRY(launch_unpack(g, pools, src, rows, row_map, status, st, pool_off, pool_fill, exp_off, id_base));
+    MOE_TRY(launch_unpack(g, pools, xe, rows, row_map, status, st, pool_off, pool_fill, exp_off, id_base));
+    MOE_TRY(launch_zero_tail_rows(g, xe, dl, rows, st, exp_off));
   }
   // the three waves of identical shape, one after another: wave w is the D * P experts
   // with local index in [w * P, (w + 1) * P) of every destination
@@ -446,9 +428,7 @@ moe_status_t run_experts_geo(const Geo& g, int E, int dl, int h, int id_base, co
     a.tensor_groups = p.E;
     a.ragged = 1;
     a.group_rows = rows;
-    a.gather_rows = src;
-    a.gather_ld = g.Cr;
-    a.gather_src = pools_src(g, pools);
+    a.A[0] = expert_mat(g, xe, p.dl);
     a.B[0] = mat(w1, p.dl, p.h, p.E);
     a.Bv = mat(w3, p.dl, p.h, p.E);
     a.K[0] = p.dl;
@@ -492,20 +472,19 @@ moe_status_t run_experts_geo(const Geo& g, int E, int dl, int h, int id_base, co
 }
 
 moe_status_t run_experts(const moe_plan& p, const uint16_t* w1, const uint16_t* w3, const uint16_t* w2,
-                         const uint16_t* pools, int32_t* src, int32_t* rows, int32_t* row_map, uint16_t* ae,
+                         const uint16_t* pools, uint16_t* xe, int32_t* rows, int32_t* row_map, uint16_t* ae,
                          uint16_t* be, uint16_t* he, uint16_t* ye, int32_t* status, cudaStream_t st,
                          const int32_t* pool_off = nullptr, const int32_t* pool_fill = nullptr,
                          int32_t* exp_off = nullptr) {
-  return run_experts_geo(p.g, p.E, p.dl, p.h, 0, w1, w3, w2, pools, src, rows, row_map, ae, be, he, ye, status, st,
+  return run_experts_geo(p.g, p.E, p.dl, p.h, 0, w1, w3, w2, pools, xe, rows, row_map, ae, be, he, ye, status, st,
                          pool_off, pool_fill, exp_off);
 }
 
 // Backward of the routed experts on a receiver's rows, given dY (rows of dye):
-// dH = dY w2 -> (dA, dB);  dw2 = dY^T H;  dX = dA w1 + dB w3;  dw1 = dA^T X, dw3 = dB^T X,
-// with X gathered from the pools through src.  g: the receiver's geometry, E its experts.
+// dH = dY w2 -> (dA, dB);  dw2 = dY^T H;  dX = dA w1 + dB w3;  dw1 = dA^T X, dw3 = dB^T X.
+// g: the receiver's geometry, E its experts.
 moe_status_t routed_backward(const Geo& g, int E, int dl, int h, const uint16_t* w1, const uint16_t* w3,
-                             const uint16_t* w2, const int32_t* rows, const int32_t* src, const uint16_t* pools,
-                             const uint16_t* ae, const uint16_t* be, const uint16_t* he, const uint16_t* dye,
+                             const uint16_t* w2, const int32_t* rows, const uint16_t* xe, const uint16_t* ae, const uint16_t* be, const uint16_t* he, const uint16_t* dye,
                              uint16_t* dae, uint16_t* dbe, uint16_t* dxe, float* gw1, float* gw3, float* gw2,
                              cudaStream_t st, const int32_t* exp_off) {
   const int64_t Cr = g.Cr;
@@ -588,10 +567,7 @@ moe_status_t routed_backward(const Geo& g, int E, int dl, int h, const uint16_t*
     a.group_rows = rows;
     a.m_fastest = false;  // concurrent tiles write whole rows of dW
     a.A[0] = expert_mat(g, dae, h);
-    // B = X, the expert rows gathered from the saved pools along K
-    a.gather_rows = src;
-    a.gather_ld = Cr;
-    a.gather_src = pools_src(g, pools);
+    a.B[0] = expert_mat(g, xe, dl);
     a.out = gw1;
     a.ldo = dl;
     a.out_gs = int64_t(h) * dl;
@@ -780,8 +756,7 @@ moe_status_t moe_saved_view(moe_plan_t p, const void* saved, moe_saved_view_t* o
   out->topk_gate = q.gate;
   out->slot = q.slot;
   out->expert_rows = q.rows;
-  out->pools = q.pools;
-  out->expert_src = q.src;
+  out->expert_in = q.xe;
   out->expert_out = q.ye;
   out->r = q.r;
   return MOE_OK;
@@ -827,7 +802,7 @@ moe_status_t moe_expert_ffn(moe_plan_t p, const moe_expert_weights_t* w, const u
   MOE_TRY(device_ok());
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int32_t* rows = expert_rows ? expert_rows : at<int32_t>(ws, p->ws_ffn_rows);
-  return run_experts(*p, w->w1, w->w3, w->w2, pools, at<int32_t>(ws, p->ws_ffn_src), rows,
+  return run_experts(*p, w->w1, w->w3, w->w2, pools, at<uint16_t>(ws, p->ws_ffn_xe), rows,
                      at<int32_t>(ws, p->ws_ffn_rowmap), nullptr, nullptr, at<uint16_t>(ws, p->ws_ffn_he), expert_out,
                      nullptr, st);
 }
@@ -931,8 +906,7 @@ moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const uint16_t* x
     ProfScope ps("fwd.slot_scan", st);
     MOE_TRY(launch_slot_scan(g, c.idx, c.slot, s, at<int32_t>(ws, p->ws_scan), st));
   }
-  // training keeps the pools in the forward context for the weight gradients
-  uint16_t* pools = training ? c.pools : at<uint16_t>(ws, p->ws_pools);
+  uint16_t* pools = at<uint16_t>(ws, p->ws_pools);
   // dropless: pools and expert buffers are packed; their offsets come from the counts
   int32_t* pool_off = g.dropless ? c.pool_off : nullptr;
   int32_t* exp_off = g.dropless ? c.exp_off : nullptr;
@@ -941,7 +915,7 @@ moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const uint16_t* x
     if (g.dropless) MOE_TRY(launch_offsets(s + stats_pool_fill(g), g.NPS, 1, pool_off, st));
     MOE_TRY(launch_pack(g, c.z, c.idx, c.slot, s, pools, st, pool_off));
   }
-  MOE_TRY(run_experts(*p, w->w1, w->w3, w->w2, pools, c.src, c.rows, at<int32_t>(ws, p->ws_rowmap), c.ae, c.be,
+  MOE_TRY(run_experts(*p, w->w1, w->w3, w->w2, pools, c.xe, c.rows, at<int32_t>(ws, p->ws_rowmap), c.ae, c.be,
                       c.he, c.ye, status, st, pool_off, g.dropless ? s + stats_pool_fill(g) : nullptr, exp_off));
   {
     ProfScope ps("fwd.combine", st);
@@ -1098,7 +1072,7 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
     MOE_TRY(launch_zero_tail_rows(g, dye, dl, c.rows, st, exp_off));
   }
   MOE_TRY(routed_backward(g, static_cast<int>(E), static_cast<int>(dl), static_cast<int>(h), w->w1, w->w3, w->w2,
-                          c.rows, c.src, c.pools, c.ae, c.be, c.he, dye, dae, dbe, dxe, gr->w1, gr->w3, gr->w2, st,
+                          c.rows, c.xe, c.ae, c.be, c.he, dye, dae, dbe, dxe, gr->w1, gr->w3, gr->w2, st,
                           exp_off));
   // un-dispatch and the softmax backward to the logits
   {
@@ -1218,9 +1192,9 @@ moe_status_t moe_gemm_bf16(int32_t M, int32_t N, int32_t K, const uint16_t* A, i
 namespace {
 
 struct EpPtrs {
-  uint16_t *z, *r, *as, *bs, *hsh, *y_in, *recv_pools, *ae, *be, *he, *ye;
+  uint16_t *z, *r, *as, *bs, *hsh, *y_in, *recv_pools, *xe, *ae, *be, *he, *ye;
   float *logits, *gate;
-  int32_t *idx, *slot, *src, *rows, *row_map;
+  int32_t *idx, *slot, *rows, *row_map;
   int32_t* scan;
   uint16_t *send_pools, *y_out, *dy_out, *dy_in, *dx_out, *dx_in, *dr, *das, *dbs, *dlog, *dz;
   float *dg, *dzr;
@@ -1242,7 +1216,7 @@ EpPtrs ep_ptrs(const moe_plan& p, const void* saved, void* ws) {
   q.hsh = at<uint16_t>(sv, e.hsh);
   q.y_in = at<uint16_t>(sv, e.y_in);
   q.recv_pools = at<uint16_t>(sv, e.recv_pools);
-  q.src = at<int32_t>(sv, e.src);
+  q.xe = at<uint16_t>(sv, e.xe);
   q.rows = at<int32_t>(sv, e.rows);
   q.row_map = at<int32_t>(sv, e.row_map);
   q.ae = at<uint16_t>(sv, e.ae);
@@ -1398,10 +1372,7 @@ moe_status_t moe_ep_forward_experts(moe_plan_t p, const moe_expert_weights_t* ew
   const Geo& r = p->gr;
   EpPtrs c = ep_ptrs(*p, saved, ws);
   int32_t* status = static_cast<int32_t*>(stats) + 3;
-  // the zero row after the received pools (padding rows of the experts read it)
-  MOE_TRY(cuda_check(cudaMemsetAsync(c.recv_pools + r.pool_rows * (p->dl + 8), 0, sizeof(uint16_t) * (p->dl + 8), st),
-                     "received pools zero row"));
-  MOE_TRY(run_experts_geo(r, p->E_loc, p->dl, p->h, p->rank * p->E_loc, ew->w1, ew->w3, ew->w2, c.recv_pools, c.src,
+  MOE_TRY(run_experts_geo(r, p->E_loc, p->dl, p->h, p->rank * p->E_loc, ew->w1, ew->w3, ew->w2, c.recv_pools, c.xe,
                           c.rows, c.row_map, c.ae, c.be, c.he, c.ye, status, st));
   ProfScope ps("experts.return", st);
   return launch_map_rows(c.ye, c.y_out, c.row_map, c.recv_pools, p->dl + 8, p->dl, r.pool_rows, p->dl, p->dl,
@@ -1553,8 +1524,8 @@ moe_status_t moe_ep_backward_experts(moe_plan_t p, const moe_expert_weights_t* e
     MOE_TRY(launch_map_rows(c.dy_in, c.dye, c.row_map, nullptr, 0, 0, r.pool_rows, p->dl, p->dl, false, st));
     MOE_TRY(launch_zero_tail_rows(r, c.dye, p->dl, c.rows, st));
   }
-  MOE_TRY(routed_backward(r, p->E_loc, p->dl, p->h, ew->w1, ew->w3, ew->w2, c.rows, c.src, c.recv_pools, c.ae, c.be,
-                          c.he, c.dye, c.dae, c.dbe, c.dxe, gr->w1, gr->w3, gr->w2, st, nullptr));
+  MOE_TRY(routed_backward(r, p->E_loc, p->dl, p->h, ew->w1, ew->w3, ew->w2, c.rows, c.xe, c.ae, c.be, c.he, c.dye,
+                          c.dae, c.dbe, c.dxe, gr->w1, gr->w3, gr->w2, st, nullptr));
   ProfScope ps("bwd.experts_return", st);
   return launch_map_rows(c.dxe, c.dx_out, c.row_map, c.recv_pools, p->dl + 8, p->dl, r.pool_rows, p->dl, p->dl, true,
                          st);

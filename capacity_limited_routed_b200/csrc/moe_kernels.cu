@@ -12,9 +12,7 @@
 //   pack            sender: z rows into the fixed pools with the expert id in a 16-byte row
 //                   header (same page, §2: one pool per receiving GPU, ids in the payload)
 //   unpack          receiver: reads only the pools; ranks rows of each local expert by the
-//                   packed id, keeps the first C_r, and records for each expert row the
-//                   pool row it came from (the expert GEMMs gather their rows from the
-//                   pools by these indices)
+//                   packed id, keeps the first C_r, gathers them per expert
 //   combine         r_t = sum_j kept g_tj Y[e_tj][rslot_tj], fixed j order, fp32 accumulation
 //   combine_bwd     dY = g dr on kept rows, dg = <dr, Y>
 //   undispatch      dz_routed = sum_j kept dX, and the softmax backward to the logits
@@ -559,15 +557,16 @@ __global__ void unpack_rank_kernel(const uint16_t* __restrict__ pools, int Cs, i
   if (threadIdx.x < P) rows_out[e_first + threadIdx.x] = packed ? s_run[threadIdx.x] : min(s_run[threadIdx.x], Cr);
 }
 
-// receiver, pass 2: one thread per pool row.  A kept row's receive-buffer row d (e * C_r +
-// slot, or exp_off[e] + slot for packed buffers) records the pool row it came from:
-// src[d] = pool row.  The expert GEMMs gather their input rows through src.
-__global__ void unpack_index_kernel(const uint16_t* __restrict__ pools, const int32_t* __restrict__ row_map,
-                                    long long n_rows, int dl, int32_t* __restrict__ src,
-                                    const int32_t* __restrict__ exp_off, int E) {
+// receiver, pass 2: one warp per pool row, up to 8 vectors per lane in flight
+__global__ void unpack_copy_kernel(const uint16_t* __restrict__ pools, const int32_t* __restrict__ row_map,
+                                   long long n_rows, int dl, uint16_t* __restrict__ xe,
+                                   const int32_t* __restrict__ exp_off, int E) {
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
   const long long row_elems = dl + 8;
-  for (long long r = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; r < n_rows;
-       r += static_cast<long long>(gridDim.x) * blockDim.x) {
+  const int nvec = dl / 8;
+  for (long long r = static_cast<long long>(blockIdx.x) * warps + (threadIdx.x >> 5); r < n_rows;
+       r += static_cast<long long>(gridDim.x) * warps) {
     long long d = row_map[r];
     if (d < 0) continue;
     if (exp_off != nullptr) {  // packed buffers: the row map holds the slot within the expert
@@ -575,7 +574,17 @@ __global__ void unpack_index_kernel(const uint16_t* __restrict__ pools, const in
       if (e < 0 || e >= E) continue;
       d += exp_off[e];
     }
-    src[d] = static_cast<int32_t>(r);
+    const uint4* src = reinterpret_cast<const uint4*>(pools + r * row_elems);
+    uint4* dst = reinterpret_cast<uint4*>(xe + d * dl);
+    for (int v0 = lane; v0 < nvec; v0 += 32 * 8) {
+      uint4 val[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (v0 + 32 * u < nvec) val[u] = src[v0 + 32 * u];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = val[u];
+    }
   }
 }
 
@@ -1022,11 +1031,6 @@ moe_status_t launch_slot_scan(const Geo& g, const int32_t* idx, int32_t* slot, i
 
 moe_status_t launch_pack(const Geo& g, const uint16_t* z, const int32_t* idx, const int32_t* slot,
                          int32_t* stats, uint16_t* pools, cudaStream_t st, const int32_t* pool_off) {
-  // the trailing all-zero row after the pools (the receiver's padding rows read it)
-  {
-    const cudaError_t e = cudaMemsetAsync(pools + g.pool_rows * (g.dl + 8), 0, sizeof(uint16_t) * (g.dl + 8), st);
-    if (e != cudaSuccess) return cuda_check(e, "pools zero row");
-  }
   if (g.T > 0) {
     // two row buffers per warp; rows too wide for that take the register path
     const size_t smem = static_cast<size_t>(kPackWarps) * 2 * g.dl * 2;
@@ -1068,7 +1072,7 @@ moe_status_t launch_offsets(const int32_t* counts, int n, int align, int32_t* of
   return cuda_check(cudaGetLastError(), "offsets");
 }
 
-moe_status_t launch_unpack(const Geo& g, const uint16_t* pools, int32_t* src, int32_t* rows, int32_t* row_map,
+moe_status_t launch_unpack(const Geo& g, const uint16_t* pools, uint16_t* xe, int32_t* rows, int32_t* row_map,
                            int32_t* status, cudaStream_t st, const int32_t* pool_off, const int32_t* pool_fill,
                            int32_t* exp_off, int id_base) {
   if (g.P > 32) return fail(MOE_ERR_UNSUPPORTED, "more than 32 experts per wave");
@@ -1080,8 +1084,9 @@ moe_status_t launch_unpack(const Geo& g, const uint16_t* pools, int32_t* src, in
   count_launch();
   if (packed) MOE_TRY_K(launch_offsets(rows, g.E, 128, exp_off, st));
   const long long n_rows = g.pool_rows;
-  unpack_index_kernel<<<blocks_for(n_rows, 256), 256, 0, st>>>(pools, row_map, n_rows, g.dl, src,
-                                                               packed ? exp_off : nullptr, g.E);
+  const int warps = 8;
+  unpack_copy_kernel<<<blocks_for(n_rows, warps), 32 * warps, 0, st>>>(pools, row_map, n_rows, g.dl, xe,
+                                                                       packed ? exp_off : nullptr, g.E);
   count_launch();
   return cuda_check(cudaGetLastError(), "unpack");
 }

@@ -333,31 +333,6 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
       : "memory");
 }
 
-// ---------------------------------------------------------------- row gathers (tile::gather4)
-//
-// Four rows of a 2-D tensor, chosen by row index, each `box columns` wide from column
-// c0, land as four consecutive 128-byte rows of shared memory (the tensor map's box is
-// one row high; its swizzle applies as for a tiled load).  No multicast.
-
-__device__ __forceinline__ void tma_gather4(const CUtensorMap* map, void* dst, uint64_t* bar, int c0, int r0, int r1,
-                                            int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// the same into this CTA's shared memory, completion counted on the pair leader's barrier
-__device__ __forceinline__ void tma_gather4_pair(const CUtensorMap* map, void* dst, uint32_t leader_bar, int c0,
-                                                 int r0, int r1, int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(leader_bar)
-      : "memory");
-}
-
 // ---------------------------------------------------------------- untiled bulk copies
 
 // global -> this CTA's shared memory, completion counted on `bar` (bytes: multiple of 16,

@@ -69,8 +69,7 @@ class moe_profile_record_t(ctypes.Structure):
 
 class moe_saved_view_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
-        "z", "logits", "topk_idx", "topk_gate", "slot", "expert_rows", "pools", "expert_src", "expert_out",
-        "r")]
+        "z", "logits", "topk_idx", "topk_gate", "slot", "expert_rows", "expert_in", "expert_out", "r")]
 
 
 class moe_ep_view_t(ctypes.Structure):

@@ -118,8 +118,7 @@ typedef struct {
   int32_t cap_send;          /* C_s, rows of one pool (0: dropless) */
   int32_t cap_recv;          /* C_r, rows of one expert (0: dropless) */
   int32_t pool_row_elems;    /* bf16 elements per pool row: d_latent payload + 8 header */
-  uint64_t pools_bytes;      /* [D*W][C_s][pool_row_elems] bf16 (dropless: [T*k][...]) and one
-                              * trailing all-zero row, written by moe_dispatch */
+  uint64_t pools_bytes;      /* [D*W][C_s][pool_row_elems] bf16 (dropless: [T*k][...]) */
   uint64_t expert_out_bytes; /* [E][C_r][d_latent] bf16 (dropless: [T*k + 127*E][...]) */
   uint64_t slot_bytes;       /* [T][k][2] int32 */
   uint64_t stats_bytes;      /* moe_stats_t + per-expert and per-pool counters */
@@ -176,10 +175,7 @@ typedef struct {
   const float* topk_gate;     /* [T][k] */
   const int32_t* slot;        /* [T][k][2]: sender slot, receiver slot (-1 = dropped) */
   const int32_t* expert_rows; /* [E] rows each expert received (<= C_r) */
-  const uint16_t* pools;      /* [n_pools * C_s + 1][d_latent + 8] bf16, as dispatched (the last
-                               * row all zeros); the experts read their input rows from here */
-  const int32_t* expert_src;  /* [E][C_r] int32: pool row of each expert row (rows below the
-                               * expert's count; the rest unspecified) */
+  const uint16_t* expert_in;  /* [E][C_r][d_latent] bf16, receiver-side rows */
   const uint16_t* expert_out; /* [E][C_r][d_latent] bf16 */
   const uint16_t* r;          /* [T][d_latent] bf16, combined routed output */
 } moe_saved_view_t;
@@ -211,8 +207,7 @@ MOE_API moe_status_t moe_route(moe_plan_t plan, const float* logits, const float
  * order, then packing of z rows into the fixed pools.
  *   z [T][d_latent] bf16 device; topk_idx [T][k] int32 device;
  *   pools [D*W][C_s][d_latent + 8] bf16 device: row = payload, then a 16-byte header
- *     whose first int32 is the global expert id (-1 for an empty row); one more row
- *     after the last pool is written all zeros (pools_bytes counts it);
+ *     whose first int32 is the global expert id (-1 for an empty row);
  *   slot [T][k][2] int32 device: (sender slot | -1, receiver slot | -1);
  *   stats: stats buffer (device), counters overwritten (hist left as is);
  *   ws: scratch of ws_bytes >= workspace_bytes.
@@ -251,9 +246,7 @@ MOE_API moe_status_t moe_dispatch_noalloc(moe_plan_t plan, const uint16_t* z, co
  * MoE-модели с 535 млрд параметров", §2: the receiver learns each row's expert from
  * the id in the payload, with no separate count or metadata exchange;
  * "Marin 535B-A23B：一场完全公开的前沿 MoE 训练直播", §2.2: SwiGLU experts of width 3072.)
- *   pools as written by moe_dispatch (with its trailing all-zero row: the expert GEMMs
- *   read their input rows straight from the pools by row index, and padding rows read
- *   the zero row); expert_out [E][C_r][d_latent] bf16 device
+ *   pools as written by moe_dispatch; expert_out [E][C_r][d_latent] bf16 device
  *   (rows at and past the expert's row count are zero or unspecified);
  *   expert_rows [E] int32 device, rows each expert received (may be NULL). */
 MOE_API moe_status_t moe_expert_ffn(moe_plan_t plan, const moe_expert_weights_t* w,
@@ -343,7 +336,7 @@ typedef struct {
   int32_t ranks, rank, dest_per_rank, n_waves, cap_send;
   int32_t pool_row_elems;     /* d_latent + 8 */
   int32_t row_elems;          /* d_latent */
-  uint16_t* send_pools;       /* [D*W*C_s][d_latent + 8] bf16 (ws), then one zero row */
+  uint16_t* send_pools;       /* [D*W*C_s][d_latent + 8] bf16 (ws) */
   uint16_t* recv_pools;       /* [D*W*C_s][d_latent + 8] bf16 (saved): blocks from every source */
   uint16_t* y_send;           /* [D*W*C_s][d_latent] (ws): expert outputs back to their sources */
   uint16_t* y_recv;           /* [D*W*C_s][d_latent] (saved): this source's rows back */

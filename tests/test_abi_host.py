@@ -38,8 +38,7 @@ def test_plan_capacities_match_oracle(M, wid):
     assert plan.info.local_experts == g.L and plan.info.experts_per_wave == g.P
     assert plan.info.n_pools == g.D * g.W
     assert plan.info.pool_row_elems == s.d_latent + 8
-    # the pools and one trailing all-zero row
-    assert plan.info.pools_bytes == (g.D * g.W * g.C_s + 1) * (s.d_latent + 8) * 2
+    assert plan.info.pools_bytes == g.D * g.W * g.C_s * (s.d_latent + 8) * 2
     assert plan.info.expert_out_bytes == s.n_experts * g.C_r * s.d_latent * 2
     assert plan.info.stats_bytes == 4 * (8 + 4 * s.n_experts + g.D * g.W)
     assert plan.info.workspace_bytes % 256 == 0 and plan.info.saved_bytes % 256 == 0
@@ -111,7 +110,7 @@ def test_dropless_plan_sizes(M):
     p = M.Plan(T=T, d_model=128, d_latent=dl, n_experts=E, top_k=k, n_dest=4, hidden_routed=128,
                n_shared=1, hidden_shared=128, cap_send=(0, 1), cap_recv=(0, 1))
     assert p.info.cap_send == 0 and p.info.cap_recv == 0
-    assert p.info.pools_bytes == (T * k + 1) * (dl + 8) * 2
+    assert p.info.pools_bytes == T * k * (dl + 8) * 2
     assert p.info.expert_out_bytes == (T * k + 127 * E) * dl * 2
     # only one numerator 0 is an error, as before
     with pytest.raises(M.MoEError):
@@ -128,7 +127,7 @@ def test_plan_with_sources(M):
         assert p.info.n_pools == S * 4 * 3
         assert p.info.cap_send == -(-512 * 2 * 110 // (100 * 12 * S))
         assert p.info.cap_recv == -(-512 * 2 * 115 // (100 * 24))
-        assert p.info.pools_bytes == (S * 12 * p.info.cap_send + 1) * (64 + 8) * 2
+        assert p.info.pools_bytes == S * 12 * p.info.cap_send * (64 + 8) * 2
     with pytest.raises(M.MoEError):
         M.Plan(**base, n_sources=3)    # 512 / 3 is not whole
     with pytest.raises(M.MoEError):

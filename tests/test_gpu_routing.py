@@ -101,10 +101,7 @@ def test_dispatch_bit_exact(M, shape, skew):
     assert np.array_equal(st[8 + 4 * E:8 + 4 * E + NP], slots["pool_fill"])
     assert st[4] == slots["pool_fill"].max() and st[5] == slots["expert_kept"].max()
     # pools: packed ids in the header, rows copied bit for bit
-    # the pools, then one trailing all-zero row
-    flat = pools.view(torch.int16).cpu().numpy().reshape(-1, s.d_latent + 8)
-    assert flat.shape[0] == NP * g.C_s + 1 and not flat[-1, : s.d_latent].any()
-    rows = flat[:-1].reshape(NP, g.C_s, s.d_latent + 8)
+    rows = pools.view(torch.int16).cpu().numpy().reshape(NP, g.C_s, s.d_latent + 8)
     hdr = rows[:, :, s.d_latent:].copy().view(np.int32)[:, :, 0]
     assert np.array_equal(hdr, header)
     got = rows[:, :, : s.d_latent].view(np.uint16)
@@ -119,15 +116,14 @@ def test_dispatch_bit_exact(M, shape, skew):
 
 
 def _pools_device(plan, s, g, payload, header):
-    """The oracle's pools in the device layout: pool rows, then the trailing all-zero row."""
+    """The oracle's pools in the device layout."""
     rows = np.zeros((g.n_pools, g.C_s, s.d_latent + 8), dtype=np.uint16)
     rows[:, :, : s.d_latent] = synth.to_bf16_bits(payload.astype(np.float32))
     hdr = np.zeros((g.n_pools, g.C_s, 4), dtype=np.int32)
     hdr[:, :, 0] = header
     rows[:, :, s.d_latent:] = hdr.view(np.uint16)
-    flat = np.concatenate([rows.reshape(-1, s.d_latent + 8), np.zeros((1, s.d_latent + 8), np.uint16)])
-    assert flat.nbytes == plan.info.pools_bytes
-    return torch.from_numpy(flat.view(np.int16)).to(dev()).view(torch.bfloat16)
+    assert rows.nbytes == plan.info.pools_bytes
+    return torch.from_numpy(rows.view(np.int16)).to(dev()).view(torch.bfloat16)
 
 
 @pytest.mark.parametrize("shape,skew", [(synth.TINY, 1.0), (synth.MID, 0.5)])

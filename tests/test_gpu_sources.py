@@ -43,10 +43,7 @@ def test_dispatch_bit_exact_with_sources(M, S, skew):
     E, NPS = s.n_experts, S * g.n_pools
     assert (st[0], st[1], st[2], st[3]) == (sl["kept"], sl["dropped_sender"], sl["dropped_receiver"], 0)
     assert np.array_equal(st[8 + 4 * E:8 + 4 * E + NPS], sl["pool_fill"])
-    # the pools, then one trailing all-zero row
-    flat = pools.view(torch.int16).cpu().numpy().reshape(-1, s.d_latent + 8)
-    assert flat.shape[0] == NPS * g.C_s + 1 and not flat[-1, : s.d_latent].any()
-    rows = flat[:-1].reshape(NPS, g.C_s, s.d_latent + 8)
+    rows = pools.view(torch.int16).cpu().numpy().reshape(NPS, g.C_s, s.d_latent + 8)
     hdr = rows[:, :, s.d_latent:].copy().view(np.int32)[:, :, 0]
     assert np.array_equal(hdr, header)
     filled = header >= 0

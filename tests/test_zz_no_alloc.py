@@ -59,9 +59,7 @@ def _check_against_oracle(shape, plan, idx_np, z_bits, pools, slot, stats):
     assert np.array_equal(stats[8 + E:8 + 4 * E], np.concatenate(
         [sl["expert_kept"], sl["expert_dropped_sender"], sl["expert_dropped_receiver"]]))
     assert np.array_equal(stats[8 + 4 * E:8 + 4 * E + plan.info.n_pools], sl["pool_fill"])
-    flat = pools.reshape(-1, dl + 8)
-    assert flat.shape[0] == plan.info.n_pools * plan.info.cap_send + 1 and not flat[-1, :dl].any()
-    rows = flat[:-1].reshape(plan.info.n_pools, plan.info.cap_send, dl + 8)
+    rows = pools.reshape(plan.info.n_pools, plan.info.cap_send, dl + 8)
     hdr = rows[:, :, dl:dl + 2].copy().view(np.int32)[:, :, 0]
     assert np.array_equal(hdr, header)
     used = header >= 0
