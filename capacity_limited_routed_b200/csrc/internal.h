@@ -135,12 +135,14 @@ struct Geo {
 
 constexpr int kScanTokensPerChunk = 32;
 
+// hist may be nullptr: the forward leaves the histogram to the slot scan (write_hist)
 moe_status_t launch_route(const Geo& g, const float* logits, const float* bias, int32_t* idx, float* gate,
                           int32_t* hist, int32_t* nan_count, cudaStream_t st);
 // scratch ints needed by the slot scan
 size_t scan_scratch_ints(const Geo& g);
+// write_hist: also write the selection histogram into the stats (every assignment's expert)
 moe_status_t launch_slot_scan(const Geo& g, const int32_t* idx, int32_t* slot, int32_t* stats, int32_t* scratch,
-                              cudaStream_t st);
+                              cudaStream_t st, bool write_hist = false);
 moe_status_t launch_pack(const Geo& g, const uint16_t* z, const int32_t* idx, const int32_t* slot,
                          int32_t* stats, uint16_t* pools, cudaStream_t st, const int32_t* pool_off = nullptr);
 // off[i] = sum over j < i of round_up(counts[j], align), i = 0..n

@@ -900,11 +900,11 @@ moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const uint16_t* x
   }
   {
     ProfScope ps("fwd.route_topk", st);
-    MOE_TRY(launch_route(g, c.logits, bias, c.idx, c.gate, s + stats_hist(g), s + 7, st));
+    MOE_TRY(launch_route(g, c.logits, bias, c.idx, c.gate, nullptr, s + 7, st));
   }
   {
-    ProfScope ps("fwd.slot_scan", st);
-    MOE_TRY(launch_slot_scan(g, c.idx, c.slot, s, at<int32_t>(ws, p->ws_scan), st));
+    ProfScope ps("fwd.slot_scan", st);  // also the selection histogram
+    MOE_TRY(launch_slot_scan(g, c.idx, c.slot, s, at<int32_t>(ws, p->ws_scan), st, true));
   }
   uint16_t* pools = at<uint16_t>(ws, p->ws_pools);
   // dropless: pools and expert buffers are packed; their offsets come from the counts
@@ -1350,11 +1350,11 @@ moe_status_t moe_ep_forward_send(moe_plan_t p, const moe_weights_t* w, const uin
     }
     {
       ProfScope ps("fwd.route_topk", st);
-      MOE_TRY(launch_route(g, c.logits, bias, c.idx, c.gate, s + stats_hist(g), s + 7, st));
+      MOE_TRY(launch_route(g, c.logits, bias, c.idx, c.gate, nullptr, s + 7, st));
     }
     {
-      ProfScope ps("fwd.slot_scan", st);
-      MOE_TRY(launch_slot_scan(g, c.idx, c.slot, s, c.scan, st));
+      ProfScope ps("fwd.slot_scan", st);  // also the selection histogram
+      MOE_TRY(launch_slot_scan(g, c.idx, c.slot, s, c.scan, st, true));
     }
   }
   {

@@ -49,8 +49,10 @@ template <int VPL>
 __global__ void route_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E,
                                   int k, int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
                                   int32_t* __restrict__ hist, int32_t* __restrict__ nan_count) {
+  // hist == nullptr: the histogram is left to the slot scan, which counts every assignment
   __shared__ int sh_hist[kMaxE];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) sh_hist[e] = 0;
+  if (hist != nullptr)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) sh_hist[e] = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const int warps = blockDim.x >> 5;
@@ -126,13 +128,14 @@ __global__ void route_topk_kernel(const float* __restrict__ logits, const float*
     if (lane < k) {
       idx_out[static_cast<long long>(t) * k + lane] = my_e;
       gate_out[static_cast<long long>(t) * k + lane] = ex / sum;
-      if (my_e >= 0 && my_e < E) atomicAdd(&sh_hist[my_e], 1);
+      if (hist != nullptr && my_e >= 0 && my_e < E) atomicAdd(&sh_hist[my_e], 1);
     }
   }
   if (nan_local && nan_count != nullptr) atomicAdd(nan_count, nan_local);
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x)
-    if (sh_hist[e]) atomicAdd(&hist[e], sh_hist[e]);
+  if (hist != nullptr)
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+      if (sh_hist[e]) atomicAdd(&hist[e], sh_hist[e]);
 }
 
 // ---------------------------------------------------------------------- slot scan
@@ -293,9 +296,11 @@ __global__ void scan_receiver_slots(const int32_t* __restrict__ idx, int A_total
   }
 }
 
-// totals and maxima from the per-expert / per-pool counters (one block)
+// totals and maxima from the per-expert / per-pool counters (one block); with write_hist
+// also the selection histogram, kept + sender-dropped + receiver-dropped of each expert
+// (every assignment is exactly one of the three)
 __global__ void scan_totals(int32_t* __restrict__ stats, int E, int NP, int A_total, int off_kept, int off_ds,
-                            int off_dr, int off_fill) {
+                            int off_dr, int off_fill, int off_hist, int write_hist) {
   __shared__ int s_kept, s_ds, s_dr, s_mp, s_me;
   if (threadIdx.x == 0) s_kept = s_ds = s_dr = s_mp = s_me = 0;
   __syncthreads();
@@ -305,6 +310,7 @@ __global__ void scan_totals(int32_t* __restrict__ stats, int E, int NP, int A_to
     ds += stats[off_ds + e];
     dr += stats[off_dr + e];
     me = max(me, stats[off_kept + e]);
+    if (write_hist) stats[off_hist + e] = stats[off_kept + e] + stats[off_ds + e] + stats[off_dr + e];
   }
   for (int p = threadIdx.x; p < NP; p += blockDim.x) mp = max(mp, stats[off_fill + p]);
   atomicAdd(&s_kept, k);
@@ -995,7 +1001,7 @@ size_t scan_scratch_ints(const Geo& g) {
 }
 
 moe_status_t launch_slot_scan(const Geo& g, const int32_t* idx, int32_t* slot, int32_t* stats, int32_t* scratch,
-                              cudaStream_t st) {
+                              cudaStream_t st, bool write_hist) {
   const int A = g.T * g.k;
   const int chunk_assign = kScanTokensPerChunk * g.k;
   int32_t* cnt_pool = scratch;                                        // [NP][n_chunks]
@@ -1008,6 +1014,7 @@ moe_status_t launch_slot_scan(const Geo& g, const int32_t* idx, int32_t* slot, i
   if (e != cudaSuccess) return cuda_check(e, "slot scan memset");
   if (A == 0) {
     e = cudaMemsetAsync(stats + stats_pool_fill(g), 0, sizeof(int32_t) * g.NPS, st);
+    if (e == cudaSuccess && write_hist) e = cudaMemsetAsync(stats + stats_hist(g), 0, sizeof(int32_t) * g.E, st);
     return cuda_check(e, "slot scan memset");
   }
   scan_count_pools<<<g.n_chunks, 256, g.NP * sizeof(int), st>>>(idx, A, chunk_assign, g.n_chunks, g.L, g.P, g.W,
@@ -1024,7 +1031,7 @@ moe_status_t launch_slot_scan(const Geo& g, const int32_t* idx, int32_t* slot, i
       idx, A, chunk_assign, g.n_chunks, g.E, g.Cr, cnt_exp, slot, stats + stats_kept_e(g), stats + stats_ds_e(g),
       stats + stats_dr_e(g));
   scan_totals<<<1, 256, 0, st>>>(stats, g.E, g.NPS, A, stats_kept_e(g), stats_ds_e(g), stats_dr_e(g),
-                                 stats_pool_fill(g));
+                                 stats_pool_fill(g), stats_hist(g), write_hist ? 1 : 0);
   count_launch(6);
   return cuda_check(cudaGetLastError(), "slot scan");
 }
