@@ -647,6 +647,10 @@ def main():
             "roofline": roof,
             "dispatch_hbm_frac": kernels.get("fwd.dispatch_pack", {}).get("frac"),
             "kernels": kernels,
+            "kernels_note": ("per training step; the shared experts run on a second stream (forward: beside the "
+                             "routing, slot scan, pack, unpack and first routed launches; backward: beside "
+                             "un-dispatch and the router's backward), so those steps' event times include time "
+                             "spent sharing the GPU, and the times add up to more than ms_per_step"),
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches,

@@ -851,8 +851,39 @@ struct PairCfg {
 // An epilogue warp's share of a pair tile: 32 rows (row0..) x 128 columns (col_lo..) of
 // this CTA's accumulator half, per 32-column chunk TMEM -> registers -> staging -> one
 // TMA store (the copy engine clips rows and columns past the output's edge).
+#ifndef MOE_WB_PREFETCH
+#define MOE_WB_PREFETCH 0
+#endif
+
 __device__ __forceinline__ void pair_drain(const TmaMaps& maps, const KParams& p, uint32_t tbase, int col_lo,
                                            int ntile, int row0, int g, uint8_t* buf, uint32_t row_addr, int lane) {
+  if (MOE_WB_PREFETCH) {
+    // the next chunk's TMEM load is in flight while this chunk waits for the staging
+    // buffer and is written to it
+    uint32_t r[2][32];
+    tmem_ld_32cols_async(tbase + col_lo, r[0]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = col_lo + 32 * i;
+      const int col0 = ntile * 256 + c;
+      tmem_wait_ld();
+      if (i + 1 < 4) tmem_ld_32cols_async(tbase + c + 32, r[(i + 1) & 1]);
+      if (col0 >= p.N || row0 >= p.M) continue;  // warp-uniform
+      if (lane == 0) bulk_wait_read<0>();  // the previous chunk's store has read the buffer
+      __syncwarp();
+      const uint32_t* v = r[i & 1];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        st_shared_v4(row_addr + ((j ^ (lane & 7)) << 4), v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+      fence_async_shared();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_3d(&maps.out, buf, col0, row0, g);
+        bulk_commit();
+      }
+    }
+    return;
+  }
 #pragma unroll 1
   for (int c = col_lo; c < col_lo + 128; c += 32) {
     const int col0 = ntile * 256 + c;
@@ -870,48 +901,6 @@ __device__ __forceinline__ void pair_drain(const TmaMaps& maps, const KParams& p
     if (lane == 0) {
       tma_store_3d(&maps.out, buf, col0, row0, g);
       bulk_commit();
-    }
-  }
-}
-
-#ifndef MOE_WB_DIRECT
-#define MOE_WB_DIRECT 0
-#endif
-
-// The same share drained straight to global memory: per 16-row half and 64 columns, one
-// 16x256b TMEM load (a thread holds two rows, two adjacent columns of each 8-column group)
-// and st.global.v2 stores, each instruction writing eight whole 32-byte sectors; the next
-// load is in flight while the current registers are stored.  No shared-memory staging.
-__device__ __forceinline__ void pair_drain_direct(const KParams& p, uint32_t tbase, int col_lo, int ntile, int row0,
-                                                  int g, int lane) {
-  float* obase = static_cast<float*>(p.out) + static_cast<long long>(g) * p.out_gs;
-  const int rq = lane >> 2, cq = 2 * (lane & 3);
-  uint32_t r[2][32];
-  auto issue = [&](int it, uint32_t (&dst)[32]) {
-    const int h = it >> 1, c = col_lo + 64 * (it & 1);
-    tmem_ld_16x256b_x8_async(tbase + (static_cast<uint32_t>(16 * h) << 16) + static_cast<uint32_t>(c), dst);
-  };
-  issue(0, r[0]);
-#pragma unroll
-  for (int it = 0; it < 4; ++it) {
-    tmem_wait_ld();
-    if (it + 1 < 4) issue(it + 1, r[(it + 1) & 1]);
-    const int h = it >> 1, c = col_lo + 64 * (it & 1);
-    const int ra = row0 + 16 * h + rq, rb = ra + 8;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int col = ntile * 256 + c + 8 * i + cq;
-      if (col < p.N) {
-        const uint32_t* v = &r[it & 1][4 * i];
-        if (ra < p.M)
-          asm volatile("st.global.v2.b32 [%0], {%1, %2};" ::"l"(obase + static_cast<long long>(ra) * p.ldo + col),
-                       "r"(v[0]), "r"(v[1])
-                       : "memory");
-        if (rb < p.M)
-          asm volatile("st.global.v2.b32 [%0], {%1, %2};" ::"l"(obase + static_cast<long long>(rb) * p.ldo + col),
-                       "r"(v[2]), "r"(v[3])
-                       : "memory");
-      }
     }
   }
 }
@@ -1154,11 +1143,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         break;
       }
       tc_fence_after();
-      if (MOE_WB_DIRECT)
-        pair_drain_direct(p, tmem_base + lane_off + static_cast<uint32_t>(acc * 256), col_lo, ntile, row0, g, lane);
-      else
-        pair_drain(maps, p, tmem_base + lane_off + static_cast<uint32_t>(acc * 256), col_lo, ntile, row0, g, buf,
-                   row_addr, lane);
+      pair_drain(maps, p, tmem_base + lane_off + static_cast<uint32_t>(acc * 256), col_lo, ntile, row0, g, buf,
+                 row_addr, lane);
       __syncwarp();
       tc_fence_before();
       // hand the accumulator back to the leader's MMA warp

@@ -380,16 +380,9 @@ Mat expert_mat(const Geo& g, const void* ptr, int64_t width) {
   return g.dropless ? mat(ptr, width, g.exp_rows, 1) : mat(ptr, width, g.Cr, g.E);
 }
 
-// Routed (ragged-row) GEMMs on CTA pairs.  An expert's ~341 rows fill three 128-row
-// tiles (11% padding) but two 256-row pair tiles (33% padding).  Only the capped
-// layout may take pair tiles: a dropless expert region is padded to 128 rows, and a
-// 256-row tile would reach into the next expert's rows.
-#ifndef MOE_ROUTED_PAIR
-#define MOE_ROUTED_PAIR 0
-#endif
-
+// Routed (ragged-row) GEMMs keep one CTA per 128-row tile: an expert's ~341 rows fill
+// three of them (11% padding) but two 256-row pair tiles (50%), which measured slower.
 void pack_groups(const Geo& g, GemmArgs& a, const int32_t* exp_off) {
-  if (a.ragged == 1) a.pair = MOE_ROUTED_PAIR && !g.dropless;
   if (!g.dropless) return;
   a.group_off = exp_off;
   a.rows_total = g.exp_rows;
@@ -842,29 +835,6 @@ moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const uint16_t* x
   int32_t* status = s + 3;
   const int64_t SH = int64_t(p->S) * p->hs;
 
-  // shared experts on the side stream: H_s = silu(x ws1^T) * (x ws3^T)
-  SideStream* ss = nullptr;
-  MOE_TRY(side_stream(&ss));
-  MOE_TRY(fork_to(ss, st));
-  {
-    ProfScope ps("fwd.shared_gate_up", ss->s);
-    GemmArgs a;
-    a.pair = true;  // dense rows: 256-row tiles on CTA pairs
-    a.epi = EPI_SWIGLU;
-    a.M = g.T;
-    a.N = static_cast<int>(SH);
-    a.A[0] = mat(x, p->dm, g.T);
-    a.B[0] = mat(w->ws1, p->dm, SH);
-    a.Bv = mat(w->ws3, p->dm, SH);
-    a.K[0] = p->dm;
-    a.out = c.hsh;
-    a.ldo = SH;
-    a.save_a = c.as;
-    a.save_b = c.bs;
-    a.status = status;
-    MOE_TRY(gemm_run(a, ss->s));
-  }
-
   // latent down-projection: z = x W_lat_down^T
   {
     ProfScope ps("fwd.lat_down", st);
@@ -898,6 +868,30 @@ moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const uint16_t* x
     a.status = status;
     MOE_TRY(gemm_run(a, st));
   }
+  // shared experts on the side stream, beside the routing, movement and expert kernels:
+  // H_s = silu(x ws1^T) * (x ws3^T)
+  SideStream* ss = nullptr;
+  MOE_TRY(side_stream(&ss));
+  MOE_TRY(fork_to(ss, st));
+  {
+    ProfScope ps("fwd.shared_gate_up", ss->s);
+    GemmArgs a;
+    a.pair = true;  // dense rows: 256-row tiles on CTA pairs
+    a.epi = EPI_SWIGLU;
+    a.M = g.T;
+    a.N = static_cast<int>(SH);
+    a.A[0] = mat(x, p->dm, g.T);
+    a.B[0] = mat(w->ws1, p->dm, SH);
+    a.Bv = mat(w->ws3, p->dm, SH);
+    a.K[0] = p->dm;
+    a.out = c.hsh;
+    a.ldo = SH;
+    a.save_a = c.as;
+    a.save_b = c.bs;
+    a.status = status;
+    MOE_TRY(gemm_run(a, ss->s));
+  }
+
   {
     ProfScope ps("fwd.route_topk", st);
     MOE_TRY(launch_route(g, c.logits, bias, c.idx, c.gate, nullptr, s + 7, st));
@@ -1002,8 +996,33 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
     a.ldo = dl;
     MOE_TRY(gemm_run(a, st));
   }
-  // the shared experts' backward on the side stream (joined before dx): dH_s = dy ws2 ->
-  // SwiGLU backward -> (dA_s, dB_s);  dws2 = dy^T H_s;  dws1 = dA_s^T x, dws3 = dB_s^T x
+  // dW_up = dy^T r
+  {
+    ProfScope ps("bwd.wgrad_lat_up", st);
+    GemmArgs a;
+    a.a_mn = a.b_mn = true;
+    a.epi = EPI_F32;
+    a.M = static_cast<int>(dm);
+    a.N = static_cast<int>(dl);
+    a.A[0] = mat(dy, dm, T);
+    a.B[0] = mat(c.r, dl, T);
+    a.K[0] = T;
+    a.out = gr->w_lat_up;
+    a.ldo = dl;
+    MOE_TRY(gemm_run(a, st));
+  }
+  // combine backward: dY = g dr on kept rows, dg = <dr, Y>
+  {
+    ProfScope ps("bwd.combine", st);
+    MOE_TRY(launch_combine_bwd(g, dr, c.ye, c.gate, c.idx, c.slot, dye, dg, st, exp_off));
+    MOE_TRY(launch_zero_tail_rows(g, dye, dl, c.rows, st, exp_off));
+  }
+  MOE_TRY(routed_backward(g, static_cast<int>(E), static_cast<int>(dl), static_cast<int>(h), w->w1, w->w3, w->w2,
+                          c.rows, c.xe, c.ae, c.be, c.he, dye, dae, dbe, dxe, gr->w1, gr->w3, gr->w2, st,
+                          exp_off));
+  // the shared experts' backward on the side stream, beside un-dispatch and the router's
+  // backward (joined before dx): dH_s = dy ws2 -> SwiGLU backward -> (dA_s, dB_s);
+  // dws2 = dy^T H_s;  dws1 = dA_s^T x, dws3 = dB_s^T x
   SideStream* ss = nullptr;
   MOE_TRY(side_stream(&ss));
   MOE_TRY(fork_to(ss, st));
@@ -1050,30 +1069,6 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
     a.out = gr->ws3;
     MOE_TRY(gemm_run(a, ss->s));
   }
-  // dW_up = dy^T r
-  {
-    ProfScope ps("bwd.wgrad_lat_up", st);
-    GemmArgs a;
-    a.a_mn = a.b_mn = true;
-    a.epi = EPI_F32;
-    a.M = static_cast<int>(dm);
-    a.N = static_cast<int>(dl);
-    a.A[0] = mat(dy, dm, T);
-    a.B[0] = mat(c.r, dl, T);
-    a.K[0] = T;
-    a.out = gr->w_lat_up;
-    a.ldo = dl;
-    MOE_TRY(gemm_run(a, st));
-  }
-  // combine backward: dY = g dr on kept rows, dg = <dr, Y>
-  {
-    ProfScope ps("bwd.combine", st);
-    MOE_TRY(launch_combine_bwd(g, dr, c.ye, c.gate, c.idx, c.slot, dye, dg, st, exp_off));
-    MOE_TRY(launch_zero_tail_rows(g, dye, dl, c.rows, st, exp_off));
-  }
-  MOE_TRY(routed_backward(g, static_cast<int>(E), static_cast<int>(dl), static_cast<int>(h), w->w1, w->w3, w->w2,
-                          c.rows, c.xe, c.ae, c.be, c.he, dye, dae, dbe, dxe, gr->w1, gr->w3, gr->w2, st,
-                          exp_off));
   // un-dispatch and the softmax backward to the logits
   {
     ProfScope ps("bwd.undispatch", st);
