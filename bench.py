@@ -79,6 +79,7 @@ def workload_shape(name):
     from capacity_limited_routed_b200 import synth
     return {"train": synth.TRAIN, "full": synth.FULL, "mid": synth.MID, "skewed": synth.SKEWED,
             "tiny": synth.TINY.with_(backward=True), "profile": synth.PROFILE,
+            "profile_movers": synth.PROFILE_MOVERS,
             "train_dropless": synth.TRAIN_DROPLESS, "skewed_dropless": synth.SKEWED_DROPLESS}[name]
 
 

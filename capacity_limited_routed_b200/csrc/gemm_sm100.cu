@@ -833,14 +833,21 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
 // both CTAs' shared memory, each CTA draining its 128 accumulator rows.  Per output
 // element this reads a third fewer operand bytes than the single-CTA kernel, which is
 // what bounds these short (rows-per-expert) contractions.
-constexpr int kPairEpiWarps = 8;
+#ifndef MOE_PAIR_EPI_WARPS
+#define MOE_PAIR_EPI_WARPS 8
+#endif
+#ifndef MOE_PAIR_EARLY
+#define MOE_PAIR_EARLY 0
+#endif
+constexpr int kPairEpiWarps = MOE_PAIR_EPI_WARPS;
 constexpr int kPairThreads = 64 + 32 * kPairEpiWarps;
+constexpr int kPairCols = 256 / (kPairEpiWarps / 4);  // accumulator columns per epilogue warp
 
 struct PairCfg {
   static constexpr int kABytes = 128 * kBK * 2;
   static constexpr int kBBytes = 128 * kBK * 2;
   static constexpr int kStage = kABytes + kBBytes;  // 32 KB per CTA
-  static constexpr int kStages = 6;
+  static constexpr int kStages = kPairEpiWarps > 8 ? 5 : 6;
   static constexpr int kTmemCols = 512;             // two 256-column accumulators
   static constexpr int kStaging = kPairEpiWarps * 4096;
   static constexpr int kBarBytes = 8 * (2 * kStages + 5) + 16;
@@ -848,33 +855,33 @@ struct PairCfg {
   static_assert(kSmem <= 232448, "shared memory budget");
 };
 
-// An epilogue warp's share of a pair tile: 32 rows (row0..) x 128 columns (col_lo..) of
-// this CTA's accumulator half, per 32-column chunk TMEM -> registers -> staging -> one
-// TMA store (the copy engine clips rows and columns past the output's edge).
-#ifndef MOE_WB_PREFETCH
-#define MOE_WB_PREFETCH 0
-#endif
-
+// An epilogue warp's share of a pair tile: 32 rows (row0..) x kPairCols columns (col_lo..)
+// of this CTA's accumulator half, per 32-column chunk registers -> staging -> one TMA
+// store (the copy engine clips rows and columns past the output's edge).  MOE_PAIR_EARLY:
+// all of the share is read from TMEM first and the accumulator handed back before the
+// stores (tempty_addr: the leader's barrier); otherwise chunk by chunk, released by the
+// caller.
 __device__ __forceinline__ void pair_drain(const TmaMaps& maps, const KParams& p, uint32_t tbase, int col_lo,
-                                           int ntile, int row0, int g, uint8_t* buf, uint32_t row_addr, int lane) {
-  if (MOE_WB_PREFETCH) {
-    // the next chunk's TMEM load is in flight while this chunk waits for the staging
-    // buffer and is written to it
-    uint32_t r[2][32];
-    tmem_ld_32cols_async(tbase + col_lo, r[0]);
+                                           int ntile, int row0, int g, uint8_t* buf, uint32_t row_addr, int lane,
+                                           uint32_t tempty_addr) {
+  if (MOE_PAIR_EARLY) {
+    uint32_t r[kPairCols / 32][32];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int c = col_lo + 32 * i;
-      const int col0 = ntile * 256 + c;
-      tmem_wait_ld();
-      if (i + 1 < 4) tmem_ld_32cols_async(tbase + c + 32, r[(i + 1) & 1]);
-      if (col0 >= p.N || row0 >= p.M) continue;  // warp-uniform
-      if (lane == 0) bulk_wait_read<0>();  // the previous chunk's store has read the buffer
+    for (int i = 0; i < kPairCols / 32; ++i) tmem_ld_32cols_async(tbase + col_lo + 32 * i, r[i]);
+    tmem_wait_ld();
+    tc_fence_before();
+    __syncwarp();
+    mbar_arrive_cluster(tempty_addr);
+#pragma unroll
+    for (int i = 0; i < kPairCols / 32; ++i) {
+      const int col0 = ntile * 256 + col_lo + 32 * i;
+      if (col0 >= p.N || row0 >= p.M) break;  // warp-uniform
+      if (lane == 0) bulk_wait_read<0>();     // the previous chunk's store has read the buffer
       __syncwarp();
-      const uint32_t* v = r[i & 1];
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        st_shared_v4(row_addr + ((j ^ (lane & 7)) << 4), v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        st_shared_v4(row_addr + ((j ^ (lane & 7)) << 4), r[i][4 * j], r[i][4 * j + 1], r[i][4 * j + 2],
+                     r[i][4 * j + 3]);
       fence_async_shared();
       __syncwarp();
       if (lane == 0) {
@@ -885,7 +892,7 @@ __device__ __forceinline__ void pair_drain(const TmaMaps& maps, const KParams& p
     return;
   }
 #pragma unroll 1
-  for (int c = col_lo; c < col_lo + 128; c += 32) {
+  for (int c = col_lo; c < col_lo + kPairCols; c += 32) {
     const int col0 = ntile * 256 + c;
     if (col0 >= p.N || row0 >= p.M) break;
     float v[32];
@@ -910,7 +917,7 @@ __device__ __forceinline__ void pair_zero(const KParams& p, int col_lo, int ntil
   float* obase = static_cast<float*>(p.out) + static_cast<long long>(g) * p.out_gs;
   const int row = row0 + lane;
   if (row < p.M)
-    for (int c = col_lo; c < col_lo + 128; c += 4) {
+    for (int c = col_lo; c < col_lo + kPairCols; c += 4) {
       const int col = ntile * 256 + c;
       if (col >= p.N) break;
       *reinterpret_cast<float4*>(obase + static_cast<long long>(row) * p.ldo + col) = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1113,7 +1120,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;
     const int ew = warp - 2;
-    const int col_lo = (ew >> 2) * 128;
+    const int col_lo = (ew >> 2) * kPairCols;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     uint8_t* buf = staging + ew * 4096;  // one 32 x 32 float32 chunk, rows swizzled as the TMA expects
     const uint32_t row_addr = smem_u32(buf) + lane * 128;
@@ -1143,12 +1150,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         break;
       }
       tc_fence_after();
+      const uint32_t tempty_addr = tempty_leader + static_cast<uint32_t>(acc * 8);
       pair_drain(maps, p, tmem_base + lane_off + static_cast<uint32_t>(acc * 256), col_lo, ntile, row0, g, buf,
-                 row_addr, lane);
-      __syncwarp();
-      tc_fence_before();
-      // hand the accumulator back to the leader's MMA warp
-      mbar_arrive_cluster(tempty_leader + static_cast<uint32_t>(acc * 8));
+                 row_addr, lane, tempty_addr);
+      if (!MOE_PAIR_EARLY) {
+        __syncwarp();
+        tc_fence_before();
+        // hand the accumulator back to the leader's MMA warp
+        mbar_arrive_cluster(tempty_addr);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }

@@ -75,6 +75,10 @@ WORKLOADS = {1: TINY, 2: MID, 3: FULL, 4: SKEWED, 5: TRAIN}
 # over 4 destinations and T=1024, so each expert still receives ~341 of C_r=393 rows
 # as in the full layer, with ~4.5 GB on the device instead of ~50 GB.
 PROFILE = TRAIN.with_(name="profile", T=1024, n_experts=24, n_dest=4, seed=5)
+# The forward with the same 24 experts and T=8192: the routing and movement kernels move
+# 50 MB to 400 MB per launch (their traffic does not depend on the expert count), beyond
+# L2, with ~4 GB on the device.
+PROFILE_MOVERS = FULL.with_(name="profile_movers", T=8192, n_experts=24, n_dest=4, seed=6)
 # the dropless variant of the full-width training step and of the skewed stress
 TRAIN_DROPLESS = TRAIN.with_(name="train_dropless", dropless=True)
 SKEWED_DROPLESS = SKEWED.with_(name="skewed_dropless", dropless=True)
