@@ -41,8 +41,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # captured ones, and as null once they change.
 NCU_TRAFFIC = {
     "bwd.experts_wgrad_gate_up": {
-        "sources_sha256": "b8180b322e5c65f9c4f5b29f722025f314cf24729e6e9241eb2720eef64c3dc6",
-        "dram_bytes": 1918638848, "experts": 24, "tokens": 1024, "d_latent": 3072, "hidden_routed": 3072,
+        "sources_sha256": "2ad97d30aee5f9e57042a956aabda2cacb4f6731e7f608ad1f475937aa62bf08",
+        "dram_bytes": 1917320960, "experts": 24, "tokens": 1024, "d_latent": 3072, "hidden_routed": 3072,
     },
 }
 KERNEL_SOURCES = ("gemm_sm100.cu", "ptx.cuh")  # the GEMM kernels and the PTX they use
