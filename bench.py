@@ -80,6 +80,7 @@ def workload_shape(name):
     return {"train": synth.TRAIN, "full": synth.FULL, "mid": synth.MID, "skewed": synth.SKEWED,
             "tiny": synth.TINY.with_(backward=True), "profile": synth.PROFILE,
             "profile_movers": synth.PROFILE_MOVERS,
+            "profile_router": synth.PROFILE_ROUTER,
             "train_dropless": synth.TRAIN_DROPLESS, "skewed_dropless": synth.SKEWED_DROPLESS}[name]
 
 

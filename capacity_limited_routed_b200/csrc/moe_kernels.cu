@@ -79,23 +79,19 @@ __global__ void route_topk_kernel(const float* __restrict__ logits, const float*
         sc[i] = -INFINITY;
       }
     }
-    // each lane's best unchosen logit; after a round only the lane that supplied the
-    // winner looks again
-    float lbv = -INFINITY;
-    int lbe = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const int e = i * 32 + lane;
-      if (e < E && better(sc[i], e, lbv, lbe)) {
-        lbv = sc[i];
-        lbe = e;
-      }
-    }
     float my_raw = 0.0f;  // lane j < k keeps the raw logit of its rank-j choice
     int my_e = 0;
     for (int j = 0; j < k; ++j) {
-      float bv = lbv;
-      int be = lbe;
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int e = i * 32 + lane;
+        if (e < E && !((chosen >> i) & 1u) && better(sc[i], e, bv, be)) {
+          bv = sc[i];
+          be = e;
+        }
+      }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) {
         const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
@@ -105,26 +101,16 @@ __global__ void route_topk_kernel(const float* __restrict__ logits, const float*
           be = oe;
         }
       }
-      // be is now the same on every lane; its owner marks it, shares the raw logit and
-      // finds its next best
+      // be is now the same on every lane; its owner marks it and shares the raw logit
       const int owner = be & 31;
+      const int slot = be >> 5;
       float r = 0.0f;
-      if (lane == owner) {
-        const int slot = be >> 5;
-        lbv = -INFINITY;
-        lbe = 0x7fffffff;
 #pragma unroll
-        for (int i = 0; i < VPL; ++i) {
-          const int e = i * 32 + lane;
-          if (i == slot) {
-            chosen |= 1u << i;
-            r = raw[i];
-          } else if (e < E && !((chosen >> i) & 1u) && better(sc[i], e, lbv, lbe)) {
-            lbv = sc[i];
-            lbe = e;
-          }
+      for (int i = 0; i < VPL; ++i)
+        if (i == slot && lane == owner) {
+          chosen |= 1u << i;
+          r = raw[i];
         }
-      }
       r = __shfl_sync(0xffffffffu, r, owner);
       if (lane == j) {
         my_raw = r;

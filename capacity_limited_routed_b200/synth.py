@@ -79,6 +79,10 @@ PROFILE = TRAIN.with_(name="profile", T=1024, n_experts=24, n_dest=4, seed=5)
 # 50 MB to 400 MB per launch (their traffic does not depend on the expert count), beyond
 # L2, with ~4 GB on the device.
 PROFILE_MOVERS = FULL.with_(name="profile_movers", T=8192, n_experts=24, n_dest=4, seed=6)
+# The routing kernels at the full layer's size (T=16384, 384 experts top-8, 64 x 3 pools,
+# latent 3072) with the routed hidden width cut to 256, so ~5 GB sit on the device: the
+# router, top-k and slot scan see exactly the full layer's inputs.
+PROFILE_ROUTER = FULL.with_(name="profile_router", hidden_routed=256, seed=8)
 # the dropless variant of the full-width training step and of the skewed stress
 TRAIN_DROPLESS = TRAIN.with_(name="train_dropless", dropless=True)
 SKEWED_DROPLESS = SKEWED.with_(name="skewed_dropless", dropless=True)
