@@ -566,9 +566,11 @@ def main():
     barrier()
     launches = (M.moe_kernel_launches() - launches0) if graph is None else graph_launches * args.steps
     ms = ev0.elapsed_time(ev1)
-    # the same K steps again with the library's per-step CUDA events on (two events around
-    # each named step cost ~1.3% of the step, so they stay out of the region above): the
-    # per-kernel table and the roofline come from this second timed region
+    # the same K steps again, launched one by one with the library's per-step CUDA events on
+    # (two events around each named step cost ~1.3% of the step, so they stay out of the
+    # region above) and every step in order on one stream (so no step's event time includes
+    # another's): the per-kernel table and the roofline come from this second timed region
+    M.moe_set_side_stream(False)  # each step's event time its own: the shared experts in order
     M.moe_profile_start()
     ev2 = torch.cuda.Event(enable_timing=True)
     ev3 = torch.cuda.Event(enable_timing=True)
@@ -581,6 +583,7 @@ def main():
     torch.cuda.synchronize()
     barrier()
     prof = M.moe_profile_stop()
+    M.moe_set_side_stream(True)
     ms_prof = ev2.elapsed_time(ev3)
     clk = clocks.stop()
     ms_t = torch.tensor([ms, ms_prof], dtype=torch.float64, device=dev)
@@ -686,12 +689,11 @@ def main():
             "roofline": roof,
             "dispatch_hbm_frac": kernels.get("fwd.dispatch_pack", {}).get("frac"),
             "kernels": kernels,
-            "kernels_note": ("per training step, from a second timed region of the same K steps with the "
-                             "library's per-step CUDA events on (ms_per_step_profiled; the events stay out of "
-                             "the region that gives value); the shared experts run on a second stream (forward: "
-                             "beside the routing, slot scan, pack, unpack and first routed launches; backward: "
-                             "beside un-dispatch and the router's backward), so those steps' event times include "
-                             "time spent sharing the GPU, and the times add up to more than the step"),
+            "kernels_note": ("per training step, from a second timed region of the same K steps launched one "
+                             "by one with the library's per-step CUDA events on and every step in order on one "
+                             "stream (ms_per_step_profiled); the region that gives value replays a CUDA graph "
+                             "with the shared experts on a second stream beside the routing and movement "
+                             "kernels and no per-step events"),
             "ms_per_step_profiled": ms_prof_max / args.steps,
             "cpu_baseline": cpu,
             "e2e": e2e,

@@ -298,7 +298,17 @@ struct SideStream {
   cudaEvent_t fork = nullptr, join = nullptr;
 };
 
-moe_status_t side_stream(SideStream** out) {
+std::atomic<int> g_use_side_stream{1};
+
+// the side stream, or (moe_set_side_stream(0)) the caller's stream itself with no fork or join
+moe_status_t side_stream(SideStream** out, cudaStream_t st) {
+  if (g_use_side_stream.load(std::memory_order_relaxed) == 0) {
+    thread_local SideStream inline_ss;
+    inline_ss.s = st;
+    inline_ss.fork = inline_ss.join = nullptr;
+    *out = &inline_ss;
+    return MOE_OK;
+  }
   thread_local SideStream per_dev[kMaxDevices];
   const int dev = current_device();
   if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device index out of range for the side stream");
@@ -314,12 +324,14 @@ moe_status_t side_stream(SideStream** out) {
 
 // side stream waits for everything issued so far on st
 moe_status_t fork_to(SideStream* ss, cudaStream_t st) {
+  if (ss->fork == nullptr) return MOE_OK;  // the caller's stream itself
   MOE_TRY(cuda_check(cudaEventRecord(ss->fork, st), "fork record"));
   return cuda_check(cudaStreamWaitEvent(ss->s, ss->fork, 0), "fork wait");
 }
 
 // st waits for everything issued so far on the side stream
 moe_status_t join_from(SideStream* ss, cudaStream_t st) {
+  if (ss->join == nullptr) return MOE_OK;
   MOE_TRY(cuda_check(cudaEventRecord(ss->join, ss->s), "join record"));
   return cuda_check(cudaStreamWaitEvent(st, ss->join, 0), "join wait");
 }
@@ -616,6 +628,12 @@ moe_status_t moe_profile_stop(moe_profile_record_t* out, int32_t cap, int32_t* c
 
 int64_t moe_kernel_launches(void) { return launches_so_far(); }
 
+moe_status_t moe_set_side_stream(int32_t side_stream) {
+  if (side_stream != 0 && side_stream != 1) return fail(MOE_ERR_INVALID_ARG, "side_stream must be 0 or 1");
+  g_use_side_stream.store(side_stream, std::memory_order_relaxed);
+  return MOE_OK;
+}
+
 moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out) {
   if (cfg == nullptr || out == nullptr) return fail(MOE_ERR_INVALID_ARG, "null argument");
   *out = nullptr;
@@ -871,7 +889,7 @@ moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const uint16_t* x
   // shared experts on the side stream, beside the routing, movement and expert kernels:
   // H_s = silu(x ws1^T) * (x ws3^T)
   SideStream* ss = nullptr;
-  MOE_TRY(side_stream(&ss));
+  MOE_TRY(side_stream(&ss, st));
   MOE_TRY(fork_to(ss, st));
   {
     ProfScope ps("fwd.shared_gate_up", ss->s);
@@ -1024,7 +1042,7 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
   // backward (joined before dx): dH_s = dy ws2 -> SwiGLU backward -> (dA_s, dB_s);
   // dws2 = dy^T H_s;  dws1 = dA_s^T x, dws3 = dB_s^T x
   SideStream* ss = nullptr;
-  MOE_TRY(side_stream(&ss));
+  MOE_TRY(side_stream(&ss, st));
   MOE_TRY(fork_to(ss, st));
   {
     ProfScope ps("bwd.shared_dgrad_swiglu", ss->s);
@@ -1291,7 +1309,7 @@ moe_status_t moe_ep_forward_send(moe_plan_t p, const moe_weights_t* w, const uin
   int32_t* status = s + 3;
   const int64_t SH = int64_t(p->S) * p->hs;
   SideStream* ss = nullptr;
-  MOE_TRY(side_stream(&ss));
+  MOE_TRY(side_stream(&ss, st));
   MOE_TRY(fork_to(ss, st));
   if (g.T > 0) {
     ProfScope ps("fwd.shared_gate_up", ss->s);
@@ -1423,7 +1441,7 @@ moe_status_t moe_ep_backward_send(moe_plan_t p, const moe_weights_t* w, const vo
   if (!x || !dy) return fail(MOE_ERR_INVALID_ARG, "null buffer");
   EpPtrs c = ep_ptrs(*p, saved, ws);
   SideStream* ss = nullptr;
-  MOE_TRY(side_stream(&ss));
+  MOE_TRY(side_stream(&ss, st));
   MOE_TRY(fork_to(ss, st));
   {
     ProfScope ps("bwd.shared_dgrad_swiglu", ss->s);

@@ -18,6 +18,7 @@ EXPORTS = (
     "moe_plan_create", "moe_plan_destroy", "moe_plan_info", "moe_route", "moe_dispatch", "moe_dispatch_noalloc",
     "moe_expert_ffn", "moe_combine", "moe_forward", "moe_backward", "moe_bias_update",
     "moe_saved_view", "moe_gemm_bf16", "moe_profile_start", "moe_profile_stop", "moe_kernel_launches",
+    "moe_set_side_stream",
     "moe_last_error", "moe_ep_view", "moe_ep_forward_send", "moe_ep_forward_experts", "moe_ep_forward_combine",
     "moe_ep_backward_send", "moe_ep_backward_experts", "moe_ep_backward_finish",
 )
@@ -100,6 +101,7 @@ def _load():
         "moe_saved_view": [P, P, ctypes.POINTER(moe_saved_view_t)],
         "moe_gemm_bf16": [I, I, I, P, I, P, I, P, I, P, P],
         "moe_profile_start": [],
+        "moe_set_side_stream": [I],
         "moe_profile_stop": [ctypes.POINTER(moe_profile_record_t), I, ctypes.POINTER(I)],
         "moe_ep_view": [P, P, P, ctypes.POINTER(moe_ep_view_t)],
         "moe_ep_forward_send": [P, ctypes.POINTER(moe_weights_t), P, P, P, P, P, P, S, P],
@@ -277,6 +279,12 @@ def moe_profile_stop(cap: int = 65536) -> list[tuple[str, float, int]]:
     n = ctypes.c_int32(0)
     _check(_lib.moe_profile_stop(buf, cap, ctypes.byref(n)), "moe_profile_stop")
     return [(buf[i].name.decode(), float(buf[i].ms), int(buf[i].launches)) for i in range(min(n.value, cap))]
+
+
+def moe_set_side_stream(enable: bool) -> None:
+    """Shared experts on the library's second stream (True, the default) or in order on
+    the caller's stream (False)."""
+    _check(_lib.moe_set_side_stream(1 if enable else 0), "moe_set_side_stream")
 
 
 def moe_kernel_launches() -> int:

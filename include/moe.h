@@ -396,6 +396,17 @@ MOE_API moe_status_t moe_profile_stop(moe_profile_record_t* out, int32_t cap, in
 /* Kernels launched by this library since it was loaded. */
 MOE_API int64_t moe_kernel_launches(void);
 
+/* Streams of moe_forward / moe_backward.  side_stream = 1 (the default): the shared
+ * experts, which do not depend on routing, run on a second stream of this library that
+ * forks from the caller's stream by an event and joins back by another (forward: beside
+ * the routing, slot scan, dispatch, unpack and first routed launches; backward: beside
+ * un-dispatch and the router's backward).  side_stream = 0: every step of a call runs in
+ * order on the caller's stream, so per-step event times (moe_profile_start) are each
+ * step's own.  The results are the same either way.  Process-wide; takes effect for calls
+ * made after it returns.  Any value other than 0 or 1 is rejected with
+ * MOE_ERR_INVALID_ARG. */
+MOE_API moe_status_t moe_set_side_stream(int32_t side_stream);
+
 /* Message for the last failing call on this thread ("" if none). */
 MOE_API const char* moe_last_error(void);
 

@@ -103,6 +103,12 @@ def test_null_arguments_are_rejected(M):
     assert lib.moe_dispatch(p.handle, fake, fake, fake, fake, fake, fake, 16, None) == 3
 
 
+def test_side_stream_switch_rejects_other_values(M):
+    lib = M.lib()
+    assert lib.moe_set_side_stream(2) == 1 and lib.moe_set_side_stream(-1) == 1
+    assert lib.moe_set_side_stream(0) == 0 and lib.moe_set_side_stream(1) == 0
+
+
 def test_dropless_plan_sizes(M):
     """Both capacity numerators 0 select the dropless variant: no caps, pools packed to
     T*k rows, expert buffers packed by expert with each expert padded to 128 rows."""

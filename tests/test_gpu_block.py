@@ -157,3 +157,23 @@ def test_backward_idle_experts_get_zero_gradients():
         assert np.isfinite(got).all(), name
         busy = ~idle & np.array([e not in affected for e in range(s.n_experts)])
         assert_close_rms(got[busy], grads_o[name][busy], tol=ROUTED_GRAD_TOL, what=f"d{name}")
+
+
+def test_side_stream_off_gives_identical_results():
+    """moe_set_side_stream(0) runs the shared experts in order on the caller's stream; the
+    outputs, dx, every gradient and the statistics must be bit for bit those of the default
+    (shared experts on the second stream)."""
+    from capacity_limited_routed_b200 import moe as M
+    runs = []
+    try:
+        for on in (True, False):
+            M.moe_set_side_stream(on)
+            r = _run(synth.MID.with_(T=2048, seed=33), backward=True)
+            runs.append((r["y"].clone(), r["dx"].clone(), {n: g.clone() for n, g in r["blk"].grads.items()},
+                         r["blk"].stats.clone()))
+    finally:
+        M.moe_set_side_stream(True)
+    (y0, dx0, g0, st0), (y1, dx1, g1, st1) = runs
+    assert torch.equal(y0, y1) and torch.equal(dx0, dx1) and torch.equal(st0, st1)
+    for n in g0:
+        assert torch.equal(g0[n], g1[n]), n
