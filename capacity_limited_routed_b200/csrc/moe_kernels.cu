@@ -45,19 +45,51 @@ __device__ __forceinline__ bool better(float v, int e, float bv, int be) {
 
 // ---------------------------------------------------------------------- routing
 
+// Sort 32 distinct (score, expert, raw) keys across the warp, best first under `better`
+// (bitonic network over the lanes: lane 0 ends with the best).
+__device__ __forceinline__ void warp_sort_best_first(float& v, int& e, float& r, int lane) {
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const float pv = __shfl_xor_sync(0xffffffffu, v, stride);
+      const int pe = __shfl_xor_sync(0xffffffffu, e, stride);
+      const float pr = __shfl_xor_sync(0xffffffffu, r, stride);
+      const bool lower = (lane & stride) == 0;
+      const bool best_first = (lane & size) == 0;  // direction of this block of the network
+      const bool pb = better(pv, pe, v, e);
+      if ((lower == best_first) ? pb : !pb) {
+        v = pv;
+        e = pe;
+        r = pr;
+      }
+    }
+  }
+}
+
+// One warp per token.  The k-th best of the 32 lane maxima bounds the k-th best score from
+// below (the k best lane maxima are k distinct scores at or above it), so the top k are
+// among the scores not worse than it; those candidates (usually a few more than k) are
+// gathered with ballots and sorted across the warp.  More than 32 candidates (many equal
+// scores) take k rounds of warp arg-max instead.  Either way the result is the exact top k
+// under (score descending, expert ascending), in that order.
 template <int VPL>
-__global__ void route_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E,
+__global__ void __launch_bounds__(256, 3) route_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E,
                                   int k, int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
                                   int32_t* __restrict__ hist, int32_t* __restrict__ nan_count) {
   // hist == nullptr: the histogram is left to the slot scan, which counts every assignment
   __shared__ int sh_hist[kMaxE];
+  __shared__ float sh_cv[8][32], sh_cr[8][32];  // candidates of each warp (blocks of <= 8 warps)
+  __shared__ int sh_ce[8][32];
   if (hist != nullptr)
     for (int e = threadIdx.x; e < E; e += blockDim.x) sh_hist[e] = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
   const int warps = blockDim.x >> 5;
-  const int gw = blockIdx.x * warps + (threadIdx.x >> 5);
+  const int gw = blockIdx.x * warps + wib;
   const int nw = gridDim.x * warps;
+  const unsigned lt_mask = (1u << lane) - 1u;
   float bsv[VPL];
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
@@ -68,7 +100,8 @@ __global__ void route_topk_kernel(const float* __restrict__ logits, const float*
   for (int t = gw; t < T; t += nw) {
     const float* row = logits + static_cast<long long>(t) * E;
     float raw[VPL], sc[VPL];
-    unsigned chosen = 0;
+    float mv = -INFINITY;
+    int me = 0x7fffffe0 + lane;  // a lane with no expert ranks below every expert
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int e = i * 32 + lane;
@@ -78,43 +111,93 @@ __global__ void route_topk_kernel(const float* __restrict__ logits, const float*
         ++nan_local;          // input error, counted; the expert ranks last
         sc[i] = -INFINITY;
       }
+      if (e < E && better(sc[i], e, mv, me)) {
+        mv = sc[i];
+        me = e;
+      }
     }
+    // threshold: the k-th best lane maximum
+    float tv = mv, tr = 0.0f;
+    int te = me;
+    warp_sort_best_first(tv, te, tr, lane);
+    tv = __shfl_sync(0xffffffffu, tv, k - 1);
+    te = __shfl_sync(0xffffffffu, te, k - 1);
+    // candidates: scores not worse than the threshold
+    int cnt = 0;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = i * 32 + lane;
+      cnt += (e < E && !better(tv, te, sc[i], e)) ? 1 : 0;
+    }
+    int total = cnt;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) total += __shfl_xor_sync(0xffffffffu, total, off);
     float my_raw = 0.0f;  // lane j < k keeps the raw logit of its rank-j choice
     int my_e = 0;
-    for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
+    if (total <= 32) {
+      int base = 0;
 #pragma unroll
       for (int i = 0; i < VPL; ++i) {
         const int e = i * 32 + lane;
-        if (e < E && !((chosen >> i) & 1u) && better(sc[i], e, bv, be)) {
-          bv = sc[i];
-          be = e;
+        const bool c = e < E && !better(tv, te, sc[i], e);
+        const unsigned m = __ballot_sync(0xffffffffu, c);
+        if (c) {
+          const int pos = base + __popc(m & lt_mask);
+          sh_cv[wib][pos] = sc[i];
+          sh_ce[wib][pos] = e;
+          sh_cr[wib][pos] = raw[i];
         }
+        base += __popc(m);
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        if (better(ov, oe, bv, be)) {
-          bv = ov;
-          be = oe;
-        }
+      __syncwarp();
+      float cv = -INFINITY, cr = 0.0f;
+      int ce = 0x7fffffe0 + lane;
+      if (lane < total) {
+        cv = sh_cv[wib][lane];
+        ce = sh_ce[wib][lane];
+        cr = sh_cr[wib][lane];
       }
-      // be is now the same on every lane; its owner marks it and shares the raw logit
-      const int owner = be & 31;
-      const int slot = be >> 5;
-      float r = 0.0f;
+      __syncwarp();
+      warp_sort_best_first(cv, ce, cr, lane);
+      my_raw = cr;
+      my_e = ce;
+    } else {
+      unsigned chosen = 0;
+      for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int be = 0x7fffffff;
 #pragma unroll
-      for (int i = 0; i < VPL; ++i)
-        if (i == slot && lane == owner) {
-          chosen |= 1u << i;
-          r = raw[i];
+        for (int i = 0; i < VPL; ++i) {
+          const int e = i * 32 + lane;
+          if (e < E && !((chosen >> i) & 1u) && better(sc[i], e, bv, be)) {
+            bv = sc[i];
+            be = e;
+          }
         }
-      r = __shfl_sync(0xffffffffu, r, owner);
-      if (lane == j) {
-        my_raw = r;
-        my_e = be;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+          const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+          if (better(ov, oe, bv, be)) {
+            bv = ov;
+            be = oe;
+          }
+        }
+        // be is now the same on every lane; its owner marks it and shares the raw logit
+        const int owner = be & 31;
+        const int slot = be >> 5;
+        float r = 0.0f;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i)
+          if (i == slot && lane == owner) {
+            chosen |= 1u << i;
+            r = raw[i];
+          }
+        r = __shfl_sync(0xffffffffu, r, owner);
+        if (lane == j) {
+          my_raw = r;
+          my_e = be;
+        }
       }
     }
     // softmax over the k chosen raw logits (lanes 0..k-1)

@@ -60,6 +60,38 @@ def test_route_signed_zero_and_empty(M):
     assert np.allclose(gate.cpu().numpy(), 1.0 / s.top_k)
 
 
+@pytest.mark.parametrize("shape", [
+    synth.TINY,
+    synth.MoEShape("e48k3", T=333, d_model=192, d_latent=128, n_experts=48, top_k=3, n_dest=8,
+                   hidden_routed=128, n_shared=1, hidden_shared=128, seed=41),
+    synth.MoEShape("e48k12", T=200, d_model=192, d_latent=128, n_experts=48, top_k=12, n_dest=8,
+                   hidden_routed=128, n_shared=1, hidden_shared=128, seed=42),
+    synth.MoEShape("e96k20", T=130, d_model=192, d_latent=192, n_experts=96, top_k=20, n_dest=8,
+                   hidden_routed=128, n_shared=1, hidden_shared=128, seed=43),
+    synth.MoEShape("e384k8", T=300, d_model=256, d_latent=256, n_experts=384, top_k=8, n_dest=64,
+                   hidden_routed=128, n_shared=1, hidden_shared=128, seed=44),
+], ids=lambda s: s.name)
+def test_forward_topk_matches_moe_route(M, shape):
+    """The forward's topk_idx and topk_gate must be bit for bit what moe_route makes of the
+    logits and bias the forward saved (T not a multiple of 128, k up to 20, E up to 384)."""
+    from capacity_limited_routed_b200.block import MoEBlock
+    inp = synth.make_inputs(shape)
+    blk = MoEBlock(shape, training=True)
+    blk.load(inp)
+    blk.forward(bf16_dev(inp["x"]))
+    torch.cuda.synchronize()
+    v = blk.saved_views()
+    T, k, E = shape.T, shape.top_k, shape.n_experts
+    idx = torch.full((T, k), -7, dtype=torch.int32, device=dev())
+    gate = torch.zeros((T, k), dtype=torch.float32, device=dev())
+    hist = torch.zeros((E,), dtype=torch.int32, device=dev())
+    M.moe_route(blk.plan, v["logits"], blk.bias, idx, gate, hist)
+    torch.cuda.synchronize()
+    assert torch.equal(v["topk_idx"], idx)
+    assert torch.equal(v["topk_gate"], gate)
+    assert int(blk.stats_dict()["nan_logits"]) == 0
+
+
 # ------------------------------------------------------------------ dispatch
 
 
