@@ -177,6 +177,8 @@ moe_status_t launch_undispatch(const Geo& g, const uint16_t* dxe, const float* g
                                const int32_t* idx, const int32_t* slot, float* dz_routed, uint16_t* dlogits,
                                cudaStream_t st, const int32_t* exp_off = nullptr, bool by_pool = false);
 moe_status_t launch_bias_update(const Geo& g, const int32_t* hist, float* bias, float step, cudaStream_t st);
+// out[i] = sum over s < S of part[s * n + i], float32, s in order (n a multiple of 4)
+moe_status_t launch_sum_partials(const float* part, int S, long long n, float* out, cudaStream_t st);
 
 // plan geometry and the device check, for entry points defined in other files
 const Geo& plan_geo(const moe_plan* p);

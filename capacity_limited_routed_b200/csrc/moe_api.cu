@@ -401,6 +401,44 @@ void pack_groups(const Geo& g, GemmArgs& a, const int32_t* exp_off) {
   if (a.ragged == 1) a.M = static_cast<int>(g.exp_rows);  // local rows never reach it
 }
 
+// dW_r = dlogits^T z over the T tokens.  With K = T long and few output tiles (E x d_latent:
+// 2 x 12 pair tiles at full width for 74 pairs) the tokens are split into S equal slices,
+// computed as S groups of one launch into float32 partials in `scratch` (when it holds them)
+// and summed in slice order.
+moe_status_t router_wgrad(int E, int dl, int64_t T, const uint16_t* dlog, const uint16_t* z, float* out,
+                          void* scratch, size_t scratch_bytes, cudaStream_t st) {
+  const long long tiles = static_cast<long long>((E + 255) / 256) * ((dl + 255) / 256);
+  int S = 1;
+  for (int c = 4; c >= 2; c /= 2)
+    if (T % c == 0 && T / c >= 1024 && tiles * c <= 2LL * device_sm_count() &&
+        static_cast<size_t>(c) * E * dl * 4 <= scratch_bytes && (static_cast<long long>(E) * dl) % 4 == 0) {
+      S = c;
+      break;
+    }
+  GemmArgs a;
+  a.a_mn = a.b_mn = true;
+  a.epi = EPI_F32;
+  a.M = E;
+  a.N = dl;
+  a.ldo = dl;
+  if (S == 1) {
+    a.A[0] = mat(dlog, E, T);
+    a.B[0] = mat(z, dl, T);
+    a.K[0] = T;
+    a.out = out;
+    return gemm_run(a, st);
+  }
+  const int64_t Ts = T / S;
+  a.groups = S;
+  a.A[0] = mat(dlog, E, Ts, S);
+  a.B[0] = mat(z, dl, Ts, S);
+  a.K[0] = Ts;
+  a.out = scratch;
+  a.out_gs = static_cast<int64_t>(E) * dl;
+  MOE_TRY(gemm_run(a, st));
+  return launch_sum_partials(static_cast<const float*>(scratch), S, static_cast<long long>(E) * dl, out, st);
+}
+
 // receiver unpack + grouped SwiGLU experts (shared by moe_expert_ffn, moe_forward and the
 // expert-parallel receiver): the receiver copies its kept rows into the expert buffers xe.
 // g: the receiver's geometry; E its experts (weights [E][..]), dl, h the widths; id_base the
@@ -1111,18 +1149,10 @@ moe_status_t moe_backward(moe_plan_t p, const moe_weights_t* w, const void* save
     MOE_TRY(gemm_run(a, st));
   }
   {
+    // the routed backward's dA buffer is free again here: it holds the split's partials
     ProfScope ps("bwd.router_wgrad", st);
-    GemmArgs a;
-    a.a_mn = a.b_mn = true;
-    a.epi = EPI_F32;
-    a.M = static_cast<int>(E);
-    a.N = static_cast<int>(dl);
-    a.A[0] = mat(dlog, E, T);
-    a.B[0] = mat(c.z, dl, T);
-    a.K[0] = T;
-    a.out = gr->w_router;
-    a.ldo = dl;
-    MOE_TRY(gemm_run(a, st));
+    MOE_TRY(router_wgrad(static_cast<int>(E), static_cast<int>(dl), T, dlog, c.z, gr->w_router, dae,
+                         p->b_dbe - p->b_dae, st));
   }
   MOE_TRY(join_from(ss, st));
   // dx = dz W_down + dA_s ws1 + dB_s ws3 (three K segments), float32 out
@@ -1559,6 +1589,7 @@ moe_status_t moe_ep_backward_finish(moe_plan_t p, const moe_weights_t* w, const 
   }
   if (!x || !dx) return fail(MOE_ERR_INVALID_ARG, "null buffer");
   EpPtrs c = ep_ptrs(*p, saved, ws);
+  const size_t dae_bytes = p->ep.dbe - p->ep.dae;
   {
     ProfScope ps("bwd.undispatch", st);
     MOE_TRY(launch_undispatch(g, c.dx_in, c.gate, c.dg, c.idx, c.slot, c.dzr, c.dlog, st, nullptr, true));
@@ -1581,18 +1612,10 @@ moe_status_t moe_ep_backward_finish(moe_plan_t p, const moe_weights_t* w, const 
     MOE_TRY(gemm_run(a, st));
   }
   {
+    // the receiver's dA buffer is free again here: it holds the split's partials
     ProfScope ps("bwd.router_wgrad", st);
-    GemmArgs a;
-    a.a_mn = a.b_mn = true;
-    a.epi = EPI_F32;
-    a.M = static_cast<int>(E);
-    a.N = static_cast<int>(dl);
-    a.A[0] = mat(c.dlog, E, T);
-    a.B[0] = mat(c.z, dl, T);
-    a.K[0] = T;
-    a.out = gr->w_router;
-    a.ldo = dl;
-    MOE_TRY(gemm_run(a, st));
+    MOE_TRY(router_wgrad(static_cast<int>(E), static_cast<int>(dl), T, c.dlog, c.z, gr->w_router, c.dae,
+                         dae_bytes, st));
   }
   {
     ProfScope ps("bwd.dx", st);

@@ -1054,6 +1054,23 @@ __global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict
   if (threadIdx.x == 0) off[n] = s_carry;
 }
 
+// out[i] = sum over s of part[s][i] (float32, s in order): the K slices of a split weight
+// gradient
+__global__ void sum_partials_kernel(const float4* __restrict__ part, int S, long long n4, float4* __restrict__ out) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float4 a = part[i];
+    for (int s = 1; s < S; ++s) {
+      const float4 b = part[s * n4 + i];
+      a.x += b.x;
+      a.y += b.y;
+      a.z += b.z;
+      a.w += b.w;
+    }
+    out[i] = a;
+  }
+}
+
 // ====================================================================== launchers
 
 moe_status_t launch_route(const Geo& g, const float* logits, const float* bias, int32_t* idx, float* gate,
@@ -1247,6 +1264,16 @@ moe_status_t launch_undispatch(const Geo& g, const uint16_t* dxe, const float* g
                                                                    row_addr(g, exp_off, by_pool));
   count_launch();
   return cuda_check(cudaGetLastError(), "undispatch");
+}
+
+moe_status_t launch_sum_partials(const float* part, int S, long long n, float* out, cudaStream_t st) {
+  if (n <= 0) return MOE_OK;
+  if (n % 4 != 0) return fail(MOE_ERR_UNSUPPORTED, "partial sums need a multiple of 4 elements");
+  const long long n4 = n / 4;
+  const int grid = static_cast<int>(std::min<long long>((n4 + 255) / 256, 4LL * device_sm_count()));
+  sum_partials_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(part), S, n4, reinterpret_cast<float4*>(out));
+  count_launch();
+  return cuda_check(cudaGetLastError(), "sum partials");
 }
 
 moe_status_t launch_bias_update(const Geo& g, const int32_t* hist, float* bias, float step, cudaStream_t st) {
