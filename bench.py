@@ -41,7 +41,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # captured ones, and as null once they change.
 NCU_TRAFFIC = {
     "bwd.experts_wgrad_gate_up": {
-        "sources_sha256": "2ad97d30aee5f9e57042a956aabda2cacb4f6731e7f608ad1f475937aa62bf08",
+        "sources_sha256": "afaf9881abd7eae8f8fbff6edbb3556277c872cd66f7ded112833393bba2dc9a",
         "dram_bytes": 1917320960, "experts": 24, "tokens": 1024, "d_latent": 3072, "hidden_routed": 3072,
     },
 }

@@ -74,14 +74,10 @@ __device__ __forceinline__ int expert_of(const KParams& p, int g) {
   return p.map_p > 0 ? (g / p.map_p) * p.map_l + p.map_off + g % p.map_p : g;
 }
 
-// Tuning of the weight-gradient (write-bound) instance: pipeline stages and staging
-// buffers per epilogue warp.
-#ifndef MOE_WB_STAGES
-#define MOE_WB_STAGES 4
-#endif
-#ifndef MOE_WB_BUFS
-#define MOE_WB_BUFS 1
-#endif
+// Pipeline stages and staging buffers per epilogue warp of the single-CTA weight-gradient
+// (write-bound) instance.
+constexpr int kWbStages = 4;
+constexpr int kWbBufs = 1;
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
@@ -107,9 +103,9 @@ struct Cfg {
   static constexpr int kABytes = kBM * kBK * 2;  // 16 KB
   static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * kBK * 2;  // a pair CTA holds half of B
   static constexpr int kStage = kABytes + kBBytes;
-  static constexpr int kStages = WRITE_BOUND ? MOE_WB_STAGES : ((BN == 256 && !PAIR) ? 4 : 6);
+  static constexpr int kStages = WRITE_BOUND ? kWbStages : ((BN == 256 && !PAIR) ? 4 : 6);
   static constexpr int kTmemCols = 2 * BN;
-  static constexpr int kBufs = WRITE_BOUND ? MOE_WB_BUFS : 1;  // staging buffers per epilogue warp
+  static constexpr int kBufs = WRITE_BOUND ? kWbBufs : 1;  // staging buffers per epilogue warp
   static constexpr int kEpiWarps = Roles<WRITE_BOUND>::kEpiWarps;
   // a buffer holds 32 rows x 128 bytes (float32 / bf16 outputs); the forward SwiGLU
   // stages three 32 x 64-byte tiles (H, a, b), its backward three slots of two 32 x
