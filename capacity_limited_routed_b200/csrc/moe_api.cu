@@ -411,7 +411,8 @@ moe_status_t router_wgrad(int E, int dl, int64_t T, const uint16_t* dlog, const 
   int S = 1;
   for (int c = 4; c >= 2; c /= 2)
     if (T % c == 0 && T / c >= 1024 && tiles * c <= 2LL * device_sm_count() &&
-        static_cast<size_t>(c) * E * dl * 4 <= scratch_bytes && (static_cast<long long>(E) * dl) % 4 == 0) {
+        static_cast<size_t>(c) * E * dl * 4 <= scratch_bytes && (static_cast<long long>(E) * dl) % 4 == 0 &&
+        (T / c) * E % 8 == 0 && (T / c) * dl % 8 == 0) {  // each slice 16-byte aligned
       S = c;
       break;
     }
