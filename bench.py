@@ -551,7 +551,7 @@ def main():
     if st0["status"] != 0:
         raise RuntimeError(f"kernel status {st0['status']} after warm-up")
 
-    # One GPU: the step (41 launches, its side-stream fork and join, the bias step) is captured
+    # One GPU: the step (its launches, side-stream fork and join, the bias step) is captured
     # once into a CUDA graph and replayed; the library allocates nothing and never syncs
     # inside a step, so the graph holds exactly the eager launches.  The launch count is
     # taken at capture, per step.
