@@ -81,6 +81,7 @@ def workload_shape(name):
             "tiny": synth.TINY.with_(backward=True), "profile": synth.PROFILE,
             "profile_movers": synth.PROFILE_MOVERS,
             "profile_router": synth.PROFILE_ROUTER,
+            "profile_router_train": synth.PROFILE_ROUTER_TRAIN,
             "train_dropless": synth.TRAIN_DROPLESS, "skewed_dropless": synth.SKEWED_DROPLESS}[name]
 
 

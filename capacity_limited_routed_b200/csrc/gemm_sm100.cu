@@ -515,6 +515,19 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
       if constexpr (EPI == EPI_SWIGLU_BWD) {
         if (lane == 0 && s_live > 0) swb_issue(0, eslot);
       }
+      // bf16 + float32 addend: the addend of this thread's row, 64 columns at a time, is
+      // loaded one piece ahead of its use; the first piece's load overlaps the MMAs
+      float4 ad[EPI == EPI_BF16_ADD_F32 ? 16 : 1];
+      auto load_addend = [&](int c) {
+        const int col = ntile * BN + c;
+        if (row_ok && col < p.N) {
+          const float* src = p.addend + static_cast<long long>(row) * p.add_ld + col;
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (col + 4 * i < p.N) ad[i] = *reinterpret_cast<const float4*>(src + 4 * i);
+        }
+      };
+      if constexpr (EPI == EPI_BF16_ADD_F32) load_addend(0);
       const bool got = mbar_wait(&tfull[acc], acc_phase, abort_v);
       __syncwarp();
       if (!__all_sync(0xffffffffu, got)) {
@@ -643,28 +656,31 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
                   make_uint4(a0, a1, a2, a3);
           }
         }
-      } else if constexpr (EPI == EPI_F32 || EPI == EPI_BF16) {
+      } else if constexpr (EPI == EPI_F32 || EPI == EPI_BF16 || EPI == EPI_BF16_ADD_F32) {
         // Four TMEM loads (128 columns) in flight before one wait, then the 128 columns
         // leave through shared memory: 32 rows x 128 bytes per staging buffer (128-byte
         // swizzle: 16-byte piece j of row r at j ^ (r & 7)), one TMA tensor store each.
         // Rows past M and columns past N are clipped by the tensor map.  The accumulator
-        // is released as soon as the whole tile is in registers.
+        // is released as soon as the whole tile is in registers.  With an addend, each
+        // 64-column piece gets its float32 addend before rounding to bf16.
         constexpr int kChunk = (EPI == EPI_F32) ? 32 : 64;  // columns per 128-byte row
+        // columns per TMEM wait (the addend's registers leave room for 64)
+        constexpr int kSpan = (EPI == EPI_BF16_ADD_F32) ? 64 : 128;
         const int row0 = mbase + q * 32;
 #pragma unroll 1
-        for (int half = 0; half < BN; half += 128) {
-          uint32_t r[4][32];
+        for (int half = 0; half < BN; half += kSpan) {
+          uint32_t r[kSpan / 32][32];
           __syncwarp();
 #pragma unroll
-          for (int i = 0; i < 4; ++i) tmem_ld_32cols_async(tbase + half + 32 * i, r[i]);
+          for (int i = 0; i < kSpan / 32; ++i) tmem_ld_32cols_async(tbase + half + 32 * i, r[i]);
           tmem_wait_ld();
-          if (half + 128 >= BN) {
+          if (half + kSpan >= BN) {
             tc_fence_before();
             release(acc);
             released = true;
           }
 #pragma unroll
-          for (int cc = 0; cc < 128 / kChunk; ++cc) {
+          for (int cc = 0; cc < kSpan / kChunk; ++cc) {
             uint32_t w[32];
             const int col0 = ntile * BN + half + cc * kChunk;
             // see the weight-gradient path: no buffer write without a committed store
@@ -677,6 +693,17 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
                 w[i] = __float_as_uint(x);
               }
             } else {
+              if constexpr (EPI == EPI_BF16_ADD_F32) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  uint32_t* x = &r[2 * cc + (i >> 3)][4 * (i & 7)];
+                  x[0] = __float_as_uint(__uint_as_float(x[0]) + ad[i].x);
+                  x[1] = __float_as_uint(__uint_as_float(x[1]) + ad[i].y);
+                  x[2] = __float_as_uint(__uint_as_float(x[2]) + ad[i].z);
+                  x[3] = __float_as_uint(__uint_as_float(x[3]) + ad[i].w);
+                }
+                if (half + (cc + 1) * kChunk < BN) load_addend(half + (cc + 1) * kChunk);
+              }
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
                 w[i] = pack_bf16x2(__uint_as_float(r[2 * cc][2 * i]), __uint_as_float(r[2 * cc][2 * i + 1]));
@@ -763,40 +790,7 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
           break;
         }
       } else {
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          float v[32];
-          __syncwarp();
-          tmem_ld_32cols(tbase + c, v);
-          const int col0 = ntile * BN + c;
-          if (row_ok && col0 < p.N) {
-          const long long off = g * p.out_gs + (long long)row * p.ldo + col0;
-          const int nvalid = p.N - col0;  // multiple of 8
-          if constexpr (EPI == EPI_BF16_ADD_F32) {
-            {
-              const float* ad = p.addend + (long long)row * p.add_ld + col0;
-#pragma unroll
-              for (int i = 0; i < 32; i += 4) {
-                if (i < nvalid) {
-                  const float4 f = *reinterpret_cast<const float4*>(ad + i);
-                  v[i] += f.x;
-                  v[i + 1] += f.y;
-                  v[i + 2] += f.z;
-                  v[i + 3] += f.w;
-                }
-              }
-            }
-            uint16_t* o = static_cast<uint16_t*>(p.out) + off;
-#pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              if (i < nvalid)
-                *reinterpret_cast<uint4*>(o + i) =
-                    make_uint4(pack_bf16x2(v[i], v[i + 1]), pack_bf16x2(v[i + 2], v[i + 3]),
-                               pack_bf16x2(v[i + 4], v[i + 5]), pack_bf16x2(v[i + 6], v[i + 7]));
-            }
-          }
-          }  // row_ok && col0 < N
-        }
+        static_assert(EPI < 0, "an epilogue without a branch");
       }
       __syncwarp();
       if (!released) {
@@ -1361,7 +1355,7 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
       if ((r = tile16(&maps.aux_b, a.aux_b, a.aux_ld, a.aux_gs, "b")) != MOE_OK) return r;
     }
   }
-  if (a.epi == EPI_F32 || a.epi == EPI_BF16) {
+  if (a.epi == EPI_F32 || a.epi == EPI_BF16 || a.epi == EPI_BF16_ADD_F32) {
     Mat o;
     o.ptr = a.out;
     o.inner = a.N;

@@ -83,6 +83,8 @@ PROFILE_MOVERS = FULL.with_(name="profile_movers", T=8192, n_experts=24, n_dest=
 # latent 3072) with the routed hidden width cut to 256, so ~5 GB sit on the device: the
 # router, top-k and slot scan see exactly the full layer's inputs.
 PROFILE_ROUTER = FULL.with_(name="profile_router", hidden_routed=256, seed=8)
+# the same with the backward and the bias step: the router's gradient GEMMs at full size
+PROFILE_ROUTER_TRAIN = PROFILE_ROUTER.with_(name="profile_router_train", backward=True)
 # the dropless variant of the full-width training step and of the skewed stress
 TRAIN_DROPLESS = TRAIN.with_(name="train_dropless", dropless=True)
 SKEWED_DROPLESS = SKEWED.with_(name="skewed_dropless", dropless=True)
