@@ -47,6 +47,25 @@ __device__ __forceinline__ bool better(float v, int e, float bv, int be) {
 
 // Sort 32 distinct (score, expert, raw) keys across the warp, best first under `better`
 // (bitonic network over the lanes: lane 0 ends with the best).
+__device__ __forceinline__ void warp_sort_best_first(float& v, int& e, int lane) {
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const float pv = __shfl_xor_sync(0xffffffffu, v, stride);
+      const int pe = __shfl_xor_sync(0xffffffffu, e, stride);
+      const bool lower = (lane & stride) == 0;
+      const bool best_first = (lane & size) == 0;  // direction of this block of the network
+      const bool pb = better(pv, pe, v, e);
+      if ((lower == best_first) ? pb : !pb) {
+        v = pv;
+        e = pe;
+      }
+    }
+  }
+}
+
+// the same network carrying a third value (the raw logit) with each key
 __device__ __forceinline__ void warp_sort_best_first(float& v, int& e, float& r, int lane) {
 #pragma unroll
   for (int size = 2; size <= 32; size <<= 1) {
@@ -97,15 +116,28 @@ __global__ void __launch_bounds__(256, 3) route_topk_kernel(const float* __restr
     bsv[i] = e < E ? bias[e] : 0.0f;
   }
   int nan_local = 0;
-  for (int t = gw; t < T; t += nw) {
+  // each warp walks tokens gw, gw + nw, ...; the next token's logits load while this
+  // token's experts are selected
+  float nxt[VPL];
+  auto load_row = [&](int t) {
     const float* row = logits + static_cast<long long>(t) * E;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = i * 32 + lane;
+      nxt[i] = e < E ? __ldcs(row + e) : 0.0f;
+    }
+  };
+  if (gw < T) load_row(gw);
+  for (int t = gw; t < T; t += nw) {
     float raw[VPL], sc[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) raw[i] = nxt[i];
+    if (t + nw < T) load_row(t + nw);
     float mv = -INFINITY;
     int me = 0x7fffffe0 + lane;  // a lane with no expert ranks below every expert
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int e = i * 32 + lane;
-      raw[i] = e < E ? row[e] : 0.0f;
       sc[i] = __fadd_rn(raw[i], bsv[i]);
       if (e < E && isnan(sc[i])) {
         ++nan_local;          // input error, counted; the expert ranks last
@@ -117,9 +149,9 @@ __global__ void __launch_bounds__(256, 3) route_topk_kernel(const float* __restr
       }
     }
     // threshold: the k-th best lane maximum
-    float tv = mv, tr = 0.0f;
+    float tv = mv;
     int te = me;
-    warp_sort_best_first(tv, te, tr, lane);
+    warp_sort_best_first(tv, te, lane);
     tv = __shfl_sync(0xffffffffu, tv, k - 1);
     te = __shfl_sync(0xffffffffu, te, k - 1);
     // candidates: scores not worse than the threshold
@@ -1082,10 +1114,17 @@ moe_status_t launch_route(const Geo& g, const float* logits, const float* bias, 
                           int32_t* hist, int32_t* nan_count, cudaStream_t st) {
   if (g.T == 0) return MOE_OK;
   const int warps = 8;
-  const int grid = blocks_for(g.T, warps);
   const int vpl = (g.E + 31) / 32;
+  // persistent: as many blocks as fit at once, each warp walking several tokens
 #define MOE_ROUTE(V)                                                                                       \
   if (vpl <= V) {                                                                                          \
+    int per_sm = 1;                                                                                        \
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_topk_kernel<V>, 32 * warps, 0) !=     \
+            cudaSuccess ||                                                                                 \
+        per_sm < 1)                                                                                        \
+      per_sm = 1;                                                                                          \
+    const int grid = static_cast<int>(                                                                     \
+        std::min<long long>(blocks_for(g.T, warps), static_cast<long long>(device_sm_count()) * per_sm));  \
     route_topk_kernel<V><<<grid, 32 * warps, 0, st>>>(logits, bias, g.T, g.E, g.k, idx, gate, hist, nan_count); \
     count_launch();                                                                                          \
     return cuda_check(cudaGetLastError(), "route_topk");                                                    \
