@@ -37,7 +37,6 @@ namespace moe {
 namespace {
 
 constexpr int kMaxE = 1024;
-constexpr int kVals = kMaxE / 32;  // logits held per lane
 
 __device__ __forceinline__ bool better(float v, int e, float bv, int be) {
   return v > bv || (v == bv && e < be);
@@ -324,6 +323,9 @@ __global__ void scan_rows(int32_t* __restrict__ data, int n, int32_t* __restrict
 }
 
 // pass C: one warp per chunk
+// rows of 32 assignments whose loads a scan warp issues before ranking them
+constexpr int kScanBatch = 8;
+
 __global__ void scan_sender_slots(const int32_t* __restrict__ idx, int A_total, int chunk_assign, int n_chunks,
                                   int L, int P, int W, int NP, int E, int Cs,
                                   const int32_t* __restrict__ base_pool, int32_t* __restrict__ slot,
@@ -339,32 +341,50 @@ __global__ void scan_sender_slots(const int32_t* __restrict__ idx, int A_total, 
   if (c >= n_chunks) return;
   const int a0 = c * chunk_assign;
   const int a1 = min(A_total, a0 + chunk_assign);
-  for (int it = a0; it < a1; it += 32) {
-    const int a = it + lane;
-    const int e_raw = a < a1 ? idx[a] : 0;
-    const bool bad = a < a1 && (e_raw < 0 || e_raw >= E);
-    if (bad) {
-      atomicCAS(status, 0, MOE_ERR_INVALID_ARG);
-      slot[2LL * a] = -1;
+  // up to kScanBatch rows of 32 assignments at a time: their expert ids, then their pools'
+  // bases, are loaded before the rows are ranked in order
+  for (int it0 = a0; it0 < a1; it0 += 32 * kScanBatch) {
+    int eb[kScanBatch], bb[kScanBatch];
+#pragma unroll
+    for (int u = 0; u < kScanBatch; ++u) {
+      const int a = it0 + 32 * u + lane;
+      eb[u] = a < a1 ? idx[a] : 0;
     }
-    const bool valid = a < a1 && !bad;
-    const int e = valid ? e_raw : 0;
-    const int p = valid ? pool_of(e, L, P, W) : -1 - lane;
-    const unsigned act = __ballot_sync(0xffffffffu, valid);
-    const unsigned peers = __match_any_sync(0xffffffffu, p) & act;
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    int s = -1;
-    if (valid) {
-      s = base_pool[static_cast<long long>(p) * n_chunks + c] + run[p] + rank;
+#pragma unroll
+    for (int u = 0; u < kScanBatch; ++u) {
+      const int a = it0 + 32 * u + lane;
+      const bool ok = a < a1 && eb[u] >= 0 && eb[u] < E;
+      bb[u] = ok ? base_pool[static_cast<long long>(pool_of(eb[u], L, P, W)) * n_chunks + c] : 0;
     }
-    __syncwarp();
-    if (valid && rank == __popc(peers) - 1) run[p] += __popc(peers);  // last of its group
-    if (valid) {
-      const bool sk = s < Cs;
-      slot[2LL * a] = sk ? s : -1;
-      if (sk) atomicAdd(&kept[e], 1);
+#pragma unroll
+    for (int u = 0; u < kScanBatch; ++u) {
+      if (it0 + 32 * u >= a1) break;  // warp-uniform
+      const int a = it0 + 32 * u + lane;
+      const int e_raw = eb[u];
+      const bool bad = a < a1 && (e_raw < 0 || e_raw >= E);
+      if (bad) {
+        atomicCAS(status, 0, MOE_ERR_INVALID_ARG);
+        slot[2LL * a] = -1;
+      }
+      const bool valid = a < a1 && !bad;
+      const int e = valid ? e_raw : 0;
+      const int p = valid ? pool_of(e, L, P, W) : -1 - lane;
+      const unsigned act = __ballot_sync(0xffffffffu, valid);
+      const unsigned peers = __match_any_sync(0xffffffffu, p) & act;
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      int s = -1;
+      if (valid) {
+        s = bb[u] + run[p] + rank;
+      }
+      __syncwarp();
+      if (valid && rank == __popc(peers) - 1) run[p] += __popc(peers);  // last of its group
+      if (valid) {
+        const bool sk = s < Cs;
+        slot[2LL * a] = sk ? s : -1;
+        if (sk) atomicAdd(&kept[e], 1);
+      }
+      __syncwarp();
     }
-    __syncwarp();
   }
   __syncwarp();
   for (int e = lane; e < E; e += 32) cnt_exp[static_cast<long long>(e) * n_chunks + c] = kept[e];
@@ -385,29 +405,48 @@ __global__ void scan_receiver_slots(const int32_t* __restrict__ idx, int A_total
   if (c >= n_chunks) return;
   const int a0 = c * chunk_assign;
   const int a1 = min(A_total, a0 + chunk_assign);
-  for (int it = a0; it < a1; it += 32) {
-    const int a = it + lane;
-    const int e_raw = a < a1 ? idx[a] : 0;
-    const bool valid = a < a1 && e_raw >= 0 && e_raw < E;
-    const int e = valid ? e_raw : 0;
-    const bool sk = valid && slot[2LL * a] >= 0;
-    const int key = sk ? e : -1 - lane;
-    const unsigned act = __ballot_sync(0xffffffffu, sk);
-    const unsigned peers = __match_any_sync(0xffffffffu, key) & act;
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    int r = -1;
-    if (sk) r = base_exp[static_cast<long long>(e) * n_chunks + c] + run[e] + rank;
-    __syncwarp();
-    if (sk && rank == __popc(peers) - 1) run[e] += __popc(peers);
-    if (a < a1 && !valid) slot[2LL * a + 1] = -1;
-    if (valid) {
-      const bool rk = sk && r < Cr;
-      slot[2LL * a + 1] = rk ? r : -1;
-      if (rk) atomicAdd(&stats_kept_e[e], 1);
-      else if (sk) atomicAdd(&stats_dr_e[e], 1);
-      else atomicAdd(&stats_ds_e[e], 1);
+  // as in the sender scan: ids, sender slots and the experts' bases of up to kScanBatch
+  // rows are loaded before the rows are ranked in order
+  for (int it0 = a0; it0 < a1; it0 += 32 * kScanBatch) {
+    int eb[kScanBatch], sb[kScanBatch], bb[kScanBatch];
+#pragma unroll
+    for (int u = 0; u < kScanBatch; ++u) {
+      const int a = it0 + 32 * u + lane;
+      eb[u] = a < a1 ? idx[a] : 0;
+      sb[u] = a < a1 ? slot[2LL * a] : -1;
     }
-    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < kScanBatch; ++u) {
+      const int a = it0 + 32 * u + lane;
+      const bool ok = a < a1 && eb[u] >= 0 && eb[u] < E && sb[u] >= 0;
+      bb[u] = ok ? base_exp[static_cast<long long>(eb[u]) * n_chunks + c] : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < kScanBatch; ++u) {
+      if (it0 + 32 * u >= a1) break;  // warp-uniform
+      const int a = it0 + 32 * u + lane;
+      const int e_raw = eb[u];
+      const bool valid = a < a1 && e_raw >= 0 && e_raw < E;
+      const int e = valid ? e_raw : 0;
+      const bool sk = valid && sb[u] >= 0;
+      const int key = sk ? e : -1 - lane;
+      const unsigned act = __ballot_sync(0xffffffffu, sk);
+      const unsigned peers = __match_any_sync(0xffffffffu, key) & act;
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      int r = -1;
+      if (sk) r = bb[u] + run[e] + rank;
+      __syncwarp();
+      if (sk && rank == __popc(peers) - 1) run[e] += __popc(peers);
+      if (a < a1 && !valid) slot[2LL * a + 1] = -1;
+      if (valid) {
+        const bool rk = sk && r < Cr;
+        slot[2LL * a + 1] = rk ? r : -1;
+        if (rk) atomicAdd(&stats_kept_e[e], 1);
+        else if (sk) atomicAdd(&stats_dr_e[e], 1);
+        else atomicAdd(&stats_ds_e[e], 1);
+      }
+      __syncwarp();
+    }
   }
 }
 
