@@ -102,7 +102,12 @@ def _skewed_idx(T, E, k, seed, skew):
 
 
 @pytest.mark.parametrize("shape,skew", [(synth.TINY, 0.0), (synth.TINY, 1.5), (synth.MID, 0.3),
-                                        (synth.TINY.with_(T=777, top_k=5), 0.8)])
+                                        (synth.TINY.with_(T=777, top_k=5), 0.8),
+                                        # the largest top-k a plan accepts: 32 pool rows per token
+                                        (synth.MoEShape("e96k32", T=333, d_model=192, d_latent=128,
+                                                        n_experts=96, top_k=32, n_dest=8, hidden_routed=128,
+                                                        n_shared=1, hidden_shared=128, seed=45), 0.5)],
+                         ids=["tiny", "tiny_skew", "mid", "ragged_k5", "e96k32"])
 def test_dispatch_bit_exact(M, shape, skew):
     s = shape
     g = O.geometry(s)
