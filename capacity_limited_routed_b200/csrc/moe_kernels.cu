@@ -1015,26 +1015,44 @@ __global__ void undispatch_kernel(const uint16_t* __restrict__ dxe, const float*
       s_row[wib][lane] = e_j >= 0 ? row_of(ra, e_j, slot + 2 * a) : -1;
     }
     __syncwarp();
-    for (int v = lane; v < nvec; v += 64) {
-      const bool two = v + 32 < nvec;
-      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0}, acc2[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-#pragma unroll 4
-      for (int j = 0; j < k; ++j) {
-        const long long rj = s_row[wib][j];
-        if (rj < 0) continue;
-        const uint4* xrow = reinterpret_cast<const uint4*>(dxe + rj * dl);
-        const uint4 a = xrow[v];
-        const uint4 b = two ? xrow[v + 32] : make_uint4(0, 0, 0, 0);
-        acc8(acc, a, 1.0f);
-        acc8(acc2, b, 1.0f);
+    // as in the combine: the matching vectors of up to kCombRows rows are loaded at once,
+    // then summed in j order (rows of dropped assignments are skipped)
+    for (int v0 = lane; v0 < nvec; v0 += 32 * kCombVpl) {
+      float acc[kCombVpl][8];
+#pragma unroll
+      for (int u = 0; u < kCombVpl; ++u)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[u][i] = 0.0f;
+      for (int j0 = 0; j0 < k; j0 += kCombRows) {
+        uint4 val[kCombRows][kCombVpl];
+#pragma unroll
+        for (int jj = 0; jj < kCombRows; ++jj) {
+          const int j = j0 + jj;
+          const long long rj = j < k ? s_row[wib][j] : -1;
+          const uint4* xrow = reinterpret_cast<const uint4*>(dxe + (rj >= 0 ? rj : 0) * dl);
+#pragma unroll
+          for (int u = 0; u < kCombVpl; ++u) {
+            const int v = v0 + 32 * u;
+            val[jj][u] = (rj >= 0 && v < nvec) ? xrow[v] : make_uint4(0, 0, 0, 0);
+          }
+        }
+#pragma unroll
+        for (int jj = 0; jj < kCombRows; ++jj) {
+          const int j = j0 + jj;
+          if (j >= k) break;
+          if (s_row[wib][j] < 0) continue;
+#pragma unroll
+          for (int u = 0; u < kCombVpl; ++u) acc8(acc[u], val[jj][u], 1.0f);
+        }
       }
-      float4* o = reinterpret_cast<float4*>(dz + static_cast<long long>(t) * dl + 8 * v);
-      o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
-      if (two) {
-        float4* o2 = reinterpret_cast<float4*>(dz + static_cast<long long>(t) * dl + 8 * (v + 32));
-        o2[0] = make_float4(acc2[0], acc2[1], acc2[2], acc2[3]);
-        o2[1] = make_float4(acc2[4], acc2[5], acc2[6], acc2[7]);
+#pragma unroll
+      for (int u = 0; u < kCombVpl; ++u) {
+        const int v = v0 + 32 * u;
+        if (v < nvec) {
+          float4* o = reinterpret_cast<float4*>(dz + static_cast<long long>(t) * dl + 8 * v);
+          o[0] = make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
+          o[1] = make_float4(acc[u][4], acc[u][5], acc[u][6], acc[u][7]);
+        }
       }
     }
     // softmax backward: dl_j = g_j (dg_j - sum_i g_i dg_i)
