@@ -104,7 +104,9 @@ struct Cfg {
   static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * kBK * 2;  // a pair CTA holds half of B
   static constexpr int kStage = kABytes + kBBytes;
   static constexpr int kStages = WRITE_BOUND ? kWbStages : ((BN == 256 && !PAIR) ? 4 : 6);
-  static constexpr int kTmemCols = 2 * BN;
+  // two accumulators; a 192-column one sits at a 256-column stride (allocations are powers of 2)
+  static constexpr int kAccStride = BN <= 128 ? BN : 256;
+  static constexpr int kTmemCols = 2 * kAccStride;
   static constexpr int kBufs = WRITE_BOUND ? kWbBufs : 1;  // staging buffers per epilogue warp
   static constexpr int kEpiWarps = Roles<WRITE_BOUND>::kEpiWarps;
   // a buffer holds 32 rows x 128 bytes (float32 / bf16 outputs); the forward SwiGLU
@@ -399,7 +401,7 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::kAccStride);
         for (int kb = 0; kb < kb_total; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_v)) {
             ok = false;
@@ -539,7 +541,7 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t tbase = tmem_base + lane_off + static_cast<uint32_t>(acc * BN);
+      const uint32_t tbase = tmem_base + lane_off + static_cast<uint32_t>(acc * C::kAccStride);
       bool released = false;  // accumulator handed back to the MMA warp early
 
       if constexpr (EPI == EPI_SWIGLU) {
@@ -664,8 +666,9 @@ __global__ void __launch_bounds__(Roles<A_MN && B_MN>::kThreads, 1)
         // is released as soon as the whole tile is in registers.  With an addend, each
         // 64-column piece gets its float32 addend before rounding to bf16.
         constexpr int kChunk = (EPI == EPI_F32) ? 32 : 64;  // columns per 128-byte row
-        // columns per TMEM wait (the addend's registers leave room for 64)
-        constexpr int kSpan = (EPI == EPI_BF16_ADD_F32) ? 64 : 128;
+        // columns per TMEM wait (the addend's registers leave room for 64; a 192-column tile
+        // drains in three spans)
+        constexpr int kSpan = (EPI == EPI_BF16_ADD_F32 || BN % 128 != 0) ? 64 : 128;
         const int row0 = mbase + q * 32;
 #pragma unroll 1
         for (int half = 0; half < BN; half += kSpan) {
@@ -1273,7 +1276,10 @@ int device_sm_count() {
 
 moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
   if (a.M <= 0 || a.N <= 0 || a.groups <= 0) return MOE_OK;
-  if (a.bn != 128 && a.bn != 256) return fail(MOE_ERR_UNSUPPORTED, "gemm tile width must be 128 or 256");
+  if (a.bn != 128 && a.bn != 256 &&
+      !(a.bn == 192 && a.pair && !a.a_mn && !a.b_mn && a.epi == EPI_F32 && a.nseg == 1))
+    return fail(MOE_ERR_UNSUPPORTED,
+                "gemm tile width must be 128 or 256 (192: CTA pairs, K-major operands, float32 out)");
   if (a.groups > kMaxGroups) return fail(MOE_ERR_UNSUPPORTED, "too many gemm groups");
   if (a.nseg < 1 || a.nseg > 3) return fail(MOE_ERR_INVALID_ARG, "gemm needs 1..3 K segments");
   if (a.ragged != 0 && a.group_rows == nullptr) return fail(MOE_ERR_INVALID_ARG, "ragged gemm needs group rows");
@@ -1438,6 +1444,8 @@ moe_status_t gemm_run(const GemmArgs& a, cudaStream_t st) {
   MOE_GEMM_CASE(256, false, false, EPI_SWIGLU)
   MOE_GEMM_CASE(128, false, false, EPI_F32)
   MOE_GEMM_CASE(256, false, false, EPI_F32)
+  if (a.bn == 192 && !a.a_mn && !a.b_mn && a.epi == EPI_F32 && a.pair)  // router logits, E % 192 == 0
+    return launch_instance<192, false, false, EPI_F32, true>(maps, kp, tiles, st);
   // backward: dgrad (B stored [K][N]); dx in f32; wgrad (both stored [K][.]) in f32
   MOE_GEMM_CASE(256, false, true, EPI_BF16)
   MOE_GEMM_CASE(256, false, true, EPI_SWIGLU_BWD)

@@ -401,6 +401,11 @@ void pack_groups(const Geo& g, GemmArgs& a, const int32_t* exp_off) {
   if (a.ragged == 1) a.M = static_cast<int>(g.exp_rows);  // local rows never reach it
 }
 
+// Column tile of the router-logit GEMM (256-row pair tiles, N = E): 192 when it divides E
+// and there are enough columns to matter, which turns E = 384 into two column tiles of a
+// denser tile (128 pair tiles on 74 pairs) instead of three of 128.
+int router_tile_cols(int E) { return (E >= 384 && E % 192 == 0) ? 192 : 128; }
+
 // dW_r = dlogits^T z over the T tokens.  With K = T long and few output tiles (E x d_latent:
 // 2 x 12 pair tiles at full width for 74 pairs) the tokens are split into S equal slices,
 // computed as S groups of one launch into float32 partials in `scratch` (when it holds them)
@@ -912,7 +917,7 @@ moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const uint16_t* x
     ProfScope ps("fwd.router", st);
     GemmArgs a;
     a.pair = true;  // dense rows: 256-row tiles on CTA pairs
-    a.bn = 128;
+    a.bn = router_tile_cols(p->E);
     a.epi = EPI_F32;
     a.M = g.T;
     a.N = p->E;
@@ -1379,7 +1384,7 @@ moe_status_t moe_ep_forward_send(moe_plan_t p, const moe_weights_t* w, const uin
       ProfScope ps("fwd.router", st);
       GemmArgs a;
       a.pair = true;
-      a.bn = 128;
+      a.bn = router_tile_cols(p->E);
       a.epi = EPI_F32;
       a.M = g.T;
       a.N = p->E;
