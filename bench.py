@@ -41,8 +41,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # captured ones, and as null once they change.
 NCU_TRAFFIC = {
     "bwd.experts_wgrad_gate_up": {
-        "sources_sha256": "0fb047ffc41bdb886f8f2b6b3aa3abd004e4aea0b5ea17ef033e4577af29434a",
-        "dram_bytes": 1915109632, "experts": 24, "tokens": 1024, "d_latent": 3072, "hidden_routed": 3072,
+        "sources_sha256": "4591362332d8b9b20415fee24dce1562ba2fc3cae0b03bb95434ff18b3dd29df",
+        "dram_bytes": 1915889152, "experts": 24, "tokens": 1024, "d_latent": 3072, "hidden_routed": 3072,
     },
 }
 KERNEL_SOURCES = ("gemm_sm100.cu", "ptx.cuh")  # the GEMM kernels and the PTX they use
